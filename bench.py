@@ -1,0 +1,345 @@
+"""Benchmark of the fused decode-GEMM path on one Llama-3.1-8B-shaped gate
+projection W[14336, 4096] (BF16, N(0, 0.02) with a 0.1% t_3 tail) at batch 1.
+
+One step = the whole per-call hot path over one batch:
+  uw_decode_full, uw_decode_exponent, uw_transcode_palette, and
+  uw_gemm through the four pipelines (full, exponent, transcode, direct
+  palette) with x[1, 4096].
+value = effective BF16 weight bytes delivered per second over the step
+(7 x 2*N*K bytes per step / step time), whole job (all ranks).
+
+Inputs larger than L2: four compressed copies of W (~110 MB each) are
+rotated so that an op never finds its inputs left in L2 by the previous use.
+--impl reference times the CPU oracle (plain C) on a bounded row sample of the
+same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused decode-GEMM eff. weight GB/s & TFLOP/s, % roofline, batch 1–1024"
+N_W, K_W, M_X = 14336, 4096, 1
+OPS = ["decode_full", "decode_exponent", "transcode", "gemm_full", "gemm_exponent", "gemm_transcode",
+       "gemm_direct_palette"]
+WORKLOAD = "gate projection W[14336,4096] bf16 N(0,0.02)+0.1% t3 tail, x[1,4096]; decode x3 + 4 pipelines"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        except Exception:
+            rows = []
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = sorted(float(r[1]) for r in rows)
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return dist, int(os.environ["RANK"]), ws, int(os.environ.get("LOCAL_RANK", "0"))
+    return None, 0, 1, 0
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the reference arm)
+# ---------------------------------------------------------------------------
+_sample_cache = {}
+
+
+def oracle_step_sample(rows: int = 256):
+    """Runs the oracle's version of one step on `rows` rows of the workload:
+    Huffman decode -> full / exponent / transcode, then the reference product
+    for each of the four pipelines.  Returns (seconds, weights processed)."""
+    import synthetic as S
+    from oracle import oracle as O
+    if rows not in _sample_cache:
+        _sample_cache[rows] = S.gate_projection()[:rows].copy()
+    W = _sample_cache[rows]
+    x = S.activations(M_X, K_W, seed=1 + S.X_SEED_OFFSET)
+    b = O.compress(W)
+    t0 = time.perf_counter()
+    Wd = O.decode_full(b)                 # decode_full
+    O.decode_exponent(b)                  # decode_exponent
+    O.transcode(b)                        # transcode
+    for _ in range(4):                    # four pipelines: decode form + product
+        O.decode_exponent(b)
+        O.gemm(x, Wd, "f32")
+    dt = time.perf_counter() - t0
+    return dt, W.size
+
+
+def cpu_baseline(rows: int = 256):
+    dt, nw = oracle_step_sample(rows)
+    eff = len(OPS) * 2.0 * nw / dt / 1e9
+    return {"value": eff, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of 14336 rows ({nw} weights), one step: decode x3 + 4 x (decode + GEMV), "
+                      f"single thread, {dt:.3f} s"}
+
+
+def run_reference(args):
+    dist, rank, world, _ = _dist()
+    if rank != 0:
+        return
+    rows = 256
+    for _ in range(args.warmup):
+        oracle_step_sample(rows)
+    tot = 0.0
+    nw = 0
+    for _ in range(args.steps):
+        dt, nw = oracle_step_sample(rows)
+        tot += dt
+    value = len(OPS) * 2.0 * nw * args.steps / tot / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "oracle_rows_per_step": rows, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} of 14336 rows per step, single thread"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import decode_gemm_bf16_b200 as uw
+    import synthetic as S
+
+    dist, rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_peak, tc_peak, peak_kind = _peaks()
+
+    W = S.gate_projection()
+    x = S.activations(M_X, K_W, seed=1 + S.X_SEED_OFFSET)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+    copies = [uw.uw_compress(Wd) for _ in range(4)]
+    del Wd
+    info = copies[0].info
+    n = N_W * K_W
+    xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    wsb = max(uw.uw_gemm_workspace(copies[0], M_X, p) for p in uw.PIPELINES)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    out_full = torch.empty(N_W, K_W, dtype=torch.bfloat16, device=dev)
+    out_e = torch.empty(n, dtype=torch.uint8, device=dev)
+    out_i = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    Ys = [torch.empty(M_X, N_W, dtype=torch.bfloat16, device=dev) for _ in range(4)]
+    stream = torch.cuda.current_stream()
+
+    def op(k, blob, xin):
+        if k == 0:
+            uw.uw_decode_full(blob, out_full)
+        elif k == 1:
+            uw.uw_decode_exponent(blob, out_e)
+        elif k == 2:
+            uw.uw_transcode_palette(blob, out_i)
+        else:
+            uw.uw_gemm(xin, blob, k - 3, out=Ys[k - 3], ws=ws)
+
+    nops = len(OPS)
+    ctr = [0]
+
+    def step(xin, ev=None):
+        for k in range(nops):
+            blob = copies[ctr[0] % len(copies)]
+            ctr[0] += 1
+            if ev is not None:
+                ev[k][0].record(stream)
+            op(k, blob, xin)
+            if ev is not None:
+                ev[k][1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step(xd)
+    torch.cuda.synchronize()
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nops)]
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(xd, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if dist:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    per_op_ms = [sum(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(args.steps)) / args.steps
+                 for k in range(nops)]
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    # ---- end to end: host x (pinned) -> device, the step, Y -> host (pinned)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = [torch.empty(M_X, N_W, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    xdev = torch.empty_like(xd)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        xdev.copy_(xh, non_blocking=True)
+        step(xdev)
+        for j in range(4):
+            yh[j].copy_(Ys[j], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    # ---- numbers
+    eff_bytes_step = nops * 2.0 * n
+    value = world * eff_bytes_step * args.steps / (ms / 1e3) / 1e9
+    e2e = world * eff_bytes_step * args.steps / (e2e_ms / 1e3) / 1e9
+    sec = info["sections"]
+    stream_b = sec["stream"][1] + sec["chunk_off"][1] + sec["seg_rel"][1]
+    vstore = sec["vbits"][1] + sec["vpre"][1] + sec["vexp"][1]
+    xb, yb = M_X * K_W * 2, M_X * N_W * 2
+    # algorithmic bytes per launch of each single-kernel op (what must move)
+    alg = {
+        "decode_full": stream_b + vstore + n + 2 * n,
+        "decode_exponent": stream_b + vstore + n,
+        "transcode": stream_b + n // 2,
+        "gemm_direct_palette": n + n // 2 + vstore + sec["vcol"][1] + xb + yb,
+    }
+    kernel_of = {"decode_full": "k_decode<full>", "decode_exponent": "k_decode<exponent>",
+                 "transcode": "k_decode<transcode>", "gemm_direct_palette": "k_gemm<palette>"}
+    breakdown = {}
+    for k, name in enumerate(OPS):
+        d = {"us": 1e3 * per_op_ms[k], "eff_weight_gbs": 2.0 * n / (per_op_ms[k] / 1e3) / 1e9,
+             "tflops": (2.0 * M_X * n / (per_op_ms[k] / 1e3) / 1e12) if name.startswith("gemm") else None}
+        if name in alg:
+            d["alg_bytes"] = alg[name]
+            d["alg_gbs"] = alg[name] / (per_op_ms[k] / 1e3) / 1e9
+            d["hbm_frac"] = d["alg_gbs"] / hbm_peak
+        breakdown[name] = d
+    # dominant single-kernel op: the decode_full kernel also runs inside the
+    # full pipeline, the palette GEMM inside the transcode pipeline
+    share = {"decode_full": per_op_ms[0] * 2, "decode_exponent": per_op_ms[1] * 2,
+             "transcode": per_op_ms[2] * 2, "gemm_direct_palette": per_op_ms[6] * 2}
+    dom = max(share, key=share.get)
+    dom_ms = per_op_ms[OPS.index(dom)]
+    achieved = alg[dom] / (dom_ms / 1e3) / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        try:
+            traffic = json.load(open(tp)).get(kernel_of[dom])
+        except Exception:
+            traffic = None
+    launches_per_step = 3 + 2 + 2 + 2 + 1
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_X, "N": N_W, "K": K_W, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: 4 rotating compressed copies",
+                   "ratio_huffman_form": info["bytes_huffman_form"] / (2 * n),
+                   "ratio_palette_form": info["bytes_palette_form"] / (2 * n),
+                   "mean_code_bits": info["mean_code_len"]},
+        "roofline": {"bound": "hbm", "kernel": kernel_of[dom], "achieved": achieved, "peak": hbm_peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic},
+        "breakdown": breakdown,
+        "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": xb, "d2h_bytes_per_step": 4 * yb},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

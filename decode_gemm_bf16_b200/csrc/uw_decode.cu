@@ -1,0 +1,223 @@
+// uw_decode.cu -- HBM-to-HBM Huffman decoders of the Unweight format.
+//
+// "Cloudflare推出Unweight無損壓縮系統" (easyvibecoding.app), §四種執行管道:
+//   full decode       -> the original BF16 matrix (writes the most bytes);
+//   exponent decode   -> the exponent bytes only (half the traffic);
+//   palette transcode -> 4-bit palette indices (a quarter).
+// §解壓與運算資源共享 gives the decoder a 16 KB Huffman table in shared
+// memory; here that table is a 4096-entry multi-symbol table (12-bit window ->
+// up to four symbols).
+//
+// Work split: a warp owns 32 consecutive 256-symbol segments (8192 weights).
+// Phase 1: lane l decodes segment l from its own start bit (chunk offset +
+// segment offset) into 32 words of packed nibbles in shared memory (rotated
+// by the lane index so that all lanes hit different banks).  Phase 2: the
+// warp walks its 8192 outputs in order, maps nibbles to exponents through the
+// palette (byte permutes), patches verbatim groups, merges the sign+mantissa
+// bytes and stores coalesced 16-byte vectors.
+#include "uw_device.cuh"
+#include "uw_internal.h"
+
+namespace uw {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTaskElems = 32 * kSeg;          // 8192 weights per warp task
+constexpr size_t kDecodeSmem = kLutSize * 4 + kWarps * 32 * 32 * 4;
+
+struct DecodeParams {
+    const uint32_t* stream;
+    int64_t nwords;
+    const uint64_t* chunk_off;
+    const uint16_t* seg_rel;
+    const uint32_t* lut;
+    const uint8_t* sm;
+    const uint32_t* vbits;
+    const uint32_t* vpre;
+    const uint8_t* vexp;
+    uint32_t pal[4];
+    int64_t n;       // weights
+    int64_t nseg;
+    void* out;
+};
+
+__device__ __forceinline__ uint32_t ld_word(const uint32_t* s, int64_t i, int64_t nwords) {
+    return i < nwords ? __ldg(&s[i]) : 0u;
+}
+
+// Decodes segment `seg` (nsym symbols, a multiple of 64) into `row`: word k of
+// the segment (8 nibbles) is stored at row[(k + rot) & 31].
+__device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint32_t* lut,
+                                               int64_t seg, int nsym, uint32_t* row, int rot) {
+    uint64_t bitpos = __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
+    int64_t wi = (int64_t)(bitpos >> 5);
+    if (wi + 1 >= p.nwords) {
+        raise_status(UW_ERR_DEVICE);
+        return;
+    }
+    uint32_t sh = (uint32_t)(bitpos & 31u);
+    uint64_t buf = (((uint64_t)__ldg(&p.stream[wi]) << 32) | __ldg(&p.stream[wi + 1])) << sh;
+    int avail = 64 - (int)sh;
+    int64_t nxt = wi + 2;
+    uint64_t acc = 0;
+    int accn = 0, k = 0, produced = 0;
+    const int words = nsym >> 3;
+    while (produced < nsym) {
+        if (avail < 32) {
+            buf |= (uint64_t)ld_word(p.stream, nxt++, p.nwords) << (32 - avail);
+            avail += 32;
+        }
+        uint32_t ent = lut[buf >> 52];
+        uint32_t ns = lut_nsym(ent), nb = lut_bits(ent);
+        if (ns == 0) {
+            raise_status(UW_ERR_DEVICE);
+            return;
+        }
+        acc |= (uint64_t)(ent & 0xFFFFu) << accn;
+        accn += 4 * (int)ns;
+        produced += (int)ns;
+        buf <<= nb;
+        avail -= (int)nb;
+        if (accn >= 32) {
+            if (k < words) row[(k + rot) & 31] = (uint32_t)acc;
+            k++;
+            acc >>= 32;
+            accn -= 32;
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    uint32_t* stage = smem + kLutSize;
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(p.lut);
+        uint4* dst = reinterpret_cast<uint4*>(lut);
+        for (int i = threadIdx.x; i < kLutSize / 4; i += kThreads) dst[i] = __ldg(&src[i]);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* st = stage + warp * 1024;
+    const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
+    const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
+
+    for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < ntasks;
+         task += (int64_t)gridDim.x * kWarps) {
+        const int64_t base = task * kTaskElems;
+        // ---- phase 1: one segment per lane
+        {
+            int64_t seg = task * 32 + lane;
+            int64_t e0 = seg * kSeg;
+            int64_t left = p.n - e0;
+            int nsym = left <= 0 ? 0 : (left < kSeg ? (int)left : kSeg);
+            if (nsym > 0) decode_segment(p, lut, seg, nsym, st + lane * 32, lane);
+        }
+        __syncwarp();
+        // ---- phase 2: ordered, coalesced output
+        if (MODE == kDecodeTranscode) {
+            // lane -> segment 4*it + lane/8, words 4*(lane%8) .. +3 (32 nibbles)
+            uint4* out = reinterpret_cast<uint4*>(p.out);
+#pragma unroll 2
+            for (int it = 0; it < 8; it++) {
+                int j = 4 * it + (lane >> 3);
+                int k0 = 4 * (lane & 7);
+                int64_t e = base + (int64_t)j * kSeg + k0 * 8;
+                if (e < p.n) {
+                    const uint32_t* r = st + j * 32;
+                    uint4 v;
+                    v.x = r[(k0 + 0 + j) & 31];
+                    v.y = r[(k0 + 1 + j) & 31];
+                    v.z = r[(k0 + 2 + j) & 31];
+                    v.w = r[(k0 + 3 + j) & 31];
+                    out[e >> 5] = v;
+                }
+            }
+        } else {
+            // lane -> segment 2*it + lane/16, words 2*(lane%16), +1 (16 weights)
+#pragma unroll 2
+            for (int it = 0; it < 16; it++) {
+                int j = 2 * it + (lane >> 4);
+                int k0 = 2 * (lane & 15);
+                int64_t e = base + (int64_t)j * kSeg + k0 * 8;
+                if (e >= p.n) continue;
+                const uint32_t* r = st + j * 32;
+                uint32_t w0 = r[(k0 + j) & 31], w1 = r[(k0 + 1 + j) & 31];
+                uint4 ex;
+                int64_t g = e >> 6;
+                uint32_t vw = __ldg(&p.vbits[g >> 5]);
+                if ((vw >> (g & 31)) & 1u) {
+                    int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
+                    ex = __ldg(reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + (e & 63)));
+                } else {
+                    ex.x = palette4(w0, P0, P1, P2, P3);
+                    ex.y = palette4(w0 >> 16, P0, P1, P2, P3);
+                    ex.z = palette4(w1, P0, P1, P2, P3);
+                    ex.w = palette4(w1 >> 16, P0, P1, P2, P3);
+                }
+                if (MODE == kDecodeExponent) {
+                    reinterpret_cast<uint4*>(p.out)[e >> 4] = ex;
+                } else {
+                    uint4 s = __ldg(reinterpret_cast<const uint4*>(p.sm + e));
+                    uint2 a = merge4(ex.x, s.x), b = merge4(ex.y, s.y);
+                    uint2 c = merge4(ex.z, s.z), d = merge4(ex.w, s.w);
+                    uint4* out = reinterpret_cast<uint4*>(p.out) + (e >> 3);
+                    out[0] = make_uint4(a.x, a.y, b.x, b.y);
+                    out[1] = make_uint4(c.x, c.y, d.x, d.y);
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+int decode_ctas_per_sm() { return 4; }
+
+cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s) {
+    DecodeParams p;
+    p.stream = (const uint32_t*)b->sec(UW_SEC_STREAM);
+    p.nwords = b->nwords;
+    p.chunk_off = (const uint64_t*)b->sec(UW_SEC_CHUNK_OFF);
+    p.seg_rel = (const uint16_t*)b->sec(UW_SEC_SEG_REL);
+    p.lut = (const uint32_t*)b->sec(UW_SEC_LUT);
+    p.sm = b->sec(UW_SEC_SM);
+    p.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
+    p.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
+    p.vexp = b->sec(UW_SEC_VEXP);
+    for (int i = 0; i < 4; i++)
+        p.pal[i] = (uint32_t)b->palette[4 * i] | ((uint32_t)b->palette[4 * i + 1] << 8) |
+                   ((uint32_t)b->palette[4 * i + 2] << 16) | ((uint32_t)b->palette[4 * i + 3] << 24);
+    p.n = b->geo.n;
+    p.nseg = b->geo.nseg;
+    p.out = out;
+    int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
+    int64_t need = (ntasks + kWarps - 1) / kWarps;
+    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * decode_ctas_per_sm();
+    if (grid > need) grid = (int)need;
+    if (grid < 1) grid = 1;
+    cudaError_t e = cudaSuccess;
+    switch (mode) {
+        case kDecodeFull:
+            e = cudaFuncSetAttribute(k_decode<kDecodeFull>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+            if (e == cudaSuccess) k_decode<kDecodeFull><<<grid, kThreads, kDecodeSmem, s>>>(p);
+            break;
+        case kDecodeExponent:
+            e = cudaFuncSetAttribute(k_decode<kDecodeExponent>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+            if (e == cudaSuccess) k_decode<kDecodeExponent><<<grid, kThreads, kDecodeSmem, s>>>(p);
+            break;
+        default:
+            e = cudaFuncSetAttribute(k_decode<kDecodeTranscode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+            if (e == cudaSuccess) k_decode<kDecodeTranscode><<<grid, kThreads, kDecodeSmem, s>>>(p);
+            break;
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+int decode_status_take() { return unit_status_take(); }
+
+}  // namespace uw

@@ -1,0 +1,545 @@
+// uw_gemm.cu -- Y[M,N] = X[M,K] . W[N,K]^T on the 5th-generation tensor cores,
+// with W either plain BF16 or rebuilt on chip from its compressed form.
+//
+// "Cloudflare推出Unweight無損壓縮系統" (easyvibecoding.app),
+// §重建矩陣乘法核心運作: the reconstructive matmul loads compressed data from
+// HBM, rebuilds BF16 in shared memory and feeds the tensor cores directly, so
+// the rebuilt weights never go back to HBM.  A producer role stages the
+// sign+mantissa bytes, the exponent bytes or palette indices and the
+// verbatim flags into a ring of shared-memory buffers with TMA, ahead of the
+// consumers; consumers merge exponent and sign+mantissa into BF16 tiles.
+// §四種執行管道: exponent source (after the exponent decoder), palette source
+// (after the transcoder, or straight from the stored index plane).
+//
+// B200 design (not the Hopper one of the page):
+//   * swap-AB: the weight tile is the MMA's A operand (M = 128 rows of W), the
+//     activations are B (N = batch tile MG <= 256), the accumulator lives in
+//     tensor memory (TMEM) -- no register-file accumulators, so shared memory
+//     holds only the stage ring;
+//   * warp roles: warps 0-3 epilogue (TMEM lanes 32w..32w+31), warp 4 TMA
+//     producer, warp 5 allocates TMEM and issues tcgen05.mma (one thread),
+//     warps 6-13 rebuild BF16 tiles in the 128-byte swizzled K-major layout the
+//     MMA descriptor expects;
+//   * stream-K: the (tile, 64-wide k step) iterations are split evenly over one
+//     CTA per SM; tiles cut between CTAs are finished by the last CTA to
+//     arrive, per output row, summing fp32 partials in CTA order
+//     (deterministic).  This covers batch 1-64 (HBM bound, K split) and the
+//     long-K down projection with the same kernel;
+//   * every wait is bounded (globaltimer deadline); on expiry the CTA raises
+//     UW_ERR_TIMEOUT, drains its own TMA and MMA work, frees TMEM and exits.
+#include <cstdio>
+#include <cstdlib>
+
+#include "uw_device.cuh"
+#include "uw_internal.h"
+
+namespace uw {
+namespace {
+
+constexpr int kBlockN = 128;   // weight rows per tile (MMA M)
+constexpr int kBlockK = 64;    // k per stage: one 128-byte swizzle row of BF16
+constexpr int kEpiWarps = 4;
+constexpr int kProdWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kReconWarp0 = 6;
+constexpr int kReconWarps = 8;
+constexpr int kMaxStages = 8;
+constexpr int kThreadsDense = 6 * 32;
+constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
+constexpr uint32_t kTileA = kBlockN * kBlockK * 2;       // 16 KB rebuilt / loaded BF16 tile
+constexpr uint32_t kTileSM = kBlockN * kBlockK;          //  8 KB sign+mantissa
+constexpr uint32_t kTileE = kBlockN * kBlockK;           //  8 KB exponents
+constexpr uint32_t kTileIdx = kBlockN * kBlockK / 2;     //  4 KB palette indices
+constexpr uint32_t kTileV = 16;                          // 128 verbatim flags
+
+struct GemmParams {
+    int64_t M, N, K, KG;
+    int MG, m_tiles, n_tiles, kt_count, P, stages;
+    int64_t total_iters;
+    uint32_t stage_bytes, off_b, off_sm, off_s2, off_v, tx_bytes;
+    const uint32_t* vbits;
+    const uint32_t* vpre;
+    const uint8_t* vexp;
+    uint32_t pal[4];
+    void* Y;
+    int out_f32;
+    float* partial;     // [2P][MG][128]
+    int* counters;      // [tiles][128]
+    uint64_t timeout_ns;
+};
+
+__host__ __device__ __forceinline__ int64_t iter_begin(int64_t b, int64_t total, int64_t P) {
+    return b * total / P;
+}
+// CTA that processes iteration i (the last b with iter_begin(b) <= i).
+__host__ __device__ __forceinline__ int64_t iter_owner(int64_t i, int64_t total, int64_t P) {
+    return ((i + 1) * P - 1) / total;
+}
+
+struct Segment {
+    int64_t tile;
+    int kt0, kt1;
+    bool first;   // first segment of this CTA's range
+};
+
+// Walks the segments of CTA b: [begin, end) cut at tile boundaries.
+struct SegWalker {
+    int64_t it, end;
+    int kt_count;
+    bool started = false;
+    __device__ SegWalker(int64_t b, const GemmParams& p)
+        : it(iter_begin(b, p.total_iters, p.P)), end(iter_begin(b + 1, p.total_iters, p.P)),
+          kt_count(p.kt_count) {}
+    __device__ bool next(Segment& s) {
+        if (it >= end) return false;
+        s.tile = it / kt_count;
+        s.kt0 = (int)(it % kt_count);
+        int64_t rest = end - it;
+        int64_t hi = (int64_t)s.kt0 + rest;
+        s.kt1 = (int)(hi < kt_count ? hi : kt_count);
+        s.first = !started;
+        started = true;
+        it += s.kt1 - s.kt0;
+        return true;
+    }
+};
+
+template <int SRC>
+__device__ __forceinline__ void reconstruct_tile(const GemmParams& p, uint8_t* stage, int64_t n0,
+                                                 int kt, int t /*0..255*/) {
+    uint8_t* A = stage;
+    const uint8_t* SM = stage + p.off_sm;
+    const uint8_t* S2 = stage + p.off_s2;
+    uint4 vc = make_uint4(0, 0, 0, 0);
+    if (SRC == kSrcPalette) vc = *reinterpret_cast<const uint4*>(stage + p.off_v);
+    const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int r = (t >> 3) + 32 * i;   // tile row
+        const int c = t & 7;               // 8-weight chunk within the 64-wide row
+        uint2 s = *reinterpret_cast<const uint2*>(SM + r * 64 + c * 8);
+        uint32_t e0, e1;
+        if (SRC == kSrcExponent) {
+            uint2 e = *reinterpret_cast<const uint2*>(S2 + r * 64 + c * 8);
+            e0 = e.x;
+            e1 = e.y;
+        } else {
+            uint32_t vw = i == 0 ? vc.x : i == 1 ? vc.y : i == 2 ? vc.z : vc.w;
+            if ((vw >> (r & 31)) & 1u) {
+                // verbatim group: raw exponents from the verbatim store
+                int64_t g = (n0 + r) * p.KG + kt;
+                uint32_t w = __ldg(&p.vbits[g >> 5]);
+                int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
+                uint2 e = __ldg(reinterpret_cast<const uint2*>(p.vexp + rank * kGroup + c * 8));
+                e0 = e.x;
+                e1 = e.y;
+            } else {
+                uint32_t ix = *reinterpret_cast<const uint32_t*>(S2 + r * 32 + c * 4);
+                e0 = palette4(ix, P0, P1, P2, P3);
+                e1 = palette4(ix >> 16, P0, P1, P2, P3);
+            }
+        }
+        uint2 a = merge4(e0, s.x), b = merge4(e1, s.y);
+        *reinterpret_cast<uint4*>(A + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+    }
+}
+
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRecon, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+           const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+           const GemmParams p) {
+    constexpr bool kRecon = SRC != kSrcDense;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.stages;
+    uint8_t* ctrl = smem + (size_t)S * p.stage_bytes;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
+    uint64_t* recon_bar = full_bar + kMaxStages;
+    uint64_t* empty_bar = recon_bar + kMaxStages;
+    uint64_t* accf_bar = empty_bar + kMaxStages;
+    uint64_t* acce_bar = accf_bar + 1;
+    uint64_t* final_bar = acce_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t tmem_cols = p.MG <= 32 ? 32u : p.MG <= 64 ? 64u : p.MG <= 128 ? 128u : 256u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&recon_bar[s]), kReconWarps);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        mbar_init(smem_u32(accf_bar), 1);
+        mbar_init(smem_u32(acce_bar), kEpiWarps);
+        mbar_init(smem_u32(final_bar), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+        tmem_relinquish();
+    }
+    if (warp == kProdWarp && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_a);
+        if (kRecon) {
+            tma_prefetch_desc(&tm_s2);
+            if (SRC == kSrcPalette) tma_prefetch_desc(&tm_v);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tmem_slot;
+    const uint32_t smem_base = smem_u32(smem);
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            SegWalker wk(blockIdx.x, p);
+            Segment sg;
+            int64_t q = 0;
+            bool ok = true;
+            while (ok && wk.next(sg)) {
+                const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
+                for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
+                    const int s = (int)(q % S);
+                    const uint32_t ph = (uint32_t)((q / S) & 1);
+                    if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
+                    const uint32_t st = smem_base + s * p.stage_bytes;
+                    const uint32_t fb = smem_u32(&full_bar[s]);
+                    mbar_arrive_expect_tx(fb, p.tx_bytes);
+                    tma_load_2d(st + p.off_b, &tm_x, kt * kBlockK, m_tile * p.MG, fb);
+                    if (SRC == kSrcDense) {
+                        tma_load_2d(st, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
+                    } else {
+                        tma_load_2d(st + p.off_sm, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
+                        if (SRC == kSrcExponent)
+                            tma_load_2d(st + p.off_s2, &tm_s2, kt * kBlockK, n_tile * kBlockN, fb);
+                        else {
+                            tma_load_2d(st + p.off_s2, &tm_s2, kt * (kBlockK / 2), n_tile * kBlockN, fb);
+                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt, fb);
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: every load already issued must land before the CTA exits
+                for (int64_t qq = q - S < 0 ? 0 : q - S; qq < q; qq++)
+                    mbar_wait(smem_u32(&full_bar[qq % S]), (uint32_t)((qq / S) & 1), p.timeout_ns, nullptr);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = mma_idesc_bf16(kBlockN, p.MG);
+            SegWalker wk(blockIdx.x, p);
+            Segment sg;
+            int64_t q = 0;
+            int j = 0;
+            bool ok = true;
+            while (ok && wk.next(sg)) {
+                if (!mbar_wait(smem_u32(acce_bar), (uint32_t)(j & 1) ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
+                    const int s = (int)(q % S);
+                    const uint32_t ph = (uint32_t)((q / S) & 1);
+                    const uint32_t wb = kRecon ? smem_u32(&recon_bar[s]) : smem_u32(&full_bar[s]);
+                    if (!mbar_wait(wb, ph, p.timeout_ns, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_base + s * p.stage_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; kk++) {
+                        uint64_t ad = sw128_desc(st + kk * 32);
+                        uint64_t bd = sw128_desc(st + p.off_b + kk * 32);
+                        tc_mma(tacc, ad, bd, idesc, (kt > sg.kt0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(smem_u32(&empty_bar[s]));
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(accf_bar));
+                j++;
+            }
+            // drain the tensor core before TMEM is released
+            tc_commit(smem_u32(final_bar));
+            mbar_wait(smem_u32(final_bar), 0, p.timeout_ns, nullptr);
+        }
+        __syncwarp();
+    } else if (kRecon && warp >= kReconWarp0) {
+        // ------------------------------------------------------------ reconstruct
+        const int t = threadIdx.x - kReconWarp0 * 32;
+        SegWalker wk(blockIdx.x, p);
+        Segment sg;
+        int64_t q = 0;
+        bool ok = true;
+        while (ok && wk.next(sg)) {
+            const int64_t n0 = (sg.tile / p.m_tiles) * kBlockN;
+            for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
+                const int s = (int)(q % S);
+                const uint32_t ph = (uint32_t)((q / S) & 1);
+                if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, abort_flag)) { ok = false; break; }
+                reconstruct_tile<SRC>(p, smem + (size_t)s * p.stage_bytes, n0, kt, t);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&recon_bar[s]));
+            }
+        }
+    } else if (warp < kEpiWarps) {
+        // ------------------------------------------------------------ epilogue
+        SegWalker wk(blockIdx.x, p);
+        Segment sg;
+        int j = 0;
+        const int r = warp * 32 + lane;
+        while (wk.next(sg)) {
+            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag)) break;
+            tc_fence_after();
+            const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
+            const int64_t n = (int64_t)n_tile * kBlockN + r;
+            const int64_t m0 = (int64_t)m_tile * p.MG;
+            const bool whole = sg.kt0 == 0 && sg.kt1 == p.kt_count;
+            const int64_t slot = 2 * (int64_t)blockIdx.x + (sg.first ? 0 : 1);
+            float* part = p.partial + slot * (int64_t)p.MG * kBlockN;
+            for (int c0 = 0; c0 < p.MG; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+                tmem_wait_ld();
+                if (whole) {
+                    if (n < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 16; i++) {
+                            int64_t m = m0 + c0 + i;
+                            if (m < p.M) {
+                                float f = __uint_as_float(v[i]);
+                                if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = f;
+                                else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(f);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) part[(int64_t)(c0 + i) * kBlockN + r] = __uint_as_float(v[i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acce_bar));
+            if (!whole) {
+                // stream-K fix-up, one output row per thread
+                const int64_t t0 = sg.tile * p.kt_count, t1 = t0 + p.kt_count - 1;
+                const int64_t b_first = iter_owner(t0, p.total_iters, p.P);
+                const int64_t b_last = iter_owner(t1, p.total_iters, p.P);
+                const int nsegs = (int)(b_last - b_first + 1);
+                __threadfence();
+                int* cnt = p.counters + sg.tile * kBlockN + r;
+                int old = atomicAdd(cnt, 1);
+                if (old == nsegs - 1) {
+                    __threadfence();
+                    for (int c = 0; c < p.MG; c++) {
+                        int64_t m = m0 + c;
+                        float acc = 0.f;
+                        for (int64_t b = b_first; b <= b_last; b++) {
+                            int64_t bs = iter_begin(b, p.total_iters, p.P);
+                            int64_t sl = 2 * b + ((bs / p.kt_count) == sg.tile ? 0 : 1);
+                            acc += __ldcg(p.partial + (sl * p.MG + c) * kBlockN + r);
+                        }
+                        if (m < p.M && n < p.N) {
+                            if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc;
+                            else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc);
+                        }
+                    }
+                    *cnt = 0;
+                }
+            }
+            j++;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) raise_status(UW_ERR_TIMEOUT);
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tacc, tmem_cols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)ptr;
+    }
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swz128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    (void)esize;
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int pick_mg(int64_t M) {
+    int64_t mg = (M + 15) / 16 * 16;
+    if (mg > 256) mg = 256;
+    if (mg < 16) mg = 16;
+    return (int)mg;
+}
+
+uint64_t timeout_ns() {
+    static uint64_t t = 0;
+    if (!t) {
+        const char* e = getenv("UW_TIMEOUT_MS");
+        long ms = e ? atol(e) : 2000;
+        if (ms < 10) ms = 10;
+        t = (uint64_t)ms * 1000000ull;
+    }
+    return t;
+}
+
+}  // namespace
+
+int gemm_default_grid() { return num_sms(); }
+
+int gemm_status_take() { return unit_status_take(); }
+
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
+    (void)K;
+    int P = grid > 0 ? grid : gemm_default_grid();
+    int MG = pick_mg(M);
+    int64_t m_tiles = (M + MG - 1) / MG, n_tiles = (N + kBlockN - 1) / kBlockN;
+    size_t part = (size_t)2 * P * MG * kBlockN * 4;
+    size_t cnt = (size_t)m_tiles * n_tiles * kBlockN * 4;
+    return ((part + 255) & ~size_t(255)) + ((cnt + 255) & ~size_t(255));
+}
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
+    *st = UW_OK;
+    if (a.M == 0) return cudaSuccess;
+    GemmParams p{};
+    p.M = a.M;
+    p.N = a.N;
+    p.K = a.K;
+    p.KG = a.K / kBlockK;
+    p.MG = pick_mg(a.M);
+    p.m_tiles = (int)((a.M + p.MG - 1) / p.MG);
+    p.n_tiles = (int)((a.N + kBlockN - 1) / kBlockN);
+    p.kt_count = (int)(a.K / kBlockK);
+    int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    p.total_iters = tiles * p.kt_count;
+    int P = a.grid > 0 ? a.grid : gemm_default_grid();
+    if (P > p.total_iters) P = (int)p.total_iters;
+    p.P = P;
+    p.vbits = a.vbits;
+    p.vpre = a.vpre;
+    p.vexp = a.vexp;
+    if (a.palette)
+        for (int i = 0; i < 4; i++)
+            p.pal[i] = (uint32_t)a.palette[4 * i] | ((uint32_t)a.palette[4 * i + 1] << 8) |
+                       ((uint32_t)a.palette[4 * i + 2] << 16) | ((uint32_t)a.palette[4 * i + 3] << 24);
+    p.Y = a.Y;
+    p.out_f32 = a.out_f32;
+    size_t need = gemm_ws_bytes(a.M, a.N, a.K, P);
+    if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
+    size_t part = (size_t)2 * P * p.MG * kBlockN * 4;
+    p.partial = (float*)a.ws;
+    p.counters = (int*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
+    p.timeout_ns = timeout_ns();
+
+    // stage layout
+    const uint32_t b_bytes = (uint32_t)p.MG * 128;
+    uint32_t off = kTileA;
+    p.off_b = off;
+    off += b_bytes;
+    p.tx_bytes = b_bytes;
+    if (a.src == kSrcDense) {
+        p.tx_bytes += kTileA;
+    } else {
+        p.off_sm = off;
+        off += kTileSM;
+        p.off_s2 = off;
+        if (a.src == kSrcExponent) {
+            off += kTileE;
+            p.tx_bytes += kTileSM + kTileE;
+        } else {
+            off += kTileIdx;
+            p.off_v = off;
+            off += kTileV;
+            p.tx_bytes += kTileSM + kTileIdx + kTileV;
+        }
+    }
+    p.stage_bytes = (off + 1023) & ~1023u;
+    const size_t ctrl = 1024;
+    const size_t budget = 227 * 1024 - 1024 - ctrl;
+    int S = (int)(budget / p.stage_bytes);
+    if (S > kMaxStages) S = kMaxStages;
+    if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
+    p.stages = S;
+    size_t smem = (size_t)S * p.stage_bytes + ctrl + 1024;
+
+    CUtensorMap tx{}, ta{}, ts2{}, tv{};
+    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBlockK, p.MG, true);
+    if (a.src == kSrcDense) {
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, a.K, a.N, a.K * 2, kBlockK, kBlockN, true);
+        ts2 = ta;
+        tv = ta;
+    } else {
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, kBlockK, kBlockN, false);
+        if (a.src == kSrcExponent) {
+            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, kBlockK, kBlockN, false);
+            tv = ts2;
+        } else {
+            int64_t NW = 4 * ((a.N + 127) / 128);
+            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.idx, a.K / 2, a.N, a.K / 2, kBlockK / 2,
+                                   kBlockN, false);
+            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kBlockK, NW * 4, 4, 1, false);
+        }
+    }
+    if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
+
+    cudaError_t e;
+    switch (a.src) {
+        case kSrcDense:
+            e = cudaFuncSetAttribute(k_gemm<kSrcDense>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            k_gemm<kSrcDense><<<P, kThreadsDense, smem, s>>>(tx, ta, ts2, tv, p);
+            break;
+        case kSrcExponent:
+            e = cudaFuncSetAttribute(k_gemm<kSrcExponent>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            k_gemm<kSrcExponent><<<P, kThreadsRecon, smem, s>>>(tx, ta, ts2, tv, p);
+            break;
+        default:
+            e = cudaFuncSetAttribute(k_gemm<kSrcPalette>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            k_gemm<kSrcPalette><<<P, kThreadsRecon, smem, s>>>(tx, ta, ts2, tv, p);
+            break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace uw

@@ -1,0 +1,850 @@
+// uw_host.cpp -- host side of libunweight: argument checks, the Huffman code
+// construction, the device-image layout, compress/serialize/deserialize, and
+// the dispatch of the four pipelines and of the autotuner.
+//
+// "Cloudflare推出Unweight無損壓縮系統" (easyvibecoding.app):
+//   §BF16權重壓縮原理  palette of the 16 most frequent exponents, Huffman code,
+//                      verbatim 64-weight rows;
+//   §四種執行管道      pipelines (full / exponent / transcode / direct palette);
+//   §自動調優機制      coordinate-descent autotuner measured on the hardware.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "uw_internal.h"
+
+namespace uw {
+
+Geometry Geometry::of(int64_t N, int64_t K) {
+    Geometry g;
+    g.N = N;
+    g.K = K;
+    g.n = N * K;
+    g.G = g.n / kGroup;
+    g.GW = (g.G + 31) / 32;
+    g.KG = K / kGroup;
+    g.NW = 4 * ((N + 127) / 128);
+    g.nseg = (g.n + kSeg - 1) / kSeg;
+    g.nchunk = (g.nseg + kChunkSegs - 1) / kChunkSegs;
+    return g;
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = v > 0 ? v : 148;
+    }
+    return cached[dev];
+}
+
+// ---------------------------------------------------------------------------
+// Optimal length-limited code lengths (package-merge), kept as per-level lists
+// of tags.  The deepest level holds the leaves -- used symbols ordered by
+// (count, symbol).  Each shallower level merges the leaves with the pairs
+// ("packages") of the level below; on equal weight a leaf goes first.  Then,
+// from the top level down: the first 2(n-1) items are taken; every leaf taken
+// at some level lengthens its symbol's code by one, and the k packages taken
+// at one level mean the first 2k items of the level below are taken.
+// ---------------------------------------------------------------------------
+void build_code(const uint64_t freq[16], uint8_t len[16], uint32_t code[16]) {
+    for (int s = 0; s < 16; s++) { len[s] = 0; code[s] = 0; }
+    std::vector<int> used;
+    for (int s = 0; s < 16; s++)
+        if (freq[s]) used.push_back(s);
+    std::stable_sort(used.begin(), used.end(), [&](int a, int b) { return freq[a] < freq[b]; });
+    const int n = (int)used.size();
+    if (n == 1) len[used[0]] = 1;
+    if (n >= 2) {
+        struct Tag { uint64_t w; int leaf; };   // leaf < 0: package
+        std::vector<std::vector<Tag>> level(kLmax + 1);
+        for (int i = 0; i < n; i++) level[kLmax].push_back({freq[used[i]], i});
+        for (int l = kLmax - 1; l >= 1; l--) {
+            const std::vector<Tag>& below = level[l + 1];
+            std::vector<uint64_t> pk;
+            for (size_t i = 0; i + 1 < below.size(); i += 2) pk.push_back(below[i].w + below[i + 1].w);
+            size_t a = 0, b = 0;
+            while (a < (size_t)n || b < pk.size()) {
+                bool leaf = b >= pk.size() || (a < (size_t)n && freq[used[a]] <= pk[b]);
+                if (leaf) { level[l].push_back({freq[used[a]], (int)a}); a++; }
+                else { level[l].push_back({pk[b], -1}); b++; }
+            }
+        }
+        size_t take = 2 * (size_t)(n - 1);
+        for (int l = 1; l <= kLmax && take; l++) {
+            size_t packages = 0;
+            for (size_t i = 0; i < take && i < level[l].size(); i++) {
+                if (level[l][i].leaf >= 0) len[used[level[l][i].leaf]]++;
+                else packages++;
+            }
+            take = 2 * packages;
+        }
+    }
+    // canonical assignment: by (length, symbol); a longer code continues the
+    // running count shifted left by the length difference
+    std::vector<int> order;
+    for (int s = 0; s < 16; s++)
+        if (len[s]) order.push_back(s);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return len[a] < len[b]; });
+    uint32_t c = 0;
+    int prev = order.empty() ? 0 : len[order[0]];
+    for (size_t i = 0; i < order.size(); i++) {
+        int s = order[i];
+        c <<= (len[s] - prev);
+        prev = len[s];
+        code[s] = c++;
+    }
+}
+
+// 4096-entry multi-symbol table: entry p decodes as many whole codes (up to
+// four) as fit in the 12-bit window p, read MSB first.
+void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
+    std::vector<int> one_sym(kLutSize, -1), one_len(kLutSize, 0);
+    for (int s = 0; s < 16; s++) {
+        if (!len[s]) continue;
+        uint32_t lo = code[s] << (kLmax - len[s]), hi = (code[s] + 1) << (kLmax - len[s]);
+        for (uint32_t p = lo; p < hi && p < (uint32_t)kLutSize; p++) { one_sym[p] = s; one_len[p] = len[s]; }
+    }
+    for (uint32_t p = 0; p < (uint32_t)kLutSize; p++) {
+        uint32_t syms = 0, nsym = 0, used = 0;
+        while (nsym < 4) {
+            uint32_t w = (p << used) & (kLutSize - 1);
+            if (one_sym[w] < 0 || used + one_len[w] > (uint32_t)kLmax) break;
+            syms |= (uint32_t)one_sym[w] << (4 * nsym);
+            used += one_len[w];
+            nsym++;
+        }
+        lut[p] = syms | (nsym << 16) | (used << 19);
+    }
+}
+
+static uint64_t al256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+void layout_sections(uw_blob* b) {
+    const Geometry& g = b->geo;
+    const bool huff = b->forms & UW_FORM_HUFFMAN, pal = b->forms & UW_FORM_PALETTE;
+    b->bytes[UW_SEC_SM] = g.n;
+    b->bytes[UW_SEC_VBITS] = g.GW * 4;
+    b->bytes[UW_SEC_VPRE] = g.GW * 4;
+    b->bytes[UW_SEC_VEXP] = b->V * kGroup;
+    b->bytes[UW_SEC_VCOL] = g.KG * g.NW * 4;
+    b->bytes[UW_SEC_IDX] = pal ? g.n / 2 : 0;
+    b->bytes[UW_SEC_STREAM] = huff ? b->nwords * 4 : 0;
+    b->bytes[UW_SEC_CHUNK_OFF] = huff ? g.nchunk * 8 : 0;
+    b->bytes[UW_SEC_SEG_REL] = huff ? g.nseg * 2 : 0;
+    b->bytes[UW_SEC_LUT] = huff ? kLutSize * 4 : 0;
+    uint64_t off = 0;
+    for (int s = 0; s < UW_NSECT; s++) {
+        b->off[s] = off;
+        off += al256(b->bytes[s]);
+    }
+    b->dev_bytes = off < 256 ? 256 : off;
+}
+
+static void palette_from_hist(const uint64_t hist[256], uint8_t palette[16], uint8_t inv[256]) {
+    std::vector<int> e(256);
+    for (int i = 0; i < 256; i++) e[i] = i;
+    std::stable_sort(e.begin(), e.end(), [&](int a, int b) { return hist[a] > hist[b]; });
+    memset(inv, 0xFF, 256);
+    for (int i = 0; i < 16; i++) {
+        palette[i] = (uint8_t)e[i];
+        inv[e[i]] = (uint8_t)i;
+    }
+}
+
+}  // namespace uw
+
+using namespace uw;
+
+// ===========================================================================
+// misc
+// ===========================================================================
+extern "C" const char* uw_status_str(int s) {
+    switch (s) {
+        case UW_OK: return "UW_OK";
+        case UW_ERR_INVALID_ARG: return "UW_ERR_INVALID_ARG";
+        case UW_ERR_SHAPE: return "UW_ERR_SHAPE";
+        case UW_ERR_CORRUPT: return "UW_ERR_CORRUPT";
+        case UW_ERR_UNSUPPORTED: return "UW_ERR_UNSUPPORTED";
+        case UW_ERR_WORKSPACE: return "UW_ERR_WORKSPACE";
+        case UW_ERR_CUDA: return "UW_ERR_CUDA";
+        case UW_ERR_TIMEOUT: return "UW_ERR_TIMEOUT";
+        case UW_ERR_DEVICE: return "UW_ERR_DEVICE";
+        default: return "UW_ERR_UNKNOWN";
+    }
+}
+
+extern "C" int uw_version(void) { return 10000; }
+
+extern "C" uw_status uw_last_device_status(void* stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return UW_ERR_CUDA;
+    }
+    int d = decode_status_take(), g = gemm_status_take();
+    if (d < 0 || g < 0) return UW_ERR_CUDA;
+    return (uw_status)(d ? d : g);
+}
+
+static bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+static uw_status check_shape(int64_t N, int64_t K) {
+    if (N < 1 || K < kGroup || K % kGroup) return UW_ERR_SHAPE;
+    if (N > kMaxElems / K) return UW_ERR_SHAPE;
+    return UW_OK;
+}
+
+static uw_status cuda_ok(cudaError_t e) {
+    if (e == cudaSuccess) return UW_OK;
+    cudaGetLastError();
+    return UW_ERR_CUDA;
+}
+
+// ===========================================================================
+// compress
+// ===========================================================================
+extern "C" uw_status uw_compress_scratch_bytes(int64_t N, int64_t K, size_t* bytes) {
+    if (!bytes) return UW_ERR_INVALID_ARG;
+    uw_status st = check_shape(N, K);
+    if (st) return st;
+    *bytes = compress_scratch_bytes(Geometry::of(N, K));
+    return UW_OK;
+}
+
+extern "C" uw_status uw_compress_query(const uint16_t* W, int64_t N, int64_t K, uint32_t forms, void* scratch,
+                                       size_t scratch_bytes, void* stream, uw_blob** out, size_t* dev_bytes) {
+    if (!W || !scratch || !out || !dev_bytes) return UW_ERR_INVALID_ARG;
+    if (forms == 0 || (forms & ~uint32_t(UW_FORM_HUFFMAN | UW_FORM_PALETTE))) return UW_ERR_INVALID_ARG;
+    uw_status st = check_shape(N, K);
+    if (st) return st;
+    if (!aligned(W, 16) || !aligned(scratch, 256)) return UW_ERR_INVALID_ARG;
+    Geometry g = Geometry::of(N, K);
+    if (scratch_bytes < compress_scratch_bytes(g)) return UW_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    CompressScratch sc = carve_scratch(scratch, g);
+
+    uw_blob* b = new uw_blob();
+    b->geo = g;
+    b->forms = forms;
+    auto fail = [&](uw_status e) { delete b; return e; };
+
+    std::vector<uint32_t> h32(256), f32(16);
+    if (cuda_ok(launch_histogram(W, g.n, sc.hist, s))) return fail(UW_ERR_CUDA);
+    if (cuda_ok(cudaMemcpyAsync(h32.data(), sc.hist, 256 * 4, cudaMemcpyDeviceToHost, s))) return fail(UW_ERR_CUDA);
+    if (cuda_ok(cudaStreamSynchronize(s))) return fail(UW_ERR_CUDA);
+    for (int i = 0; i < 256; i++) b->hist[i] = h32[i];
+    palette_from_hist(b->hist, b->palette, b->inv);
+
+    if (cuda_ok(launch_verbatim_freq(W, g, b->inv, sc.vbits, sc.freq, s))) return fail(UW_ERR_CUDA);
+    b->vbits_h.resize(g.GW);
+    if (cuda_ok(cudaMemcpyAsync(f32.data(), sc.freq, 16 * 4, cudaMemcpyDeviceToHost, s))) return fail(UW_ERR_CUDA);
+    if (cuda_ok(cudaMemcpyAsync(b->vbits_h.data(), sc.vbits, g.GW * 4, cudaMemcpyDeviceToHost, s)))
+        return fail(UW_ERR_CUDA);
+    if (cuda_ok(cudaStreamSynchronize(s))) return fail(UW_ERR_CUDA);
+    for (int i = 0; i < 16; i++) b->freq[i] = f32[i];
+    build_code(b->freq, b->code_len, b->code);
+
+    b->vpre_h.resize(g.GW);
+    uint64_t run = 0;
+    for (int64_t w = 0; w < g.GW; w++) {
+        b->vpre_h[w] = (uint32_t)run;
+        run += __builtin_popcount(b->vbits_h[w]);
+    }
+    b->V = (int64_t)run;
+
+    if (forms & UW_FORM_HUFFMAN) {
+        std::vector<uint32_t> segbits(g.nseg);
+        if (cuda_ok(launch_segbits(W, g, b->inv, sc.vbits, b->code_len, sc.segbits, s))) return fail(UW_ERR_CUDA);
+        if (cuda_ok(cudaMemcpyAsync(segbits.data(), sc.segbits, g.nseg * 4, cudaMemcpyDeviceToHost, s)))
+            return fail(UW_ERR_CUDA);
+        if (cuda_ok(cudaStreamSynchronize(s))) return fail(UW_ERR_CUDA);
+        b->chunk_off_h.resize(g.nchunk);
+        b->seg_rel_h.resize(g.nseg);
+        uint64_t pos = 0;
+        for (int64_t j = 0; j < g.nseg; j++) {
+            if (j % kChunkSegs == 0) b->chunk_off_h[j / kChunkSegs] = pos;
+            b->seg_rel_h[j] = (uint16_t)(pos - b->chunk_off_h[j / kChunkSegs]);
+            pos += segbits[j];
+        }
+        b->total_bits = pos;
+        b->nwords = (int64_t)((pos + 31) / 32) + 2;
+        b->lut_h.resize(kLutSize);
+        build_lut(b->code_len, b->code, b->lut_h.data());
+    }
+    layout_sections(b);
+    *out = b;
+    *dev_bytes = b->dev_bytes;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_compress_commit(uw_blob* b, const uint16_t* W, void* scratch, size_t scratch_bytes,
+                                        void* dev_buf, size_t dev_bytes, void* stream) {
+    if (!b || b->magic != kMagic || !W || !scratch || !dev_buf) return UW_ERR_INVALID_ARG;
+    if (b->committed) return UW_ERR_INVALID_ARG;
+    const Geometry& g = b->geo;
+    if (scratch_bytes < compress_scratch_bytes(g)) return UW_ERR_WORKSPACE;
+    if (!aligned(dev_buf, 256) || dev_bytes < b->dev_bytes) return UW_ERR_WORKSPACE;
+    if (!aligned(W, 16)) return UW_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    b->dev = (uint8_t*)dev_buf;
+    uint8_t* d = b->dev;
+    auto sec = [&](int k) { return d + b->off[k]; };
+    if (cuda_ok(cudaMemsetAsync(d, 0, b->dev_bytes, s))) return UW_ERR_CUDA;
+    if (cuda_ok(cudaMemcpyAsync(sec(UW_SEC_VBITS), b->vbits_h.data(), g.GW * 4, cudaMemcpyHostToDevice, s)))
+        return UW_ERR_CUDA;
+    if (cuda_ok(cudaMemcpyAsync(sec(UW_SEC_VPRE), b->vpre_h.data(), g.GW * 4, cudaMemcpyHostToDevice, s)))
+        return UW_ERR_CUDA;
+    const uint32_t* vbits = (const uint32_t*)sec(UW_SEC_VBITS);
+    if (cuda_ok(launch_planes(W, g, b->inv, vbits, sec(UW_SEC_SM),
+                              (b->forms & UW_FORM_PALETTE) ? sec(UW_SEC_IDX) : nullptr, s)))
+        return UW_ERR_CUDA;
+    if (b->V && cuda_ok(launch_vexp(W, g, vbits, (const uint32_t*)sec(UW_SEC_VPRE), sec(UW_SEC_VEXP), s)))
+        return UW_ERR_CUDA;
+    if (cuda_ok(launch_vcol(g, vbits, (uint32_t*)sec(UW_SEC_VCOL), s))) return UW_ERR_CUDA;
+    if (b->forms & UW_FORM_HUFFMAN) {
+        if (cuda_ok(cudaMemcpyAsync(sec(UW_SEC_CHUNK_OFF), b->chunk_off_h.data(), g.nchunk * 8,
+                                    cudaMemcpyHostToDevice, s)))
+            return UW_ERR_CUDA;
+        if (cuda_ok(cudaMemcpyAsync(sec(UW_SEC_SEG_REL), b->seg_rel_h.data(), g.nseg * 2, cudaMemcpyHostToDevice, s)))
+            return UW_ERR_CUDA;
+        if (cuda_ok(cudaMemcpyAsync(sec(UW_SEC_LUT), b->lut_h.data(), kLutSize * 4, cudaMemcpyHostToDevice, s)))
+            return UW_ERR_CUDA;
+        if (cuda_ok(launch_encode(W, g, b->inv, vbits, b->code_len, b->code, (const uint64_t*)sec(UW_SEC_CHUNK_OFF),
+                                  (const uint16_t*)sec(UW_SEC_SEG_REL), (uint32_t*)sec(UW_SEC_STREAM), b->nwords, s)))
+            return UW_ERR_CUDA;
+    }
+    if (cuda_ok(cudaStreamSynchronize(s))) return UW_ERR_CUDA;
+    b->committed = true;
+    std::vector<uint32_t>().swap(b->vbits_h);
+    std::vector<uint32_t>().swap(b->vpre_h);
+    std::vector<uint64_t>().swap(b->chunk_off_h);
+    std::vector<uint16_t>().swap(b->seg_rel_h);
+    std::vector<uint32_t>().swap(b->lut_h);
+    return UW_OK;
+}
+
+extern "C" void uw_blob_free(uw_blob* b) {
+    if (b && b->magic == kMagic) {
+        b->magic = 0;
+        delete b;
+    }
+}
+
+extern "C" uw_status uw_blob_info_get(const uw_blob* b, uw_blob_info* info) {
+    if (!b || b->magic != kMagic || !info) return UW_ERR_INVALID_ARG;
+    memset(info, 0, sizeof(*info));
+    const Geometry& g = b->geo;
+    info->N = g.N;
+    info->K = g.K;
+    info->G = g.G;
+    info->V = b->V;
+    info->nseg = g.nseg;
+    info->nchunk = g.nchunk;
+    info->forms = b->forms;
+    memcpy(info->palette, b->palette, 16);
+    memcpy(info->code_len, b->code_len, 16);
+    for (int i = 0; i < 16; i++) info->freq[i] = b->freq[i];
+    for (int i = 0; i < 256; i++) info->hist[i] = b->hist[i];
+    info->total_bits = b->total_bits;
+    const uint64_t vstore = g.GW * 8 + b->V * kGroup;
+    info->bytes_huffman_form = g.n + b->nwords * 4 + g.nchunk * 8 + g.nseg * 2 + vstore;
+    info->bytes_palette_form = g.n + g.n / 2 + vstore + g.KG * g.NW * 4;
+    info->device_bytes = b->dev_bytes;
+    info->mean_code_len = g.n ? (double)b->total_bits / (double)g.n : 0.0;
+    double H = 0.0, cover = 0.0;
+    for (int e = 0; e < 256; e++) {
+        if (!b->hist[e]) continue;
+        double p = (double)b->hist[e] / (double)g.n;
+        H -= p * std::log2(p);
+    }
+    for (int i = 0; i < 16; i++) cover += (double)b->hist[b->palette[i]];
+    info->exponent_entropy = H;
+    info->palette_coverage = cover / (double)g.n;
+    for (int s = 0; s < UW_NSECT; s++) {
+        info->section_offset[s] = b->off[s];
+        info->section_bytes[s] = b->bytes[s];
+    }
+    return UW_OK;
+}
+
+extern "C" uw_status uw_blob_section(const uw_blob* b, int section, const void** dev_ptr, size_t* bytes) {
+    if (!b || b->magic != kMagic || !dev_ptr || !bytes || section < 0 || section >= UW_NSECT) return UW_ERR_INVALID_ARG;
+    if (!b->committed) return UW_ERR_INVALID_ARG;
+    *dev_ptr = b->dev + b->off[section];
+    *bytes = b->bytes[section];
+    return UW_OK;
+}
+
+// ===========================================================================
+// serialize / deserialize ("distribution bundle")
+// ===========================================================================
+namespace {
+struct SerialHeader {
+    uint32_t magic, version;
+    int64_t N, K;
+    uint32_t forms, pad;
+    int64_t V, nwords;
+    uint64_t total_bits;
+    uint8_t palette[16], code_len[16];
+    uint64_t freq[16], hist[256];
+    uint64_t bytes[UW_NSECT];
+};
+constexpr int kSerialSections = UW_SEC_LUT;   // LUT is derived, not stored
+}  // namespace
+
+extern "C" uw_status uw_blob_serialized_bytes(const uw_blob* b, size_t* bytes) {
+    if (!b || b->magic != kMagic || !bytes || !b->committed) return UW_ERR_INVALID_ARG;
+    size_t t = sizeof(SerialHeader);
+    for (int s = 0; s < kSerialSections; s++) t += b->bytes[s];
+    *bytes = t;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_blob_serialize(const uw_blob* b, void* host_dst, size_t cap, size_t* written, void* stream) {
+    size_t need = 0;
+    uw_status st = uw_blob_serialized_bytes(b, &need);
+    if (st) return st;
+    if (!host_dst || cap < need) return UW_ERR_WORKSPACE;
+    SerialHeader h{};
+    h.magic = kMagic;
+    h.version = kFormatVersion;
+    h.N = b->geo.N;
+    h.K = b->geo.K;
+    h.forms = b->forms;
+    h.V = b->V;
+    h.nwords = b->nwords;
+    h.total_bits = b->total_bits;
+    memcpy(h.palette, b->palette, 16);
+    memcpy(h.code_len, b->code_len, 16);
+    for (int i = 0; i < 16; i++) h.freq[i] = b->freq[i];
+    for (int i = 0; i < 256; i++) h.hist[i] = b->hist[i];
+    for (int s = 0; s < UW_NSECT; s++) h.bytes[s] = s < kSerialSections ? b->bytes[s] : 0;
+    uint8_t* p = (uint8_t*)host_dst;
+    memcpy(p, &h, sizeof h);
+    p += sizeof h;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int k = 0; k < kSerialSections; k++) {
+        if (b->bytes[k] && cuda_ok(cudaMemcpyAsync(p, b->dev + b->off[k], b->bytes[k], cudaMemcpyDeviceToHost, s)))
+            return UW_ERR_CUDA;
+        p += b->bytes[k];
+    }
+    if (cuda_ok(cudaStreamSynchronize(s))) return UW_ERR_CUDA;
+    if (written) *written = need;
+    return UW_OK;
+}
+
+// Builds a handle from a header, checking everything that can be checked
+// without the sections.  Returns null on inconsistency.
+static uw_blob* blob_from_header(const void* host_src, size_t n) {
+    if (!host_src || n < sizeof(SerialHeader)) return nullptr;
+    SerialHeader h;
+    memcpy(&h, host_src, sizeof h);
+    if (h.magic != kMagic || h.version != kFormatVersion) return nullptr;
+    if (check_shape(h.N, h.K) != UW_OK) return nullptr;
+    if (h.forms == 0 || (h.forms & ~uint32_t(UW_FORM_HUFFMAN | UW_FORM_PALETTE))) return nullptr;
+    Geometry g = Geometry::of(h.N, h.K);
+    if (h.V < 0 || h.V > g.G) return nullptr;
+    uw_blob* b = new uw_blob();
+    b->geo = g;
+    b->forms = h.forms;
+    b->V = h.V;
+    b->nwords = h.nwords;
+    b->total_bits = h.total_bits;
+    memcpy(b->palette, h.palette, 16);
+    memcpy(b->code_len, h.code_len, 16);
+    for (int i = 0; i < 16; i++) b->freq[i] = h.freq[i];
+    for (int i = 0; i < 256; i++) b->hist[i] = h.hist[i];
+    bool ok = true;
+    // palette: distinct values
+    bool seen[256] = {false};
+    memset(b->inv, 0xFF, 256);
+    for (int i = 0; i < 16; i++) {
+        if (seen[b->palette[i]]) ok = false;
+        seen[b->palette[i]] = true;
+        b->inv[b->palette[i]] = (uint8_t)i;
+    }
+    uint64_t hsum = 0, fsum = 0;
+    for (int i = 0; i < 256; i++) hsum += b->hist[i];
+    for (int i = 0; i < 16; i++) fsum += b->freq[i];
+    if (hsum != (uint64_t)g.n || fsum != (uint64_t)g.n) ok = false;
+    if (b->forms & UW_FORM_HUFFMAN) {
+        // code lengths: <= 12, used exactly by the symbols that occur, prefix-free (Kraft <= 1)
+        uint64_t kraft = 0;
+        int used = 0;
+        for (int i = 0; i < 16; i++) {
+            if (b->code_len[i] > kLmax) ok = false;
+            if ((b->code_len[i] != 0) != (b->freq[i] != 0)) ok = false;
+            if (b->code_len[i]) { kraft += 1ull << (kLmax - b->code_len[i]); used++; }
+        }
+        if (kraft > (1ull << kLmax) || used == 0) ok = false;
+        if (used >= 2 && kraft != (1ull << kLmax)) ok = false;
+        uint64_t bits = 0;
+        for (int i = 0; i < 16; i++) bits += b->freq[i] * b->code_len[i];
+        if (bits != b->total_bits) ok = false;
+        if (b->nwords != (int64_t)((b->total_bits + 31) / 32) + 2) ok = false;
+        if (ok) {
+            // canonical codes follow from the stored lengths alone
+            std::vector<int> order;
+            for (int s = 0; s < 16; s++)
+                if (b->code_len[s]) order.push_back(s);
+            std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return b->code_len[x] < b->code_len[y]; });
+            uint32_t c = 0;
+            int prev = order.empty() ? 0 : b->code_len[order[0]];
+            for (int s : order) {
+                c <<= (b->code_len[s] - prev);
+                prev = b->code_len[s];
+                b->code[s] = c++;
+            }
+        }
+    } else {
+        b->nwords = 0;
+        b->total_bits = 0;
+    }
+    if (!ok) { delete b; return nullptr; }
+    layout_sections(b);
+    for (int s = 0; s < kSerialSections; s++)
+        if (h.bytes[s] != b->bytes[s]) { delete b; return nullptr; }
+    size_t need = sizeof h;
+    for (int s = 0; s < kSerialSections; s++) need += b->bytes[s];
+    if (n < need) { delete b; return nullptr; }
+    return b;
+}
+
+extern "C" uw_status uw_blob_device_bytes(const void* host_src, size_t n, size_t* dev_bytes) {
+    if (!dev_bytes) return UW_ERR_INVALID_ARG;
+    uw_blob* b = blob_from_header(host_src, n);
+    if (!b) return UW_ERR_CORRUPT;
+    *dev_bytes = b->dev_bytes;
+    delete b;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_blob_deserialize(const void* host_src, size_t n, void* dev_buf, size_t dev_bytes, void* stream,
+                                         uw_blob** out) {
+    if (!out || !dev_buf) return UW_ERR_INVALID_ARG;
+    uw_blob* b = blob_from_header(host_src, n);
+    if (!b) return UW_ERR_CORRUPT;
+    if (!aligned(dev_buf, 256) || dev_bytes < b->dev_bytes) { delete b; return UW_ERR_WORKSPACE; }
+    const Geometry& g = b->geo;
+    const uint8_t* p = (const uint8_t*)host_src + sizeof(SerialHeader);
+    const uint8_t* sec[UW_NSECT] = {nullptr};
+    for (int s = 0; s < kSerialSections; s++) { sec[s] = p; p += b->bytes[s]; }
+    // verbatim store consistency
+    const uint32_t* vbits = (const uint32_t*)sec[UW_SEC_VBITS];
+    const uint32_t* vpre = (const uint32_t*)sec[UW_SEC_VPRE];
+    uint64_t run = 0;
+    bool ok = true;
+    for (int64_t w = 0; w < g.GW; w++) {
+        if (vpre[w] != run) ok = false;
+        run += __builtin_popcount(vbits[w]);
+    }
+    if (g.G & 31) {
+        uint32_t tail = vbits[g.GW - 1] >> (g.G & 31);
+        if (tail) ok = false;
+    }
+    if (run != (uint64_t)b->V) ok = false;
+    // vcol must be the transpose of vbits
+    {
+        const uint32_t* vcol = (const uint32_t*)sec[UW_SEC_VCOL];
+        uint64_t colbits = 0;
+        for (int64_t t = 0; t < g.KG * g.NW; t++) colbits += __builtin_popcount(vcol[t]);
+        if (colbits != run) ok = false;
+        for (int64_t gi = 0; ok && gi < g.G; gi++) {
+            if (!((vbits[gi >> 5] >> (gi & 31)) & 1u)) continue;
+            int64_t nn = gi / g.KG, kt = gi % g.KG;
+            if (!((vcol[kt * g.NW + nn / 32] >> (nn % 32)) & 1u)) ok = false;
+        }
+    }
+    if (b->forms & UW_FORM_HUFFMAN) {
+        const uint64_t* co = (const uint64_t*)sec[UW_SEC_CHUNK_OFF];
+        const uint16_t* sr = (const uint16_t*)sec[UW_SEC_SEG_REL];
+        if (g.nchunk && co[0] != 0) ok = false;
+        for (int64_t c = 0; ok && c < g.nchunk; c++) {
+            if (c && co[c] < co[c - 1]) ok = false;
+            if (co[c] > b->total_bits) ok = false;
+        }
+        for (int64_t j = 0; ok && j < g.nseg; j++) {
+            uint64_t pos = co[j / kChunkSegs] + sr[j];
+            if (j % kChunkSegs == 0 && sr[j] != 0) ok = false;
+            if (pos > b->total_bits) ok = false;
+            if ((uint64_t)sr[j] > (uint64_t)(j % kChunkSegs) * kSeg * kLmax) ok = false;
+        }
+    }
+    if (!ok) { delete b; return UW_ERR_CORRUPT; }
+    cudaStream_t s = (cudaStream_t)stream;
+    b->dev = (uint8_t*)dev_buf;
+    for (int k = 0; k < kSerialSections; k++)
+        if (b->bytes[k] && cuda_ok(cudaMemcpyAsync(b->dev + b->off[k], sec[k], b->bytes[k], cudaMemcpyHostToDevice, s))) {
+            delete b;
+            return UW_ERR_CUDA;
+        }
+    if (b->forms & UW_FORM_HUFFMAN) {
+        b->lut_h.resize(kLutSize);
+        build_lut(b->code_len, b->code, b->lut_h.data());
+        if (cuda_ok(cudaMemcpyAsync(b->dev + b->off[UW_SEC_LUT], b->lut_h.data(), kLutSize * 4, cudaMemcpyHostToDevice, s))) {
+            delete b;
+            return UW_ERR_CUDA;
+        }
+    }
+    if (cuda_ok(cudaStreamSynchronize(s))) { delete b; return UW_ERR_CUDA; }
+    std::vector<uint32_t>().swap(b->lut_h);
+    b->committed = true;
+    *out = b;
+    return UW_OK;
+}
+
+// ===========================================================================
+// decode
+// ===========================================================================
+static uw_status check_committed(const uw_blob* b) {
+    if (!b || b->magic != kMagic || !b->committed) return UW_ERR_INVALID_ARG;
+    return UW_OK;
+}
+
+static uw_status decode_common(const uw_blob* b, void* out, int mode, void* stream) {
+    uw_status st = check_committed(b);
+    if (st) return st;
+    if (!out || !aligned(out, 16)) return UW_ERR_INVALID_ARG;
+    if (!(b->forms & UW_FORM_HUFFMAN)) return UW_ERR_UNSUPPORTED;
+    return cuda_ok(launch_decode(b, mode, out, 0, (cudaStream_t)stream));
+}
+
+extern "C" uw_status uw_decode_full(const uw_blob* b, uint16_t* W_out, void* stream) {
+    return decode_common(b, W_out, kDecodeFull, stream);
+}
+extern "C" uw_status uw_decode_exponent(const uw_blob* b, uint8_t* E_out, void* stream) {
+    return decode_common(b, E_out, kDecodeExponent, stream);
+}
+extern "C" uw_status uw_transcode_palette(const uw_blob* b, uint8_t* idx_out, void* stream) {
+    return decode_common(b, idx_out, kDecodeTranscode, stream);
+}
+
+// ===========================================================================
+// GEMM
+// ===========================================================================
+static size_t decode_buffer_bytes(const uw_blob* b, int pipeline) {
+    switch (pipeline) {
+        case UW_PIPE_FULL: return al256(b->geo.n * 2);
+        case UW_PIPE_EXPONENT: return al256(b->geo.n);
+        case UW_PIPE_TRANSCODE: return al256(b->geo.n / 2);
+        default: return 0;
+    }
+}
+
+extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gemm_opts* o, size_t* bytes) {
+    uw_status st = check_committed(b);
+    if (st) return st;
+    if (!o || !bytes || M < 0) return UW_ERR_INVALID_ARG;
+    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (M == 0) { *bytes = 0; return UW_OK; }
+    *bytes = decode_buffer_bytes(b, o->pipeline) + gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid);
+    return UW_OK;
+}
+
+extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, void* Y, const uw_gemm_opts* o,
+                             void* stream) {
+    uw_status st = check_committed(b);
+    if (st) return st;
+    if (!o || M < 0) return UW_ERR_INVALID_ARG;
+    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (o->sm_dec < 0 || o->grid < 0) return UW_ERR_INVALID_ARG;
+    if (M == 0) return UW_OK;
+    if (!X || !Y || !aligned(X, 16) || !aligned(Y, 16)) return UW_ERR_INVALID_ARG;
+    const bool needs_huff = o->pipeline != UW_PIPE_DIRECT_PALETTE;
+    if (needs_huff && !(b->forms & UW_FORM_HUFFMAN)) return UW_ERR_UNSUPPORTED;
+    if (!needs_huff && !(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
+    if (o->sm_dec > 0) return UW_ERR_UNSUPPORTED;
+    size_t need = 0;
+    uw_gemm_workspace(b, M, o, &need);
+    if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* ws = (uint8_t*)o->workspace;
+    const size_t dbuf = decode_buffer_bytes(b, o->pipeline);
+
+    GemmArgs a;
+    a.X = X;
+    a.M = M;
+    a.N = b->geo.N;
+    a.K = b->geo.K;
+    a.Y = Y;
+    a.out_f32 = o->out_f32 ? 1 : 0;
+    a.grid = o->grid;
+    a.ws = ws + dbuf;
+    a.ws_bytes = o->workspace_bytes - dbuf;
+    a.sm = b->sec(UW_SEC_SM);
+    a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
+    a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
+    a.vexp = b->sec(UW_SEC_VEXP);
+    a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
+    a.palette = b->palette;
+    switch (o->pipeline) {
+        case UW_PIPE_FULL:
+            if (cuda_ok(launch_decode(b, kDecodeFull, ws, 0, s))) return UW_ERR_CUDA;
+            a.src = kSrcDense;
+            a.W = (const uint16_t*)ws;
+            break;
+        case UW_PIPE_EXPONENT:
+            if (cuda_ok(launch_decode(b, kDecodeExponent, ws, 0, s))) return UW_ERR_CUDA;
+            a.src = kSrcExponent;
+            a.ex = ws;
+            break;
+        case UW_PIPE_TRANSCODE:
+            if (cuda_ok(launch_decode(b, kDecodeTranscode, ws, 0, s))) return UW_ERR_CUDA;
+            a.src = kSrcPalette;
+            a.idx = ws;
+            break;
+        default:
+            a.src = kSrcPalette;
+            a.idx = b->sec(UW_SEC_IDX);
+            break;
+    }
+    cudaError_t e = launch_gemm(a, s, &st);
+    if (st) return st;
+    return cuda_ok(e);
+}
+
+extern "C" uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int grid, size_t* bytes) {
+    if (!bytes || M < 0 || grid < 0) return UW_ERR_INVALID_ARG;
+    uw_status st = check_shape(N, K);
+    if (st) return st;
+    *bytes = M ? gemm_ws_bytes(M, N, K, grid) : 0;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K, void* Y,
+                                   int out_f32, int grid, void* workspace, size_t workspace_bytes, void* stream) {
+    if (M < 0 || grid < 0) return UW_ERR_INVALID_ARG;
+    uw_status st = check_shape(N, K);
+    if (st) return st;
+    if (M == 0) return UW_OK;
+    if (!X || !W || !Y || !aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16)) return UW_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < gemm_ws_bytes(M, N, K, grid)) return UW_ERR_WORKSPACE;
+    GemmArgs a;
+    a.src = kSrcDense;
+    a.X = X;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.W = W;
+    a.Y = Y;
+    a.out_f32 = out_f32 ? 1 : 0;
+    a.grid = grid;
+    a.ws = workspace;
+    a.ws_bytes = workspace_bytes;
+    cudaError_t e = launch_gemm(a, (cudaStream_t)stream, &st);
+    if (st) return st;
+    return cuda_ok(e);
+}
+
+// ===========================================================================
+// autotune (§自動調優機制)
+// ===========================================================================
+extern "C" uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const int64_t* Ms, int nM,
+                                 const uint16_t* const* X, void* const* Y, void* workspace, size_t workspace_bytes,
+                                 int reps, uw_plan_entry* plan, const char* plan_json_path, void* stream) {
+    if (!blobs || nblobs < 1 || !Ms || nM < 1 || !X || !Y || !plan || reps < 1) return UW_ERR_INVALID_ARG;
+    for (int i = 0; i < nblobs; i++) {
+        uw_status st = check_committed(blobs[i]);
+        if (st) return st;
+        if (!X[i] || !Y[i]) return UW_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaEvent_t e0, e1;
+    if (cuda_ok(cudaEventCreate(&e0)) || cuda_ok(cudaEventCreate(&e1))) return UW_ERR_CUDA;
+    struct Cand { int pipe, sm_dec; };
+    std::vector<Cand> cands;
+    for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_DIRECT_PALETTE; pp++) cands.push_back({pp, 0});
+    uw_status result = UW_OK;
+    for (int mi = 0; mi < nM && result == UW_OK; mi++) {
+        const int64_t M = Ms[mi];
+        // feasible candidates per projection
+        std::vector<std::vector<int>> feas(nblobs);
+        for (int i = 0; i < nblobs; i++)
+            for (int c = 0; c < (int)cands.size(); c++) {
+                uw_gemm_opts o{};
+                o.pipeline = cands[c].pipe;
+                o.sm_dec = cands[c].sm_dec;
+                size_t need = 0;
+                bool has = cands[c].pipe == UW_PIPE_DIRECT_PALETTE ? (blobs[i]->forms & UW_FORM_PALETTE)
+                                                                   : (blobs[i]->forms & UW_FORM_HUFFMAN);
+                if (has && uw_gemm_workspace(blobs[i], M, &o, &need) == UW_OK && need <= workspace_bytes)
+                    feas[i].push_back(c);
+            }
+        for (int i = 0; i < nblobs; i++)
+            if (feas[i].empty()) result = UW_ERR_WORKSPACE;
+        if (result) break;
+        std::vector<int> choice(nblobs);
+        for (int i = 0; i < nblobs; i++) choice[i] = feas[i][0];
+        std::vector<double> per(nblobs, 0.0);
+        auto run_layer = [&](const std::vector<int>& ch, std::vector<double>* per_out) -> double {
+            double total = 0.0;
+            for (int i = 0; i < nblobs; i++) {
+                uw_gemm_opts o{};
+                o.pipeline = cands[ch[i]].pipe;
+                o.sm_dec = cands[ch[i]].sm_dec;
+                o.workspace = workspace;
+                o.workspace_bytes = workspace_bytes;
+                // warm-up
+                if (uw_gemm(X[i], M, blobs[i], Y[i], &o, stream) != UW_OK) return -1.0;
+                cudaEventRecord(e0, s);
+                for (int r = 0; r < reps; r++) uw_gemm(X[i], M, blobs[i], Y[i], &o, stream);
+                cudaEventRecord(e1, s);
+                if (cudaEventSynchronize(e1) != cudaSuccess) return -1.0;
+                float ms = 0.f;
+                cudaEventElapsedTime(&ms, e0, e1);
+                double us = 1000.0 * ms / reps;
+                if (per_out) (*per_out)[i] = us;
+                total += us;
+            }
+            return total;
+        };
+        double best = run_layer(choice, &per);
+        if (best < 0) { result = UW_ERR_CUDA; break; }
+        for (int round = 0; round < 8; round++) {
+            bool improved = false;
+            for (int i = 0; i < nblobs; i++) {
+                for (int c : feas[i]) {
+                    if (c == choice[i]) continue;
+                    std::vector<int> trial = choice;
+                    trial[i] = c;
+                    std::vector<double> tp(nblobs, 0.0);
+                    double t = run_layer(trial, &tp);
+                    if (t < 0) { result = UW_ERR_CUDA; break; }
+                    if (t < best * 0.99) { best = t; choice = trial; per = tp; improved = true; }
+                }
+                if (result) break;
+            }
+            if (!improved || result) break;
+        }
+        for (int i = 0; i < nblobs; i++) {
+            uw_plan_entry& pe = plan[mi * nblobs + i];
+            pe.blob_index = i;
+            pe.M = M;
+            pe.pipeline = cands[choice[i]].pipe;
+            pe.sm_dec = cands[choice[i]].sm_dec;
+            pe.grid = 0;
+            pe.us = per[i];
+        }
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (result == UW_OK && plan_json_path) {
+        FILE* f = fopen(plan_json_path, "w");
+        if (!f) return UW_ERR_INVALID_ARG;
+        static const char* names[] = {"full", "exponent", "transcode", "direct_palette"};
+        fprintf(f, "{\"plan\": [\n");
+        for (int k = 0; k < nM * nblobs; k++)
+            fprintf(f, "  {\"projection\": %d, \"M\": %lld, \"pipeline\": \"%s\", \"sm_dec\": %d, \"us\": %.3f}%s\n",
+                    plan[k].blob_index, (long long)plan[k].M, names[plan[k].pipeline], plan[k].sm_dec, plan[k].us,
+                    k + 1 < nM * nblobs ? "," : "");
+        fprintf(f, "]}\n");
+        fclose(f);
+    }
+    return result;
+}

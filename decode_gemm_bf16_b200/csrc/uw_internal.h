@@ -1,0 +1,133 @@
+// uw_internal.h -- host-side state shared by the translation units of
+// libunweight.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/unweight.h"
+
+namespace uw {
+
+constexpr int kGroup = 64;        // weights per verbatim decision
+constexpr int kPalette = 16;      // palette entries
+constexpr int kSeg = 256;         // symbols per decode segment
+constexpr int kChunkSegs = 16;    // segments per chunk offset
+constexpr int kLmax = 12;         // longest Huffman code, bits
+constexpr int kLutSize = 1 << kLmax;
+constexpr uint32_t kMagic = 0x31425755u;  // "UWB1"
+constexpr uint32_t kFormatVersion = 1;
+constexpr int64_t kMaxElems = (int64_t(1) << 31) - 256;
+
+// Decode-table entry (derived from the code lengths):
+//   bits  0..15  up to four symbols, symbol i in bits 4i..4i+3
+//   bits 16..18  number of symbols decoded from the 12-bit window (0 = invalid)
+//   bits 19..23  bits consumed by those symbols
+__host__ __device__ constexpr uint32_t lut_nsym(uint32_t e) { return (e >> 16) & 7u; }
+__host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return (e >> 19) & 31u; }
+
+struct Geometry {
+    int64_t N = 0, K = 0, n = 0, G = 0, GW = 0, KG = 0, NW = 0, nseg = 0, nchunk = 0;
+    static Geometry of(int64_t N, int64_t K);
+};
+
+}  // namespace uw
+
+struct uw_blob {
+    uint32_t magic = uw::kMagic;
+    uw::Geometry geo;
+    uint32_t forms = 0;
+    int64_t V = 0;
+    uint8_t palette[16] = {0};
+    uint8_t inv[256] = {0};
+    uint8_t code_len[16] = {0};
+    uint32_t code[16] = {0};
+    uint64_t freq[16] = {0};
+    uint64_t hist[256] = {0};
+    uint64_t total_bits = 0;
+    int64_t nwords = 0;
+    uint64_t off[UW_NSECT] = {0};
+    uint64_t bytes[UW_NSECT] = {0};
+    uint64_t dev_bytes = 0;
+    uint8_t* dev = nullptr;      // committed device image (caller-owned)
+    bool committed = false;
+    // compress-time host state (between query and commit)
+    std::vector<uint32_t> vbits_h, vpre_h;
+    std::vector<uint64_t> chunk_off_h;
+    std::vector<uint16_t> seg_rel_h;
+    std::vector<uint32_t> lut_h;
+
+    const uint8_t* sec(int s) const { return dev + off[s]; }
+};
+
+namespace uw {
+
+// ---- host helpers (uw_host.cpp)
+void build_code(const uint64_t freq[16], uint8_t len[16], uint32_t code[16]);
+void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut);
+void layout_sections(uw_blob* b);
+int num_sms();
+
+// ---- device status words (one per kernel translation unit)
+int decode_status_take();
+int gemm_status_take();
+
+// ---- compress kernels (uw_compress.cu)
+struct CompressScratch {
+    uint32_t* hist;     // [256]
+    uint32_t* freq;     // [16]
+    uint32_t* vbits;    // [GW]
+    uint32_t* segbits;  // [nseg]
+};
+size_t compress_scratch_bytes(const Geometry& g);
+CompressScratch carve_scratch(void* base, const Geometry& g);
+cudaError_t launch_histogram(const uint16_t* W, int64_t n, uint32_t* hist, cudaStream_t s);
+cudaError_t launch_verbatim_freq(const uint16_t* W, const Geometry& g, const uint8_t inv[256],
+                                 uint32_t* vbits, uint32_t* freq, cudaStream_t s);
+cudaError_t launch_segbits(const uint16_t* W, const Geometry& g, const uint8_t inv[256],
+                           const uint32_t* vbits, const uint8_t len[16], uint32_t* segbits,
+                           cudaStream_t s);
+cudaError_t launch_planes(const uint16_t* W, const Geometry& g, const uint8_t inv[256],
+                          const uint32_t* vbits, uint8_t* sm, uint8_t* idx, cudaStream_t s);
+cudaError_t launch_vexp(const uint16_t* W, const Geometry& g, const uint32_t* vbits,
+                        const uint32_t* vpre, uint8_t* vexp, cudaStream_t s);
+cudaError_t launch_vcol(const Geometry& g, const uint32_t* vbits, uint32_t* vcol, cudaStream_t s);
+cudaError_t launch_encode(const uint16_t* W, const Geometry& g, const uint8_t inv[256],
+                          const uint32_t* vbits, const uint8_t len[16], const uint32_t code[16],
+                          const uint64_t* chunk_off, const uint16_t* seg_rel, uint32_t* stream,
+                          int64_t nwords, cudaStream_t s);
+
+// ---- decoders (uw_decode.cu)
+enum DecodeMode { kDecodeFull = 0, kDecodeExponent = 1, kDecodeTranscode = 2 };
+cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s);
+int decode_ctas_per_sm();
+
+// ---- GEMM (uw_gemm.cu)
+enum GemmSource { kSrcDense = 0, kSrcExponent = 1, kSrcPalette = 2 };
+struct GemmArgs {
+    int src = kSrcDense;
+    const uint16_t* X = nullptr;
+    int64_t M = 0, N = 0, K = 0;
+    const uint16_t* W = nullptr;      // dense source
+    const uint8_t* sm = nullptr;      // sign+mantissa plane
+    const uint8_t* ex = nullptr;      // exponent plane (exponent source)
+    const uint8_t* idx = nullptr;     // index plane (palette source)
+    const uint32_t* vbits = nullptr;
+    const uint32_t* vpre = nullptr;
+    const uint8_t* vexp = nullptr;
+    const uint32_t* vcol = nullptr;
+    const uint8_t* palette = nullptr; // host array of 16
+    void* Y = nullptr;
+    int out_f32 = 0;
+    int grid = 0;
+    void* ws = nullptr;               // partial sums + tile counters
+    size_t ws_bytes = 0;
+};
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid);
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st);
+int gemm_default_grid();
+
+}  // namespace uw

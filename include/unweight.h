@@ -1,0 +1,244 @@
+/*
+ * unweight.h -- C ABI of libunweight: lossless BF16 weight compression with
+ * the decode fused into the matrix product, for NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described on the web page "Cloudflare推出Unweight無損壓縮
+ * 系統，將LLM模型大小壓縮15-22%" (easyvibecoding.app):
+ *   §BF16權重壓縮原理   each BF16 weight splits into a sign+mantissa byte, kept
+ *                       as is, and an exponent byte; exponents are Huffman
+ *                       coded or mapped to a 4-bit index into a per-matrix
+ *                       palette of the 16 most frequent exponents; a 64-weight
+ *                       row holding an exponent outside the palette is stored
+ *                       verbatim.
+ *   §四種執行管道       four pipelines: full decode + dense GEMM, exponent-only
+ *                       decode + reconstructive GEMM, palette transcode +
+ *                       reconstructive GEMM, direct palette GEMM.
+ *   §重建矩陣乘法核心運作 the reconstructive GEMM rebuilds BF16 tiles in shared
+ *                       memory and feeds them straight to the tensor cores.
+ *   §解壓與運算資源共享  decoder and GEMM may share the GPU, split by SMs.
+ *   §自動調優機制       an autotuner picks pipeline and SM split per projection
+ *                       and batch size by measurement.
+ *
+ * Conventions for every call:
+ *   - Pointers named *_dev / device buffers are device memory owned by the
+ *     caller; the library never allocates device memory.  Host pointers are
+ *     owned by the caller as well.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     Calls are asynchronous on that stream unless stated otherwise.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns a status and launches nothing.
+ *   - Device-detected problems (an undecodable stream, a bounded wait that
+ *     expired) set a device status word; read it with uw_last_device_status.
+ *   - Matrices are row-major.  W is [N, K] (output features x input features,
+ *     the nn.Linear layout), X is [M, K], Y is [M, N].  BF16 values are passed
+ *     as their 16-bit patterns (uint16_t).
+ *   - K must be a positive multiple of 64 and N*K at most 2^31 - 256.
+ */
+#ifndef UNWEIGHT_H
+#define UNWEIGHT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UW_OK = 0,
+    UW_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, misaligned pointer    */
+    UW_ERR_SHAPE = 2,        /* K % 64 != 0, K < 64, N < 1, N*K too large     */
+    UW_ERR_CORRUPT = 3,      /* serialized blob fails validation              */
+    UW_ERR_UNSUPPORTED = 4,  /* pipeline needs a form the blob does not hold  */
+    UW_ERR_WORKSPACE = 5,    /* buffer too small or misaligned                */
+    UW_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed             */
+    UW_ERR_TIMEOUT = 7,      /* a bounded device-side wait expired            */
+    UW_ERR_DEVICE = 8        /* a device-side check failed (bad stream data)  */
+} uw_status;
+
+/* The four pipelines of §四種執行管道. */
+typedef enum {
+    UW_PIPE_FULL = 0,            /* Huffman full decode -> BF16 W in workspace -> dense GEMM  */
+    UW_PIPE_EXPONENT = 1,        /* Huffman exponent decode -> E in workspace -> reconstructive GEMM */
+    UW_PIPE_TRANSCODE = 2,       /* Huffman -> 4-bit index plane in workspace -> reconstructive GEMM */
+    UW_PIPE_DIRECT_PALETTE = 3   /* reconstructive GEMM straight from the stored index plane */
+} uw_pipeline;
+
+/* Forms a compressed matrix may hold (bit mask). */
+enum { UW_FORM_HUFFMAN = 1, UW_FORM_PALETTE = 2 };
+
+/* Sections of a compressed matrix's device image. */
+typedef enum {
+    UW_SEC_SM = 0,        /* u8[N*K]  sign+mantissa bytes                          */
+    UW_SEC_VBITS = 1,     /* u32[ceil(G/32)] verbatim flag per 64-weight group     */
+    UW_SEC_VPRE = 2,      /* u32[ceil(G/32)] verbatim groups before word w         */
+    UW_SEC_VEXP = 3,      /* u8[V*64] raw exponents of verbatim groups             */
+    UW_SEC_VCOL = 4,      /* u32[(K/64)*4*ceil(N/128)] verbatim flags, by column   */
+    UW_SEC_IDX = 5,       /* u8[N*K/2] 4-bit palette indices (palette form)        */
+    UW_SEC_STREAM = 6,    /* u32[] Huffman stream, MSB first (Huffman form)        */
+    UW_SEC_CHUNK_OFF = 7, /* u64[ceil(nseg/16)] bit offset of symbol 4096c         */
+    UW_SEC_SEG_REL = 8,   /* u16[nseg] bit offset of symbol 256j minus chunk offset */
+    UW_SEC_LUT = 9,       /* u32[4096] derived multi-symbol decode table (not serialized) */
+    UW_NSECT = 10
+} uw_section;
+
+typedef struct uw_blob uw_blob;   /* opaque host handle of one compressed matrix */
+
+typedef struct {
+    int64_t N, K;             /* matrix shape                                         */
+    int64_t G;                /* 64-weight groups = N*K/64                             */
+    int64_t V;                /* verbatim groups                                       */
+    int64_t nseg, nchunk;     /* 256-symbol segments, 16-segment chunks                */
+    uint32_t forms;           /* UW_FORM_* held                                        */
+    uint8_t palette[16];      /* exponent of each palette index                        */
+    uint8_t code_len[16];     /* Huffman code length of each index (0 = unused)        */
+    uint64_t freq[16];        /* symbol counts                                         */
+    uint64_t hist[256];       /* exponent histogram                                    */
+    uint64_t total_bits;      /* Huffman stream length                                 */
+    uint64_t bytes_huffman_form;  /* sm + stream + offsets + verbatim store            */
+    uint64_t bytes_palette_form;  /* sm + idx + verbatim store + vcol                  */
+    uint64_t device_bytes;    /* size of the device image                              */
+    double mean_code_len;     /* bits per weight of the Huffman stream                 */
+    double exponent_entropy;  /* entropy of the exponent histogram, bits               */
+    double palette_coverage;  /* share of weights whose exponent is in the palette     */
+    uint64_t section_offset[UW_NSECT];  /* byte offset in the device image             */
+    uint64_t section_bytes[UW_NSECT];   /* byte length (0 = absent)                    */
+} uw_blob_info;
+
+typedef struct {
+    int32_t pipeline;        /* uw_pipeline                                               */
+    int32_t sm_dec;          /* >0: the Huffman decoder runs on sm_dec SMs beside the GEMM
+                                in one launch (§解壓與運算資源共享); 0: decode, then GEMM */
+    int32_t grid;            /* GEMM CTAs; 0 = one per SM                                  */
+    int32_t out_f32;         /* 0: Y is BF16 (round to nearest even); 1: Y is float32      */
+    void* workspace;         /* device, 256-byte aligned, zero-filled before first use;
+                                every call leaves it reusable                              */
+    size_t workspace_bytes;
+} uw_gemm_opts;
+
+/* One autotuner decision: best configuration for one projection and batch. */
+typedef struct {
+    int32_t blob_index;      /* which projection (index into the blobs array)  */
+    int64_t M;               /* batch size                                     */
+    int32_t pipeline;        /* chosen uw_pipeline                             */
+    int32_t sm_dec;          /* chosen decoder SM count                        */
+    int32_t grid;            /* chosen GEMM CTA count                          */
+    double us;               /* measured time of this projection, microseconds */
+} uw_plan_entry;
+
+/* ---------------------------------------------------------------- misc */
+
+/* Human-readable name of a status.  Never NULL. */
+const char* uw_status_str(int status);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int uw_version(void);
+
+/* Synchronizes `stream`, then returns and clears the device status word of
+ * the current device: UW_OK, UW_ERR_TIMEOUT or UW_ERR_DEVICE. */
+uw_status uw_last_device_status(void* stream);
+
+/* ---------------------------------------------------------------- compress
+ * Load-time compression (§BF16權重壓縮原理; "模型載入時預轉", §四種執行管道).
+ * Two steps so that the caller allocates the device image:
+ *   1. uw_compress_query analyses W (histogram, palette, verbatim groups,
+ *      Huffman code, segment offsets) and reports the image size;
+ *   2. uw_compress_commit writes every section into the caller's buffer.
+ * Both synchronize `stream`.  `scratch` is device memory of at least
+ * uw_compress_scratch_bytes(N, K), 256-byte aligned, used only during these
+ * calls.  W must stay unchanged between the two calls. */
+uw_status uw_compress_scratch_bytes(int64_t N, int64_t K, size_t* bytes);
+
+/* W_dev: device BF16 [N,K]; forms: UW_FORM_HUFFMAN | UW_FORM_PALETTE (nonzero).
+ * On success *out is a new handle (free with uw_blob_free) and *dev_bytes the
+ * size of the device image to allocate (256-byte aligned). */
+uw_status uw_compress_query(const uint16_t* W_dev, int64_t N, int64_t K, uint32_t forms,
+                            void* scratch, size_t scratch_bytes, void* stream,
+                            uw_blob** out, size_t* dev_bytes);
+
+/* dev_buf: device, 256-byte aligned, at least *dev_bytes from the query.  The
+ * handle keeps dev_buf; the caller keeps it alive while the handle is used. */
+uw_status uw_compress_commit(uw_blob* blob, const uint16_t* W_dev, void* scratch,
+                             size_t scratch_bytes, void* dev_buf, size_t dev_bytes, void* stream);
+
+/* Shape, palette, code, statistics and section table of a blob. */
+uw_status uw_blob_info_get(const uw_blob* blob, uw_blob_info* info);
+
+/* Device pointer and byte length of one section of a committed blob. */
+uw_status uw_blob_section(const uw_blob* blob, int section, const void** dev_ptr, size_t* bytes);
+
+/* Serialized size in bytes (header + format sections; the LUT is rebuilt on load). */
+uw_status uw_blob_serialized_bytes(const uw_blob* blob, size_t* bytes);
+
+/* Copies header and sections into host memory (synchronizes `stream`).  The
+ * result is the "distribution bundle" form of §Llama 3.1 8B測試結果. */
+uw_status uw_blob_serialize(const uw_blob* blob, void* host_dst, size_t cap, size_t* written,
+                            void* stream);
+
+/* Device image size needed to load a serialized blob (validates the header). */
+uw_status uw_blob_device_bytes(const void* host_src, size_t n, size_t* dev_bytes);
+
+/* Validates and loads a serialized blob into dev_buf (synchronizes `stream`).
+ * Returns UW_ERR_CORRUPT if any size, offset, code or count is inconsistent. */
+uw_status uw_blob_deserialize(const void* host_src, size_t n, void* dev_buf, size_t dev_bytes,
+                              void* stream, uw_blob** out);
+
+/* Frees the host handle only; device memory is the caller's. */
+void uw_blob_free(uw_blob* blob);
+
+/* ---------------------------------------------------------------- decode
+ * HBM-to-HBM decoders of the Huffman form (§四種執行管道).  A stream the
+ * decoder cannot parse sets UW_ERR_DEVICE in the device status word; output
+ * is then unspecified, but no access leaves the blob's sections or the output. */
+
+/* Full decode: W_out [N,K] BF16 bit patterns, bit-identical to the input of
+ * compression.  W_out 16-byte aligned. */
+uw_status uw_decode_full(const uw_blob* blob, uint16_t* W_out, void* stream);
+
+/* Exponent-only decode: E_out[N*K] = exponent byte of every weight (verbatim
+ * groups included).  E_out 16-byte aligned. */
+uw_status uw_decode_exponent(const uw_blob* blob, uint8_t* E_out, void* stream);
+
+/* Palette transcode: idx_out[N*K/2], byte-identical to the stored index
+ * plane of the palette form.  idx_out 16-byte aligned. */
+uw_status uw_transcode_palette(const uw_blob* blob, uint8_t* idx_out, void* stream);
+
+/* ---------------------------------------------------------------- GEMM
+ * Y[M,N] = X[M,K] . W^T with W given compressed (§重建矩陣乘法核心運作).
+ * X: device BF16 [M,K], 16-byte aligned; Y: device [M,N] BF16 or float32.
+ * M = 0 is a no-op.  Accumulation is float32 on the tensor cores. */
+
+/* Workspace bytes for uw_gemm with these options and M. */
+uw_status uw_gemm_workspace(const uw_blob* blob, int64_t M, const uw_gemm_opts* opts, size_t* bytes);
+
+uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* blob, void* Y,
+                  const uw_gemm_opts* opts, void* stream);
+
+/* The uncompressed baseline: the same tensor-core GEMM on a plain BF16 W. */
+uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int grid, size_t* bytes);
+
+uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K,
+                        void* Y, int out_f32, int grid, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------- autotune
+ * §自動調優機制: coordinate descent over (pipeline, sm_dec) for each
+ * projection, timing the whole sequence of projections with CUDA events:
+ * sweep projection 0 with the others fixed, then 1, then 2, ..., and repeat
+ * until a full round brings no improvement.  Done once per batch size in Ms.
+ *   blobs[i], X[i], Y[i]: projection i and device buffers for its input
+ *     (at least max(Ms) x K_i) and output (max(Ms) x N_i, BF16);
+ *   workspace: at least the largest uw_gemm_workspace over the candidates;
+ *   plan_out: nblobs * nM entries, written in (M, projection) order;
+ *   plan_json_path: if not NULL, the plan is also written there as JSON.
+ * Synchronizes `stream`. */
+uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const int64_t* Ms, int nM,
+                      const uint16_t* const* X, void* const* Y, void* workspace,
+                      size_t workspace_bytes, int reps, uw_plan_entry* plan_out,
+                      const char* plan_json_path, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNWEIGHT_H */

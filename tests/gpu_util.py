@@ -1,0 +1,50 @@
+"""Helpers shared by the GPU parity tests (marshalling only)."""
+import numpy as np
+import torch
+
+import synthetic as S
+
+
+def dev16(bits: np.ndarray) -> torch.Tensor:
+    """uint16 BF16 bit patterns -> CUDA bf16 tensor with the same bits."""
+    return torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def host8(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().numpy().view(np.uint8)
+
+
+def section_view(blob, name, dtype):
+    return host8(blob.section(name)).view(dtype)
+
+
+# GEMM tolerance.  The stated bound is a maximum relative error of 2e-3
+# against the fp32-accumulated reference over BF16 operands.  It applies
+# element-wise to float32 outputs, with a floor of 1e-2 * rms(R) so that
+# outputs near zero are judged against the matrix's scale.  A BF16 output
+# additionally carries its own rounding, up to 2^-8 relative (half an ulp of
+# an 8-bit significand).
+REL = 2e-3
+
+
+def check_gemm(Y: np.ndarray, R: np.ndarray, bf16_out: bool):
+    R = np.asarray(R, np.float64)
+    Y = np.asarray(Y, np.float64)
+    floor = 1e-2 * np.sqrt(np.mean(R * R)) if R.size else 0.0
+    tol = REL * np.maximum(np.abs(R), floor)
+    if bf16_out:
+        tol = tol + 2.0 ** -8 * np.abs(R)
+    err = np.abs(Y - R)
+    bad = err > tol
+    assert not bad.any(), (f"{int(bad.sum())} of {bad.size} outside tolerance; worst "
+                           f"{float((err / np.maximum(tol, 1e-30)).max()):.3g}x")
+    rel = float((err / np.maximum(np.abs(R), floor)).max()) if R.size else 0.0
+    return rel
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return S.bits_to_float(bits)

@@ -1,0 +1,149 @@
+"""GPU parity of Y = X . W^T through the four pipelines and the dense baseline
+against the CPU oracle's fp32-accumulated (and fp64) reference.
+
+Tolerance (see tests/gpu_util.py): max relative error 2e-3 element-wise with a
+1e-2*rms floor on float32 outputs, plus 2^-8 relative BF16 output rounding on
+BF16 outputs.  The rebuilt weights are bit-exact, so pipelines that share the
+tiling and split must also agree bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_gemm_bf16_b200 as uw
+import synthetic as S
+from oracle import oracle as O
+from tests.gpu_util import check_gemm, dev16, host16
+
+pytestmark = pytest.mark.gpu
+
+PIPES = ["full", "exponent", "transcode", "direct_palette"]
+
+SHAPES = {
+    # N x K: several 128-row tiles and 64-wide k steps, ragged N, verbatim rows
+    "384x512": lambda: S.weight_with_verbatim_rows(384, 512, seed=31, frac_groups=0.01),
+    "200x1408": lambda: S.weight_with_verbatim_rows(200, 1408, seed=32, frac_groups=0.01),
+}
+MS = [1, 3, 16, 17, 64, 100, 256, 300]
+
+_cache = {}
+
+
+def _case(shape):
+    if shape not in _cache:
+        W = SHAPES[shape]()
+        blob = uw.uw_compress(dev16(W))
+        _cache[shape] = (W, blob)
+    return _cache[shape]
+
+
+def _f32(t):
+    return t.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+@pytest.mark.parametrize("M", MS)
+def test_pipelines_match_oracle(shape, M):
+    W, blob = _case(shape)
+    X = S.activations(M, W.shape[1], seed=1000 + M)
+    R32 = O.gemm(X, W, "f32")
+    R64 = O.gemm(X, W, "f64")
+    Xd = dev16(X)
+    outs = {}
+    for pipe in PIPES:
+        Y32 = uw.uw_gemm(Xd, blob, pipe, out_f32=True)
+        Yb = uw.uw_gemm(Xd, blob, pipe, out_f32=False)
+        torch.cuda.synchronize()
+        check_gemm(_f32(Y32), R32, bf16_out=False)
+        check_gemm(_f32(Y32), R64, bf16_out=False)
+        check_gemm(_f32(Yb), R32, bf16_out=True)
+        outs[pipe] = (_f32(Y32), host16(Yb))
+    Yd = _f32(uw.uw_dense_gemm(Xd, dev16(W), out_f32=True))
+    check_gemm(Yd, R32, bf16_out=False)
+    for pipe in PIPES:
+        assert np.array_equal(outs[pipe][0], Yd), pipe        # same tiles, same split
+        assert np.array_equal(outs[pipe][1], outs["full"][1]), pipe
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("grid", [1, 2, 7, 33, 500])
+def test_stream_k_splits(grid):
+    """Different CTA counts cut the k loop differently; all must match."""
+    W, blob = _case("384x512")
+    X = S.activations(40, 512, seed=77)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    for pipe in ["exponent", "direct_palette"]:
+        Y = uw.uw_gemm(Xd, blob, pipe, out_f32=True, grid=grid)
+        check_gemm(_f32(Y), R, bf16_out=False)
+    Yd = uw.uw_dense_gemm(Xd, dev16(W), out_f32=True, grid=grid)
+    check_gemm(_f32(Yd), R, bf16_out=False)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_repeated_calls_reuse_workspace():
+    W, blob = _case("200x1408")
+    X = S.activations(17, 1408, seed=5)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    first = None
+    for _ in range(4):
+        Y = _f32(uw.uw_gemm(Xd, blob, "transcode", out_f32=True, grid=13))
+        check_gemm(Y, R, bf16_out=False)
+        if first is None:
+            first = Y
+        assert np.array_equal(Y, first)
+
+
+def test_empty_batch_and_errors():
+    W, blob = _case("384x512")
+    Y = torch.empty(0, 384, dtype=torch.bfloat16, device="cuda")
+    out = uw.uw_gemm(torch.empty(0, 512, dtype=torch.bfloat16, device="cuda"), blob, "exponent", out=Y)
+    assert out.shape == (0, 384)
+    bh = uw.uw_compress(dev16(W), forms=uw.UW_FORM_HUFFMAN)
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm(dev16(S.activations(2, 512, 1)), bh, "direct_palette")
+    assert ei.value.status == 4
+    small = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm(dev16(S.activations(2, 512, 1)), blob, "full", ws=small)
+    assert ei.value.status == 5
+
+
+def _sampled(X, W, Y, n_samples, seed, bf16_out):
+    rng = np.random.default_rng(seed)
+    M, N = Y.shape
+    ms = rng.integers(0, M, n_samples)
+    ns = rng.integers(0, N, n_samples)
+    ref = np.array([O.gemm_one(X, W, int(m), int(n), "f32") for m, n in zip(ms, ns)])
+    # floor from the sampled references' scale
+    check_gemm(Y[ms, ns], ref, bf16_out=bf16_out)
+
+
+@pytest.mark.parametrize("M", [1, 64])
+def test_full_size_gate_sampled(M):
+    W = S.gate_projection()
+    blob = uw.uw_compress(dev16(W))
+    X = S.activations(M, 4096, seed=1 + S.X_SEED_OFFSET)
+    Xd = dev16(X)
+    ref = None
+    for pipe in PIPES:
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
+        _sampled(X, W, Y, 256, seed=M, bf16_out=True)
+        if ref is None:
+            ref = Y
+        assert np.array_equal(Y, ref), pipe
+    Yd = _f32(uw.uw_dense_gemm(Xd, dev16(W)))
+    assert np.array_equal(Yd, ref)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_full_size_down_sampled():
+    W = S.down_projection()
+    blob = uw.uw_compress(dev16(W))
+    X = S.activations(256, 14336, seed=4 + S.X_SEED_OFFSET)
+    Xd = dev16(X)
+    for pipe in ["exponent", "direct_palette"]:
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
+        _sampled(X, W, Y, 128, seed=3, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
