@@ -254,7 +254,7 @@ _ws_cache = {}
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
-    """A zero-filled workspace of at least nbytes (cached; calls leave it reusable)."""
+    """A device workspace of at least nbytes, cached per device (contents do not matter)."""
     key = (str(device),)
     t = _ws_cache.get(key)
     if t is None or t.numel() < nbytes:

@@ -27,8 +27,10 @@
 //     long-K down projection with the same kernel;
 //   * every wait is bounded (globaltimer deadline); on expiry the CTA raises
 //     UW_ERR_TIMEOUT, drains its own TMA and MMA work, frees TMEM and exits.
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
+#include <random>
 
 #include "uw_device.cuh"
 #include "uw_internal.h"
@@ -63,10 +65,26 @@ struct GemmParams {
     uint32_t pal[4];
     void* Y;
     int out_f32;
-    float* partial;     // [2P][MG][128]
-    int* counters;      // [tiles][128]
+    float* partial;                // [2P][MG][128]
+    unsigned long long* counters;  // [tiles][128]: (epoch << 16) | arrivals
+    unsigned long long epoch;      // 48-bit tag of this call
     uint64_t timeout_ns;
 };
+
+// Counts one arrival at a stream-K fix-up counter and returns the number of
+// arrivals of this call so far.  The word holds (epoch << 16) | count; a word
+// carrying another call's tag (or any stale bytes left in the workspace) is
+// taken as a count of 0, so the workspace never needs clearing.
+__device__ __forceinline__ unsigned arrive_counter(unsigned long long* cnt, unsigned long long epoch) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+    for (;;) {
+        unsigned long long base = (cur >> 16) == epoch ? cur : (epoch << 16);
+        unsigned long long nxt = base + 1;
+        unsigned long long prev = atomicCAS(cnt, cur, nxt);
+        if (prev == cur) return (unsigned)(nxt & 0xFFFFu);
+        cur = prev;
+    }
+}
 
 __host__ __device__ __forceinline__ int64_t iter_begin(int64_t b, int64_t total, int64_t P) {
     return b * total / P;
@@ -338,9 +356,8 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                 const int64_t b_last = iter_owner(t1, p.total_iters, p.P);
                 const int nsegs = (int)(b_last - b_first + 1);
                 __threadfence();
-                int* cnt = p.counters + sg.tile * kBlockN + r;
-                int old = atomicAdd(cnt, 1);
-                if (old == nsegs - 1) {
+                unsigned long long* cnt = p.counters + sg.tile * kBlockN + r;
+                if (arrive_counter(cnt, p.epoch) == (unsigned)nsegs) {
                     __threadfence();
                     for (int c = 0; c < p.MG; c++) {
                         int64_t m = m0 + c;
@@ -355,7 +372,7 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                             else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc);
                         }
                     }
-                    *cnt = 0;
+                    *cnt = p.epoch << 16;   // count back to 0 for a replay of this call
                 }
             }
             j++;
@@ -410,6 +427,16 @@ int pick_mg(int64_t M) {
     return (int)mg;
 }
 
+// 48-bit call tags: a per-process random base plus a running count.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> ctr{0};
+    static const unsigned long long base = [] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 20) ^ (unsigned long long)rd();
+    }();
+    return (base + ctr.fetch_add(1)) & 0xFFFFFFFFFFFFull;
+}
+
 uint64_t timeout_ns() {
     static uint64_t t = 0;
     if (!t) {
@@ -433,7 +460,7 @@ size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
     int MG = pick_mg(M);
     int64_t m_tiles = (M + MG - 1) / MG, n_tiles = (N + kBlockN - 1) / kBlockN;
     size_t part = (size_t)2 * P * MG * kBlockN * 4;
-    size_t cnt = (size_t)m_tiles * n_tiles * kBlockN * 4;
+    size_t cnt = (size_t)m_tiles * n_tiles * kBlockN * 8;
     return ((part + 255) & ~size_t(255)) + ((cnt + 255) & ~size_t(255));
 }
 
@@ -467,7 +494,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
     size_t part = (size_t)2 * P * p.MG * kBlockN * 4;
     p.partial = (float*)a.ws;
-    p.counters = (int*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
+    p.counters = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
+    p.epoch = next_epoch();
     p.timeout_ns = timeout_ns();
 
     // stage layout

@@ -111,8 +111,8 @@ typedef struct {
                                 in one launch (§解壓與運算資源共享); 0: decode, then GEMM */
     int32_t grid;            /* GEMM CTAs; 0 = one per SM                                  */
     int32_t out_f32;         /* 0: Y is BF16 (round to nearest even); 1: Y is float32      */
-    void* workspace;         /* device, 256-byte aligned, zero-filled before first use;
-                                every call leaves it reusable                              */
+    void* workspace;         /* device, 256-byte aligned, any contents; a call owns it
+                                until it completes (one workspace per stream)              */
     size_t workspace_bytes;
 } uw_gemm_opts;
 

@@ -147,3 +147,26 @@ def test_full_size_down_sampled():
         Y = _f32(uw.uw_gemm(Xd, blob, pipe))
         _sampled(X, W, Y, 128, seed=3, bf16_out=True)
     assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, "random"])
+def test_workspace_contents_do_not_matter(fill):
+    """Fix-up counters carry a per-call tag, so stale bytes left in the
+    workspace by other calls (other pipelines, other layouts) are harmless."""
+    W, blob = _case("384x512")
+    X = S.activations(33, 512, seed=9)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    need = max(uw.uw_gemm_workspace(blob, 33, p) for p in PIPES)
+    ws = torch.empty(need + 4096, dtype=torch.uint8, device="cuda")
+    for pipe in PIPES + ["dense"]:
+        if fill == "random":
+            ws.random_(0, 256)
+        else:
+            ws.fill_(fill)
+        if pipe == "dense":
+            Y = uw.uw_dense_gemm(Xd, dev16(W), out_f32=True, ws=ws)
+        else:
+            Y = uw.uw_gemm(Xd, blob, pipe, out_f32=True, ws=ws)
+        check_gemm(_f32(Y), R, bf16_out=False)
+    assert uw.uw_last_device_status() == 0
