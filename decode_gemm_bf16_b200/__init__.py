@@ -35,7 +35,7 @@ EXPORTS = ["uw_status_str", "uw_version", "uw_last_device_status", "uw_compress_
            "uw_blob_serialized_bytes", "uw_blob_serialize", "uw_blob_device_bytes",
            "uw_blob_deserialize", "uw_blob_free", "uw_decode_full", "uw_decode_exponent",
            "uw_transcode_palette", "uw_gemm_workspace", "uw_gemm", "uw_dense_gemm_workspace",
-           "uw_dense_gemm", "uw_autotune"]
+           "uw_dense_gemm", "uw_autotune", "uw_gemm_direct_palette_noalloc"]
 
 
 class UnweightError(RuntimeError):
@@ -100,6 +100,7 @@ def lib():
             "uw_gemm": ([P, I64, P, P, ctypes.POINTER(GemmOpts), P], I32),
             "uw_dense_gemm_workspace": ([I64, I64, I64, I32, ctypes.POINTER(SZ)], I32),
             "uw_dense_gemm": ([P, I64, P, I64, I64, P, I32, I32, P, SZ, P], I32),
+            "uw_gemm_direct_palette_noalloc": ([P, I64, P, P, I32, P], I32),
             "uw_autotune": ([ctypes.POINTER(P), I32, ctypes.POINTER(I64), I32, ctypes.POINTER(P),
                              ctypes.POINTER(P), P, SZ, I32, ctypes.POINTER(PlanEntry), ctypes.c_char_p, P], I32),
         }
@@ -275,6 +276,20 @@ def uw_gemm(X: torch.Tensor, blob: Blob, pipeline="direct_palette", out: Optiona
         ws = workspace(uw_gemm_workspace(blob, M, pipeline, sm_dec, grid), X.device)
     o = _opts(pipeline, sm_dec, grid, out_f32, ws)
     _check(lib().uw_gemm(_ptr(X), M, blob.handle, _ptr(out), ctypes.byref(o), _stream(stream)), "uw_gemm")
+    return out
+
+
+def uw_gemm_direct_palette_noalloc(X: torch.Tensor, blob: Blob, out: Optional[torch.Tensor] = None,
+                                   out_f32: bool = False, stream=None) -> torch.Tensor:
+    """Direct-palette GEMM whose scratch is a fixed array inside the library,
+    for callers that cannot allocate device memory at call time (see the
+    header).  `out` should be preallocated by such callers."""
+    X = _bits16(X)
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, blob.N, dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
+    _check(lib().uw_gemm_direct_palette_noalloc(_ptr(X), M, blob.handle, _ptr(out), 1 if out_f32 else 0,
+                                                _stream(stream)), "uw_gemm_direct_palette_noalloc")
     return out
 
 

@@ -30,6 +30,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 #include <random>
 
 #include "uw_device.cuh"
@@ -571,3 +572,86 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
 }
 
 }  // namespace uw
+
+// ===========================================================================
+// Allocation-free variant of the direct-palette GEMM.
+//
+// Some callers cannot allocate device memory when they call the GEMM: engines
+// that reserve all memory at start-up and forbid later allocation, code that
+// must not risk the implicit device synchronisation of cudaMalloc/cudaFree,
+// and plugins whose host framework owns the allocator.  For them the stream-K
+// fix-up scratch (partial sums and per-row arrival tags) lives in the fixed
+// array below, compiled into the library: 4 MiB on every GPU that loads the
+// library, held until the process exits.  That covers batches up to 16 on a
+// 148-SM B200 for N up to about 200k rows.
+// ===========================================================================
+namespace uw {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name of the array is not a device address).
+void* noalloc_scratch(uw_status* st) {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        *st = UW_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            *st = UW_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+}  // namespace uw
+
+extern "C" uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M, const uw_blob* b, void* Y,
+                                                    int out_f32, void* stream) {
+    using namespace uw;
+    if (!b || b->magic != kMagic || !b->committed || M < 0) return UW_ERR_INVALID_ARG;
+    if (!(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
+    if (M == 0) return UW_OK;
+    if (!X || !Y || ((uintptr_t)X & 15) || ((uintptr_t)Y & 15)) return UW_ERR_INVALID_ARG;
+    if (gemm_ws_bytes(M, b->geo.N, b->geo.K, 0) > kNoAllocScratchBytes) return UW_ERR_WORKSPACE;
+    uw_status st = UW_OK;
+    void* scratch = noalloc_scratch(&st);
+    if (!scratch) return st;
+    GemmArgs a;
+    a.src = kSrcPalette;
+    a.X = X;
+    a.M = M;
+    a.N = b->geo.N;
+    a.K = b->geo.K;
+    a.sm = b->sec(UW_SEC_SM);
+    a.idx = b->sec(UW_SEC_IDX);
+    a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
+    a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
+    a.vexp = b->sec(UW_SEC_VEXP);
+    a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
+    a.palette = b->palette;
+    a.Y = Y;
+    a.out_f32 = out_f32 ? 1 : 0;
+    a.grid = 0;
+    a.ws = scratch;
+    a.ws_bytes = kNoAllocScratchBytes;
+    cudaError_t e = launch_gemm(a, (cudaStream_t)stream, &st);
+    if (st) return st;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return UW_ERR_CUDA;
+    }
+    return UW_OK;
+}

@@ -221,6 +221,29 @@ uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t
                         void* Y, int out_f32, int grid, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* ---------------------------------------------------------------- allocation-free GEMM
+ * An addition of this library; the pages have no counterpart.
+ *
+ * uw_gemm with the direct-palette pipeline for callers that cannot allocate
+ * device memory at call time: engines that reserve all memory at start-up and
+ * forbid allocation afterwards, code that must not risk the implicit device
+ * synchronisation of cudaMalloc/cudaFree, plugins whose host framework owns
+ * the allocator.  Its scratch (stream-K partial sums and arrival tags) is a
+ * fixed 4 MiB array inside the library, present on every GPU that loads the
+ * library until the process exits; no workspace argument, no allocation.
+ *   X: device BF16 [M,K], 16-byte aligned; Y: device [M,N], BF16 or float32
+ *   (out_f32), 16-byte aligned; the blob must hold the palette form.
+ * Limits: returns UW_ERR_WORKSPACE, launching nothing, when the scratch this
+ * call needs exceeds 4 MiB (on a 148-SM B200 that admits M <= 16 for N up to
+ * about 200k rows).  The array's contents carry over from call to call; they
+ * need no clearing because every entry is tagged with its call.  All calls
+ * share the one array, so calls that overlap on the GPU (other streams,
+ * other threads) race: run them one at a time.  The first call on a device
+ * looks the array's device address up (cudaGetSymbolAddress); make that first
+ * call before any stream capture. */
+uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M, const uw_blob* blob, void* Y,
+                                         int out_f32, void* stream);
+
 /* ---------------------------------------------------------------- autotune
  * §自動調優機制: coordinate descent over (pipeline, sm_dec) for each
  * projection, timing the whole sequence of projections with CUDA events:
