@@ -16,6 +16,7 @@ same workload and prints the same metric.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import subprocess
@@ -55,7 +56,7 @@ class Clocks:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index),
-                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "--query-gpu=timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
@@ -72,18 +73,33 @@ class Clocks:
                 self.proc.kill()
             self.f.close()
 
+    def mark(self, which: str):
+        setattr(self, which, datetime.datetime.now())
+
     def summary(self):
+        """Median SM clock and active throttle reasons over the samples taken
+        between mark('t0') and mark('t1')."""
         try:
-            rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+            rows = [[c.strip() for c in l.split(",")] for l in open(self.path).read().strip().splitlines()
+                    if l.strip()]
         except Exception:
             rows = []
-        if not rows:
+        t0, t1 = getattr(self, "t0", None), getattr(self, "t1", None)
+        sel = []
+        for r in rows:
+            try:
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f")
+            except Exception:
+                continue
+            if t0 is None or t1 is None or t0 <= ts <= t1:
+                sel.append(r)
+        if not sel:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = sorted(float(r[1]) for r in rows)
-        mx = max(float(r[2]) for r in rows)
+        sm = sorted(float(r[1]) for r in sel)
+        mx = max(float(r[2]) for r in sel)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in sel for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(sel)}
 
 
 def _dist():
@@ -197,37 +213,51 @@ def run_gpu(args):
             uw.uw_gemm(xin, blob, k - 3, out=Ys[k - 3], ws=ws)
 
     nops = len(OPS)
-    ctr = [0]
+    ncopy = len(copies)
+    cap = torch.cuda.Stream(device=dev)
 
-    def step(xin, ev=None):
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+        return g
+
+    # every op once eagerly (sets kernel attributes), then one graph per
+    # rotation of the weight copies: step r runs op k on copy (r + k) % 4
+    with torch.cuda.stream(cap):
         for k in range(nops):
-            blob = copies[ctr[0] % len(copies)]
-            ctr[0] += 1
-            if ev is not None:
-                ev[k][0].record(stream)
-            op(k, blob, xin)
-            if ev is not None:
-                ev[k][1].record(stream)
+            op(k, copies[k % ncopy], xd)
+    torch.cuda.synchronize()
+    step_graphs = [capture(lambda r=r: [op(k, copies[(r + k) % ncopy], xd) for k in range(nops)])
+                   for r in range(ncopy)]
+    op_graphs = [[capture(lambda k=k, c=c: op(k, copies[c], xd)) for c in range(ncopy)] for k in range(nops)]
 
-    for _ in range(max(3, args.warmup)):
-        step(xd)
+    # warm-up: W steps, and at least half a second of work so the clocks settle
+    t_w = time.time()
+    i = 0
+    while i < max(3, args.warmup) or time.time() - t_w < 0.5:
+        step_graphs[i % ncopy].replay()
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
-    # ---- timed region (device time, CUDA events on the launching stream)
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nops)]
-           for _ in range(args.steps)]
+    # ---- timed region: K steps (graph replays), device time with CUDA events
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with Clocks(local) as clk:
+        time.sleep(0.3)           # let the sampler start
+        clk.mark("t0")
         t0.record(stream)
         for i in range(args.steps):
-            step(xd, evs[i])
+            step_graphs[i % ncopy].replay()
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark("t1")
     if dist:
         dist.barrier()
     ms = t0.elapsed_time(t1)
@@ -235,8 +265,19 @@ def run_gpu(args):
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
-    per_op_ms = [sum(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(args.steps)) / args.steps
-                 for k in range(nops)]
+    # per-op device time: each op alone, rotated over the copies
+    reps = max(40, min(400, args.steps // 5))
+    per_op_ms = []
+    for k in range(nops):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(8):
+            op_graphs[k][i % ncopy].replay()
+        a.record(stream)
+        for i in range(reps):
+            op_graphs[k][i % ncopy].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per_op_ms.append(a.elapsed_time(b) / reps)
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
 
@@ -245,11 +286,16 @@ def run_gpu(args):
     yh = [torch.empty(M_X, N_W, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
     xdev = torch.empty_like(xd)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k in range(nops):
+        op(k, copies[k % ncopy], xdev)
     torch.cuda.synchronize()
     e0.record(stream)
+    ctr = 0
     for i in range(args.steps):
         xdev.copy_(xh, non_blocking=True)
-        step(xdev)
+        for k in range(nops):
+            op(k, copies[ctr % ncopy], xdev)
+            ctr += 1
         for j in range(4):
             yh[j].copy_(Ys[j], non_blocking=True)
     e1.record(stream)
@@ -330,7 +376,7 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")

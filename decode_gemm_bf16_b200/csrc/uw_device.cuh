@@ -45,6 +45,14 @@ __device__ __forceinline__ uint32_t palette4(uint32_t x, uint32_t P0, uint32_t P
     return (lo & ~m) | (hi & m);
 }
 
+// Same lookup when all 16 palette exponents are below 128 (|w| < 2): the
+// out-of-range half of each prmt then yields 0x00 by sign replication, so
+// the two halves combine with an OR.  xs = x ^ 0x8888 (shared per word).
+__device__ __forceinline__ uint32_t palette4_small(uint32_t x, uint32_t xs, uint32_t P0, uint32_t P1,
+                                                   uint32_t P2, uint32_t P3) {
+    return prmt(P0, P1, x) | prmt(P2, P3, xs);
+}
+
 // Four exponent bytes E and four sign+mantissa bytes S -> four BF16 values
 // (two words): bf16 = (s<<15) | (e<<7) | m with S = s<<7 | m.
 __device__ __forceinline__ uint2 merge4(uint32_t E, uint32_t S) {
@@ -74,14 +82,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Test for completion of the phase with the given parity; a thread whose
+// phase is not complete may be suspended for up to `hint_ns` (it wakes as soon
+// as the phase completes), so waiting roles do not steal issue slots.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
@@ -91,11 +102,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // stay cheap) or when another role of the CTA raised *abort (if given).  On
 // expiry *abort is raised.  Never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint32_t hint_ns = 1000) {
     uint64_t deadline = 0;
     for (uint32_t i = 0;; i++) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 63u) {
+        if (mbar_try_wait(bar, parity, hint_ns)) return true;
+        if ((i & 7u) == 7u) {
             if (abort && *abort) return false;
             uint64_t now = globaltimer();
             if (deadline == 0) {
@@ -156,6 +167,29 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A read from tensor memory
+// (row i of A in TMEM lane i, K elements 2j, 2j+1 in column j, low half first).
+__device__ __forceinline__ void tc_mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 TMEM lanes x 16 consecutive 32-bit columns <- 16 registers per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {

@@ -18,8 +18,14 @@
 //     holds only the stage ring;
 //   * warp roles: warps 0-3 epilogue (TMEM lanes 32w..32w+31), warp 4 TMA
 //     producer, warp 5 allocates TMEM and issues tcgen05.mma (one thread),
-//     warps 6-13 rebuild BF16 tiles in the 128-byte swizzled K-major layout the
-//     MMA descriptor expects;
+//     warps 6-13 rebuild BF16 rows;
+//   * the rebuilt tile never touches shared memory: each rebuild thread owns
+//     one weight row (one TMEM lane) and half of the 64-wide k step, reads its
+//     sign+mantissa and index bytes from TMA tiles staged with a 64/32-byte
+//     swizzle (conflict-free row-per-lane reads), and writes 16 columns of BF16
+//     pairs into tensor memory with tcgen05.st; the MMA reads A from TMEM.
+//     Shared memory then carries 3 bytes per weight (TMA write + one read)
+//     instead of 7, and holds no A tiles;
 //   * stream-K: the (tile, 64-wide k step) iterations are split evenly over one
 //     CTA per SM; tiles cut between CTAs are finished by the last CTA to
 //     arrive, per output row, summing fp32 partials in CTA order
@@ -49,7 +55,7 @@ constexpr int kReconWarps = 8;
 constexpr int kMaxStages = 8;
 constexpr int kThreadsDense = 6 * 32;
 constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
-constexpr uint32_t kTileA = kBlockN * kBlockK * 2;       // 16 KB rebuilt / loaded BF16 tile
+constexpr uint32_t kTileA = kBlockN * kBlockK * 2;       // 16 KB BF16 weight tile (dense source)
 constexpr uint32_t kTileSM = kBlockN * kBlockK;          //  8 KB sign+mantissa
 constexpr uint32_t kTileE = kBlockN * kBlockK;           //  8 KB exponents
 constexpr uint32_t kTileIdx = kBlockN * kBlockK / 2;     //  4 KB palette indices
@@ -59,14 +65,17 @@ struct GemmParams {
     int64_t M, N, K, KG;
     int MG, m_tiles, n_tiles, kt_count, P, stages;
     int64_t total_iters;
-    uint32_t stage_bytes, off_b, off_sm, off_s2, off_v, tx_bytes;
+    uint32_t stage_bytes, off_a, off_b, off_sm, off_s2, off_v, tx_bytes;
+    uint32_t tmem_cols;   // TMEM columns allocated (power of two)
+    uint32_t a_col0;      // first TMEM column of the rebuilt-A stages (32 columns each)
+    int pal_small;        // all palette exponents < 128: cheaper lookup
     const uint32_t* vbits;
     const uint32_t* vpre;
     const uint8_t* vexp;
     uint32_t pal[4];
     void* Y;
     int out_f32;
-    float* partial;                // [2P][MG][128]
+    float* partial;                // [2P][128][MG]
     unsigned long long* counters;  // [tiles][128]: (epoch << 16) | arrivals
     unsigned long long epoch;      // 48-bit tag of this call
     uint64_t timeout_ns;
@@ -123,44 +132,69 @@ struct SegWalker {
     }
 };
 
+// Offsets of 16-byte chunk c of row r in TMA tiles stored with a 64-byte
+// (rows of 64 B) or 32-byte (rows of 32 B) swizzle: chunk bits XOR address
+// bits 7 and up.
+__device__ __forceinline__ uint32_t sw64_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+__device__ __forceinline__ uint32_t sw32_off(int r, int c) { return r * 32 + ((c ^ ((r >> 2) & 1)) << 4); }
+
+// Rebuilds weight row r = 32q + lane, k = 32h .. 32h+31 of the stage's tile
+// and writes it to TMEM lane r, columns taddr_cols .. +15 (one BF16 pair per
+// column).
 template <int SRC>
-__device__ __forceinline__ void reconstruct_tile(const GemmParams& p, uint8_t* stage, int64_t n0,
-                                                 int kt, int t /*0..255*/) {
-    uint8_t* A = stage;
+__device__ __forceinline__ void rebuild_row(const GemmParams& p, const uint8_t* stage, int64_t n0, int kt,
+                                            int q, int h, int lane, uint32_t taddr) {
+    const int r = 32 * q + lane;
     const uint8_t* SM = stage + p.off_sm;
-    const uint8_t* S2 = stage + p.off_s2;
-    uint4 vc = make_uint4(0, 0, 0, 0);
-    if (SRC == kSrcPalette) vc = *reinterpret_cast<const uint4*>(stage + p.off_v);
-    const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const int r = (t >> 3) + 32 * i;   // tile row
-        const int c = t & 7;               // 8-weight chunk within the 64-wide row
-        uint2 s = *reinterpret_cast<const uint2*>(SM + r * 64 + c * 8);
-        uint32_t e0, e1;
-        if (SRC == kSrcExponent) {
-            uint2 e = *reinterpret_cast<const uint2*>(S2 + r * 64 + c * 8);
-            e0 = e.x;
-            e1 = e.y;
+    const uint4 s0 = *reinterpret_cast<const uint4*>(SM + sw64_off(r, 2 * h));
+    const uint4 s1 = *reinterpret_cast<const uint4*>(SM + sw64_off(r, 2 * h + 1));
+    uint32_t E[8];
+    if (SRC == kSrcExponent) {
+        const uint8_t* EX = stage + p.off_s2;
+        const uint4 e0 = *reinterpret_cast<const uint4*>(EX + sw64_off(r, 2 * h));
+        const uint4 e1 = *reinterpret_cast<const uint4*>(EX + sw64_off(r, 2 * h + 1));
+        E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
+        E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
+    } else {
+        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + p.off_v + 4 * q);
+        if ((vw >> lane) & 1u) {
+            // verbatim group: raw exponents from the verbatim store
+            const int64_t g = (n0 + r) * p.KG + kt;
+            const uint32_t w = __ldg(&p.vbits[g >> 5]);
+            const int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
+            const uint4* src = reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + 32 * h);
+            const uint4 e0 = __ldg(src), e1 = __ldg(src + 1);
+            E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
+            E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
         } else {
-            uint32_t vw = i == 0 ? vc.x : i == 1 ? vc.y : i == 2 ? vc.z : vc.w;
-            if ((vw >> (r & 31)) & 1u) {
-                // verbatim group: raw exponents from the verbatim store
-                int64_t g = (n0 + r) * p.KG + kt;
-                uint32_t w = __ldg(&p.vbits[g >> 5]);
-                int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
-                uint2 e = __ldg(reinterpret_cast<const uint2*>(p.vexp + rank * kGroup + c * 8));
-                e0 = e.x;
-                e1 = e.y;
+            const uint4 ix = *reinterpret_cast<const uint4*>(stage + p.off_s2 + sw32_off(r, h));
+            const uint32_t w[4] = {ix.x, ix.y, ix.z, ix.w};
+            const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
+            if (p.pal_small) {
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const uint32_t xs = w[j] ^ 0x88888888u;
+                    E[2 * j] = palette4_small(w[j], xs, P0, P1, P2, P3);
+                    E[2 * j + 1] = palette4_small(w[j] >> 16, xs >> 16, P0, P1, P2, P3);
+                }
             } else {
-                uint32_t ix = *reinterpret_cast<const uint32_t*>(S2 + r * 32 + c * 4);
-                e0 = palette4(ix, P0, P1, P2, P3);
-                e1 = palette4(ix >> 16, P0, P1, P2, P3);
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    E[2 * j] = palette4(w[j], P0, P1, P2, P3);
+                    E[2 * j + 1] = palette4(w[j] >> 16, P0, P1, P2, P3);
+                }
             }
         }
-        uint2 a = merge4(e0, s.x), b = merge4(e1, s.y);
-        *reinterpret_cast<uint4*>(A + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
     }
+    const uint32_t S[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    uint32_t out[16];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const uint2 m = merge4(E[j], S[j]);
+        out[2 * j] = m.x;
+        out[2 * j + 1] = m.y;
+    }
+    tmem_st16(taddr, out);
 }
 
 __device__ __forceinline__ uint16_t f2bf(float f) {
@@ -188,7 +222,7 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem_cols = p.MG <= 32 ? 32u : p.MG <= 64 ? 64u : p.MG <= 128 ? 128u : 256u;
+    const uint32_t tmem_cols = p.tmem_cols;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
@@ -238,7 +272,7 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
                     tma_load_2d(st + p.off_b, &tm_x, kt * kBlockK, m_tile * p.MG, fb);
                     if (SRC == kSrcDense) {
-                        tma_load_2d(st, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
+                        tma_load_2d(st + p.off_a, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
                     } else {
                         tma_load_2d(st + p.off_sm, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
                         if (SRC == kSrcExponent)
@@ -277,9 +311,14 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                     const uint32_t st = smem_base + s * p.stage_bytes;
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; kk++) {
-                        uint64_t ad = sw128_desc(st + kk * 32);
-                        uint64_t bd = sw128_desc(st + p.off_b + kk * 32);
-                        tc_mma(tacc, ad, bd, idesc, (kt > sg.kt0 || kk > 0) ? 1u : 0u);
+                        const uint64_t bd = sw128_desc(st + p.off_b + kk * 32);
+                        const uint32_t acc = (kt > sg.kt0 || kk > 0) ? 1u : 0u;
+                        if (kRecon) {
+                            // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
+                            tc_mma_tmem_a(tacc, tacc + p.a_col0 + 32u * (uint32_t)s + 8u * kk, bd, idesc, acc);
+                        } else {
+                            tc_mma(tacc, sw128_desc(st + p.off_a + kk * 32), bd, idesc, acc);
+                        }
                     }
                     tc_commit(smem_u32(&empty_bar[s]));
                 }
@@ -294,7 +333,10 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
         __syncwarp();
     } else if (kRecon && warp >= kReconWarp0) {
         // ------------------------------------------------------------ reconstruct
-        const int t = threadIdx.x - kReconWarp0 * 32;
+        // warp w may only touch TMEM lanes 32(w%4)..+31: two warps per lane
+        // quarter, one per half of the 64-wide k step
+        const int quarter = warp & 3, h = (warp - kReconWarp0) >> 2;
+        const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0 + 16u * (uint32_t)h;
         SegWalker wk(blockIdx.x, p);
         Segment sg;
         int64_t q = 0;
@@ -305,8 +347,10 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                 const int s = (int)(q % S);
                 const uint32_t ph = (uint32_t)((q / S) & 1);
                 if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, abort_flag)) { ok = false; break; }
-                reconstruct_tile<SRC>(p, smem + (size_t)s * p.stage_bytes, n0, kt, t);
-                fence_proxy_async_smem();
+                rebuild_row<SRC>(p, smem + (size_t)s * p.stage_bytes, n0, kt, quarter, h, lane,
+                                 tlane + 32u * (uint32_t)s);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&recon_bar[s]));
             }
@@ -318,14 +362,15 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
         int j = 0;
         const int r = warp * 32 + lane;
         while (wk.next(sg)) {
-            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag)) break;
+            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000)) break;
             tc_fence_after();
             const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
             const int64_t n = (int64_t)n_tile * kBlockN + r;
             const int64_t m0 = (int64_t)m_tile * p.MG;
             const bool whole = sg.kt0 == 0 && sg.kt1 == p.kt_count;
             const int64_t slot = 2 * (int64_t)blockIdx.x + (sg.first ? 0 : 1);
-            float* part = p.partial + slot * (int64_t)p.MG * kBlockN;
+            // partial sums: [slot][row][MG] so that a thread's row is contiguous
+            float* part = p.partial + (slot * kBlockN + r) * (int64_t)p.MG;
             for (int c0 = 0; c0 < p.MG; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
@@ -343,15 +388,19 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                         }
                     }
                 } else {
+                    float4* dst = reinterpret_cast<float4*>(part + c0);
 #pragma unroll
-                    for (int i = 0; i < 16; i++) part[(int64_t)(c0 + i) * kBlockN + r] = __uint_as_float(v[i]);
+                    for (int i = 0; i < 4; i++)
+                        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(acce_bar));
             if (!whole) {
-                // stream-K fix-up, one output row per thread
+                // stream-K fix-up, one output row per thread: the last CTA to
+                // arrive sums every segment's partials in CTA order
                 const int64_t t0 = sg.tile * p.kt_count, t1 = t0 + p.kt_count - 1;
                 const int64_t b_first = iter_owner(t0, p.total_iters, p.P);
                 const int64_t b_last = iter_owner(t1, p.total_iters, p.P);
@@ -360,17 +409,35 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
                 unsigned long long* cnt = p.counters + sg.tile * kBlockN + r;
                 if (arrive_counter(cnt, p.epoch) == (unsigned)nsegs) {
                     __threadfence();
-                    for (int c = 0; c < p.MG; c++) {
-                        int64_t m = m0 + c;
-                        float acc = 0.f;
+                    for (int c0 = 0; c0 < p.MG; c0 += 16) {
+                        float acc[16];
+#pragma unroll
+                        for (int i = 0; i < 16; i++) acc[i] = 0.f;
                         for (int64_t b = b_first; b <= b_last; b++) {
-                            int64_t bs = iter_begin(b, p.total_iters, p.P);
-                            int64_t sl = 2 * b + ((bs / p.kt_count) == sg.tile ? 0 : 1);
-                            acc += __ldcg(p.partial + (sl * p.MG + c) * kBlockN + r);
+                            const int64_t bs = iter_begin(b, p.total_iters, p.P);
+                            const int64_t sl = 2 * b + ((bs / p.kt_count) == sg.tile ? 0 : 1);
+                            const float4* src =
+                                reinterpret_cast<const float4*>(p.partial + (sl * kBlockN + r) * (int64_t)p.MG + c0);
+                            float4 q[4];
+#pragma unroll
+                            for (int i = 0; i < 4; i++) q[i] = __ldcg(src + i);
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                acc[4 * i] += q[i].x;
+                                acc[4 * i + 1] += q[i].y;
+                                acc[4 * i + 2] += q[i].z;
+                                acc[4 * i + 3] += q[i].w;
+                            }
                         }
-                        if (m < p.M && n < p.N) {
-                            if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc;
-                            else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc);
+                        if (n < p.N) {
+#pragma unroll
+                            for (int i = 0; i < 16; i++) {
+                                int64_t m = m0 + c0 + i;
+                                if (m < p.M) {
+                                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc[i];
+                                    else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc[i]);
+                                }
+                            }
                         }
                     }
                     *cnt = p.epoch << 16;   // count back to 0 for a replay of this call
@@ -407,7 +474,7 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swz128) {
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -416,7 +483,7 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const voi
     cuuint32_t es[2] = {1, 1};
     (void)esize;
     CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -499,53 +566,75 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.epoch = next_epoch();
     p.timeout_ns = timeout_ns();
 
-    // stage layout
+    // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
     const uint32_t b_bytes = (uint32_t)p.MG * 128;
-    uint32_t off = kTileA;
-    p.off_b = off;
-    off += b_bytes;
+    auto al1k = [](uint32_t x) { return (x + 1023u) & ~1023u; };
+    uint32_t off = 0;
     p.tx_bytes = b_bytes;
     if (a.src == kSrcDense) {
+        p.off_a = 0;
+        p.off_b = kTileA;
+        off = kTileA + b_bytes;
         p.tx_bytes += kTileA;
     } else {
-        p.off_sm = off;
-        off += kTileSM;
-        p.off_s2 = off;
+        p.off_b = 0;
+        p.off_sm = al1k(b_bytes);
+        p.off_s2 = p.off_sm + kTileSM;
         if (a.src == kSrcExponent) {
-            off += kTileE;
+            off = p.off_s2 + kTileE;
             p.tx_bytes += kTileSM + kTileE;
         } else {
-            off += kTileIdx;
-            p.off_v = off;
-            off += kTileV;
+            p.off_v = al1k(p.off_s2 + kTileIdx);
+            off = p.off_v + kTileV;
             p.tx_bytes += kTileSM + kTileIdx + kTileV;
         }
     }
-    p.stage_bytes = (off + 1023) & ~1023u;
+    p.stage_bytes = al1k(off);
     const size_t ctrl = 1024;
     const size_t budget = 227 * 1024 - 1024 - ctrl;
     int S = (int)(budget / p.stage_bytes);
     if (S > kMaxStages) S = kMaxStages;
+    // TMEM: accumulator columns [0, MG); rebuilt-A stages of 32 columns after it
+    uint32_t acc_cols = 32;
+    while (acc_cols < (uint32_t)p.MG) acc_cols <<= 1;
+    if (a.src != kSrcDense) {
+        const int s_tmem = (int)((512u - acc_cols) / 32u);
+        if (S > s_tmem) S = s_tmem;
+    }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.stages = S;
+    p.a_col0 = acc_cols;
+    uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + 32u * (uint32_t)S;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < need_cols) p.tmem_cols <<= 1;
+    if (p.tmem_cols > 512) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
+    p.pal_small = 1;
+    if (a.palette)
+        for (int i = 0; i < 16; i++)
+            if (a.palette[i] >= 128) p.pal_small = 0;
     size_t smem = (size_t)S * p.stage_bytes + ctrl + 1024;
 
     CUtensorMap tx{}, ta{}, ts2{}, tv{};
-    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBlockK, p.MG, true);
+    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBlockK, p.MG,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
     if (a.src == kSrcDense) {
-        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, a.K, a.N, a.K * 2, kBlockK, kBlockN, true);
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, a.K, a.N, a.K * 2, kBlockK, kBlockN,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
         ts2 = ta;
         tv = ta;
     } else {
-        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, kBlockK, kBlockN, false);
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, kBlockK, kBlockN,
+                               CU_TENSOR_MAP_SWIZZLE_64B);
         if (a.src == kSrcExponent) {
-            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, kBlockK, kBlockN, false);
+            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, kBlockK, kBlockN,
+                                   CU_TENSOR_MAP_SWIZZLE_64B);
             tv = ts2;
         } else {
             int64_t NW = 4 * ((a.N + 127) / 128);
             ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.idx, a.K / 2, a.N, a.K / 2, kBlockK / 2,
-                                   kBlockN, false);
-            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kBlockK, NW * 4, 4, 1, false);
+                                   kBlockN, CU_TENSOR_MAP_SWIZZLE_32B);
+            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kBlockK, NW * 4, 4, 1,
+                                   CU_TENSOR_MAP_SWIZZLE_NONE);
         }
     }
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
