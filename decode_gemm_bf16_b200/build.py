@@ -1,6 +1,7 @@
 """Builds libunweight.so (CUDA for sm_100a) in-tree with nvcc."""
 from __future__ import annotations
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -18,12 +19,23 @@ def _nvcc():
     return cand if os.path.exists(cand) else "nvcc"
 
 
+STAMP = LIB + ".srchash"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in SOURCES + HEADERS + [os.path.abspath(__file__)]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def stale() -> bool:
-    if not os.path.exists(LIB):
+    """True when the library is missing or was built from other sources."""
+    if not os.path.exists(LIB) or not os.path.exists(STAMP):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.abspath(__file__)]
-    return any(os.path.getmtime(d) > t for d in deps)
+    with open(STAMP) as fh:
+        return fh.read().strip() != source_hash()
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
@@ -37,6 +49,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as fh:
+        fh.write(source_hash())
     return LIB
 
 

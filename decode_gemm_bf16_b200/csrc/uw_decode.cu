@@ -37,6 +37,7 @@ struct DecodeParams {
     const uint32_t* vpre;
     const uint8_t* vexp;
     uint32_t pal[4];
+    int pal_small;   // all palette exponents < 128
     int64_t n;       // weights
     int64_t nseg;
     void* out;
@@ -48,41 +49,57 @@ __device__ __forceinline__ uint32_t ld_word(const uint32_t* s, int64_t i, int64_
 
 // Decodes segment `seg` (nsym symbols, a multiple of 64) into `row`: word k of
 // the segment (8 nibbles) is stored at row[(k + rot) & 31].
-__device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint32_t* lut,
-                                               int64_t seg, int nsym, uint32_t* row, int rot) {
-    uint64_t bitpos = __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
-    int64_t wi = (int64_t)(bitpos >> 5);
-    if (wi + 1 >= p.nwords) {
+//
+// Bit reservoir in two 32-bit registers: `hi` holds the next 32 stream bits
+// (always all valid when the table is read), `lo` the following ones, of
+// which the top `nlo` are valid.  One table read decodes up to four symbols
+// from the 12-bit window hi >> 20.  Consuming nb bits is a funnel shift; when
+// lo runs dry, the prefetched word `nxt` tops the reservoir up.
+__device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint32_t* lut, int64_t seg, int nsym,
+                                               uint32_t* row, int rot) {
+    const uint64_t bitpos = __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
+    const int64_t wi = (int64_t)(bitpos >> 5);
+    if (wi + 2 >= p.nwords) {
         raise_status(UW_ERR_DEVICE);
         return;
     }
-    uint32_t sh = (uint32_t)(bitpos & 31u);
-    uint64_t buf = (((uint64_t)__ldg(&p.stream[wi]) << 32) | __ldg(&p.stream[wi + 1])) << sh;
-    int avail = 64 - (int)sh;
-    int64_t nxt = wi + 2;
-    uint64_t acc = 0;
-    int accn = 0, k = 0, produced = 0;
+    const uint32_t sh = (uint32_t)(bitpos & 31u);
+    const uint32_t w0 = __ldg(&p.stream[wi]), w1 = __ldg(&p.stream[wi + 1]), w2 = __ldg(&p.stream[wi + 2]);
+    uint32_t hi = __funnelshift_l(w1, w0, sh);   // stream bits [bitpos, bitpos + 32)
+    uint32_t lo = w1 << sh;                        // the rest of w1: 32 - sh valid bits
+    int nlo = 32 - (int)sh;
+    int64_t ptr = wi + 3;
+    uint32_t nxt = w2;                             // the bits right after lo's valid ones
+    uint32_t acc = 0;
+    uint32_t accn = 0;
+    int k = 0, kr = rot;
     const int words = nsym >> 3;
-    while (produced < nsym) {
-        if (avail < 32) {
-            buf |= (uint64_t)ld_word(p.stream, nxt++, p.nwords) << (32 - avail);
-            avail += 32;
-        }
-        uint32_t ent = lut[buf >> 52];
-        uint32_t ns = lut_nsym(ent), nb = lut_bits(ent);
-        if (ns == 0) {
+    while (k < words) {
+        const uint32_t ent = lut[hi >> 20];
+        const uint32_t nb = lut_bits(ent);
+        const uint32_t nn = lut_nibble_bits(ent);
+        if (nn == 0) {
             raise_status(UW_ERR_DEVICE);
             return;
         }
-        acc |= (uint64_t)(ent & 0xFFFFu) << accn;
-        accn += 4 * (int)ns;
-        produced += (int)ns;
-        buf <<= nb;
-        avail -= (int)nb;
+        const uint32_t sy = ent & 0xFFFFu;
+        hi = __funnelshift_l(lo, hi, nb);
+        lo <<= nb;
+        nlo -= (int)nb;
+        if (nlo < 0) {
+            hi |= nxt >> (32 + nlo);
+            lo = nxt << (-nlo);
+            nlo += 32;
+            nxt = ld_word(p.stream, ptr++, p.nwords);
+        }
+        const uint32_t spill = __funnelshift_l(sy, 0u, accn);
+        acc |= sy << accn;
+        accn += nn;
         if (accn >= 32) {
-            if (k < words) row[(k + rot) & 31] = (uint32_t)acc;
+            row[kr] = acc;
+            kr = (kr + 1) & 31;
             k++;
-            acc >>= 32;
+            acc = spill;
             accn -= 32;
         }
     }
@@ -99,6 +116,10 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
         for (int i = threadIdx.x; i < kLutSize / 4; i += kThreads) dst[i] = __ldg(&src[i]);
     }
     __syncthreads();
+    // programmatic stream serialization: the table load above reads only the
+    // committed blob; outputs are touched after the previous kernel ends
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t* st = stage + warp * 1024;
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
@@ -151,6 +172,12 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
                 if ((vw >> (g & 31)) & 1u) {
                     int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
                     ex = __ldg(reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + (e & 63)));
+                } else if (p.pal_small) {
+                    const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
+                    ex.x = palette4_small(w0, x0, P0, P1, P2, P3);
+                    ex.y = palette4_small(w0 >> 16, x0 >> 16, P0, P1, P2, P3);
+                    ex.z = palette4_small(w1, x1, P0, P1, P2, P3);
+                    ex.w = palette4_small(w1 >> 16, x1 >> 16, P0, P1, P2, P3);
                 } else {
                     ex.x = palette4(w0, P0, P1, P2, P3);
                     ex.y = palette4(w0 >> 16, P0, P1, P2, P3);
@@ -191,6 +218,9 @@ cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, 
     for (int i = 0; i < 4; i++)
         p.pal[i] = (uint32_t)b->palette[4 * i] | ((uint32_t)b->palette[4 * i + 1] << 8) |
                    ((uint32_t)b->palette[4 * i + 2] << 16) | ((uint32_t)b->palette[4 * i + 3] << 24);
+    p.pal_small = 1;
+    for (int i = 0; i < 16; i++)
+        if (b->palette[i] >= 128) p.pal_small = 0;
     p.n = b->geo.n;
     p.nseg = b->geo.nseg;
     p.out = out;
@@ -199,21 +229,28 @@ cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, 
     int grid = grid_ctas > 0 ? grid_ctas : num_sms() * decode_ctas_per_sm();
     if (grid > need) grid = (int)need;
     if (grid < 1) grid = 1;
-    cudaError_t e = cudaSuccess;
-    switch (mode) {
-        case kDecodeFull:
-            e = cudaFuncSetAttribute(k_decode<kDecodeFull>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
-            if (e == cudaSuccess) k_decode<kDecodeFull><<<grid, kThreads, kDecodeSmem, s>>>(p);
-            break;
-        case kDecodeExponent:
-            e = cudaFuncSetAttribute(k_decode<kDecodeExponent>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
-            if (e == cudaSuccess) k_decode<kDecodeExponent><<<grid, kThreads, kDecodeSmem, s>>>(p);
-            break;
-        default:
-            e = cudaFuncSetAttribute(k_decode<kDecodeTranscode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
-            if (e == cudaSuccess) k_decode<kDecodeTranscode><<<grid, kThreads, kDecodeSmem, s>>>(p);
-            break;
+    void (*kern)(const DecodeParams) = mode == kDecodeFull       ? k_decode<kDecodeFull>
+                                       : mode == kDecodeExponent ? k_decode<kDecodeExponent>
+                                                                 : k_decode<kDecodeTranscode>;
+    static bool attr_set[3][64] = {{false}};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[mode][dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[mode][dev] = true;
     }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kDecodeSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

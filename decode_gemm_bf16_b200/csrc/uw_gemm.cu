@@ -38,6 +38,8 @@
 #include <cstdlib>
 #include <mutex>
 #include <random>
+#include <tuple>
+#include <vector>
 
 #include "uw_device.cuh"
 #include "uw_internal.h"
@@ -51,7 +53,8 @@ constexpr int kEpiWarps = 4;
 constexpr int kProdWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kReconWarp0 = 6;
-constexpr int kReconWarps = 8;
+constexpr int kReconWarps = 16;       // two groups of 8, one per stage parity
+constexpr int kReconGroupWarps = 8;
 constexpr int kMaxStages = 8;
 constexpr int kThreadsDense = 6 * 32;
 constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(smem_u32(&full_bar[s]), 1);
-            mbar_init(smem_u32(&recon_bar[s]), kReconWarps);
+            mbar_init(smem_u32(&recon_bar[s]), kReconGroupWarps);
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
         mbar_init(smem_u32(accf_bar), 1);
@@ -252,6 +255,10 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
     __syncthreads();
     tc_fence_after();
     const uint32_t tacc = *tmem_slot;
+    // launched with programmatic stream serialization: the prologue above may
+    // overlap the previous kernel; global memory is touched only after it ends
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t smem_base = smem_u32(smem);
 
     if (warp == kProdWarp) {
@@ -333,9 +340,12 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
         __syncwarp();
     } else if (kRecon && warp >= kReconWarp0) {
         // ------------------------------------------------------------ reconstruct
-        // warp w may only touch TMEM lanes 32(w%4)..+31: two warps per lane
-        // quarter, one per half of the 64-wide k step
-        const int quarter = warp & 3, h = (warp - kReconWarp0) >> 2;
+        // warp w may only touch TMEM lanes 32(w%4)..+31.  Two groups of 8
+        // warps take alternate stages (two stages rebuilt at once); inside a
+        // group, two warps per lane quarter, one per half of the k step.
+        const int rw = warp - kReconWarp0;
+        const int group = rw / kReconGroupWarps;
+        const int quarter = warp & 3, h = (rw % kReconGroupWarps) >> 2;
         const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0 + 16u * (uint32_t)h;
         SegWalker wk(blockIdx.x, p);
         Segment sg;
@@ -344,6 +354,7 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
         while (ok && wk.next(sg)) {
             const int64_t n0 = (sg.tile / p.m_tiles) * kBlockN;
             for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
+                if ((int)(q & 1) != group) continue;
                 const int s = (int)(q % S);
                 const uint32_t ph = (uint32_t)((q / S) & 1);
                 if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, abort_flag)) { ok = false; break; }
@@ -495,6 +506,20 @@ int pick_mg(int64_t M) {
     return (int)mg;
 }
 
+// cudaFuncSetAttribute once per (kernel, device, size): it is not free.
+cudaError_t set_smem_attr(const void* fn, int bytes) {
+    static std::mutex mu;
+    static std::vector<std::tuple<const void*, int, int>> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& t : done)
+        if (std::get<0>(t) == fn && std::get<1>(t) == dev && std::get<2>(t) >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.emplace_back(fn, dev, bytes);
+    return e;
+}
+
 // 48-bit call tags: a per-process random base plus a running count.
 unsigned long long next_epoch() {
     static std::atomic<unsigned long long> ctr{0};
@@ -639,24 +664,22 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     }
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
 
-    cudaError_t e;
-    switch (a.src) {
-        case kSrcDense:
-            e = cudaFuncSetAttribute(k_gemm<kSrcDense>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            k_gemm<kSrcDense><<<P, kThreadsDense, smem, s>>>(tx, ta, ts2, tv, p);
-            break;
-        case kSrcExponent:
-            e = cudaFuncSetAttribute(k_gemm<kSrcExponent>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            k_gemm<kSrcExponent><<<P, kThreadsRecon, smem, s>>>(tx, ta, ts2, tv, p);
-            break;
-        default:
-            e = cudaFuncSetAttribute(k_gemm<kSrcPalette>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            k_gemm<kSrcPalette><<<P, kThreadsRecon, smem, s>>>(tx, ta, ts2, tv, p);
-            break;
-    }
+    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams) =
+        a.src == kSrcDense ? k_gemm<kSrcDense> : a.src == kSrcExponent ? k_gemm<kSrcExponent> : k_gemm<kSrcPalette>;
+    cudaError_t e = set_smem_attr((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P);
+    cfg.blockDim = dim3(a.src == kSrcDense ? kThreadsDense : kThreadsRecon);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tx, ta, ts2, tv, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

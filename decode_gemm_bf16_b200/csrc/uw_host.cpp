@@ -120,7 +120,7 @@ void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
             used += one_len[w];
             nsym++;
         }
-        lut[p] = syms | (nsym << 16) | (used << 19);
+        lut[p] = syms | ((4 * nsym) << 16) | (used << 27);
     }
 }
 

@@ -24,10 +24,10 @@ constexpr int64_t kMaxElems = (int64_t(1) << 31) - 256;
 
 // Decode-table entry (derived from the code lengths):
 //   bits  0..15  up to four symbols, symbol i in bits 4i..4i+3
-//   bits 16..18  number of symbols decoded from the 12-bit window (0 = invalid)
-//   bits 19..23  bits consumed by those symbols
-__host__ __device__ constexpr uint32_t lut_nsym(uint32_t e) { return (e >> 16) & 7u; }
-__host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return (e >> 19) & 31u; }
+//   bits 16..20  4 x number of symbols decoded from the 12-bit window (0 = invalid)
+//   bits 27..31  bits consumed by those symbols
+__host__ __device__ constexpr uint32_t lut_nibble_bits(uint32_t e) { return (e >> 16) & 31u; }
+__host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return e >> 27; }
 
 struct Geometry {
     int64_t N = 0, K = 0, n = 0, G = 0, GW = 0, KG = 0, NW = 0, nseg = 0, nchunk = 0;

@@ -6,6 +6,14 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    # compile the library (and the oracle) if their sources changed
+    from decode_gemm_bf16_b200 import build as uwbuild
+    from oracle import oracle as O
+    uwbuild.build()
+    O.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long CPU test")
