@@ -51,10 +51,12 @@ __device__ __forceinline__ uint32_t ld_word(const uint32_t* s, int64_t i, int64_
 // the segment (8 nibbles) is stored at row[(k + rot) & 31].
 //
 // Bit reservoir in two 32-bit registers: `hi` holds the next 32 stream bits
-// (always all valid when the table is read), `lo` the following ones, of
-// which the top `nlo` are valid.  One table read decodes up to four symbols
-// from the 12-bit window hi >> 20.  Consuming nb bits is a funnel shift; when
-// lo runs dry, the prefetched word `nxt` tops the reservoir up.
+// (all valid whenever the table is read), `lo` the following ones, of which
+// the top `nlo` are valid.  One table read decodes up to four symbols from the
+// 12-bit window hi >> 20; consuming them is a funnel shift.  When lo runs dry
+// the prefetched word `nxt` tops the reservoir up.  Word reads are clamped to
+// the stream, so a corrupt stream cannot read outside it; an undecodable
+// window still advances (12 bits) and is reported once per segment.
 __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint32_t* lut, int64_t seg, int nsym,
                                                uint32_t* row, int rot) {
     const uint64_t bitpos = __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
@@ -63,46 +65,47 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
         raise_status(UW_ERR_DEVICE);
         return;
     }
+    const uint32_t* __restrict__ sp = p.stream + wi;
+    const int64_t room = p.nwords - 1 - wi;
+    const uint32_t last = room > 0x7FFFFFFF ? 0x7FFFFFFFu : (uint32_t)room;   // last readable index
     const uint32_t sh = (uint32_t)(bitpos & 31u);
-    const uint32_t w0 = __ldg(&p.stream[wi]), w1 = __ldg(&p.stream[wi + 1]), w2 = __ldg(&p.stream[wi + 2]);
-    uint32_t hi = __funnelshift_l(w1, w0, sh);   // stream bits [bitpos, bitpos + 32)
-    uint32_t lo = w1 << sh;                        // the rest of w1: 32 - sh valid bits
+    const uint32_t w0 = __ldg(sp), w1 = __ldg(sp + 1);
+    uint32_t nxt = __ldg(sp + 2);                   // the bits right after lo's valid ones
+    uint32_t hi = __funnelshift_l(w1, w0, sh);      // stream bits [bitpos, bitpos + 32)
+    uint32_t lo = w1 << sh;                         // rest of w1: 32 - sh valid bits
     int nlo = 32 - (int)sh;
-    int64_t ptr = wi + 3;
-    uint32_t nxt = w2;                             // the bits right after lo's valid ones
-    uint32_t acc = 0;
-    uint32_t accn = 0;
+    uint32_t idx = 3;
+    uint32_t acc = 0, accn = 0, flags = 0;
     int k = 0, kr = rot;
     const int words = nsym >> 3;
     while (k < words) {
         const uint32_t ent = lut[hi >> 20];
+        flags |= ent;
         const uint32_t nb = lut_bits(ent);
-        const uint32_t nn = lut_nibble_bits(ent);
-        if (nn == 0) {
-            raise_status(UW_ERR_DEVICE);
-            return;
-        }
-        const uint32_t sy = ent & 0xFFFFu;
         hi = __funnelshift_l(lo, hi, nb);
         lo <<= nb;
         nlo -= (int)nb;
+        const uint32_t sy = ent >> 16;
+        const uint32_t accn2 = accn + lut_nibble_bits(ent);
+        acc |= sy << accn;
         if (nlo < 0) {
             hi |= nxt >> (32 + nlo);
             lo = nxt << (-nlo);
             nlo += 32;
-            nxt = ld_word(p.stream, ptr++, p.nwords);
+            nxt = __ldg(sp + min(idx, last));
+            idx++;
         }
-        const uint32_t spill = __funnelshift_l(sy, 0u, accn);
-        acc |= sy << accn;
-        accn += nn;
-        if (accn >= 32) {
+        if (accn2 >= 32u) {
             row[kr] = acc;
             kr = (kr + 1) & 31;
             k++;
-            acc = spill;
-            accn -= 32;
+            acc = sy >> (32u - accn);     // accn >= 16 here, so the shift is in [1, 16]
+            accn = accn2 - 32u;
+        } else {
+            accn = accn2;
         }
     }
+    if (flags & kLutInvalid) raise_status(UW_ERR_DEVICE);
 }
 
 template <int MODE>
@@ -137,16 +140,18 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
             if (nsym > 0) decode_segment(p, lut, seg, nsym, st + lane * 32, lane);
         }
         __syncwarp();
-        // ---- phase 2: ordered, coalesced output
+        // ---- phase 2: ordered, coalesced output (offsets relative to the task)
+        const int64_t left = p.n - base;
+        const int lim = left < kTaskElems ? (int)left : kTaskElems;
         if (MODE == kDecodeTranscode) {
             // lane -> segment 4*it + lane/8, words 4*(lane%8) .. +3 (32 nibbles)
-            uint4* out = reinterpret_cast<uint4*>(p.out);
+            uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) + (base >> 1));
 #pragma unroll 2
             for (int it = 0; it < 8; it++) {
-                int j = 4 * it + (lane >> 3);
-                int k0 = 4 * (lane & 7);
-                int64_t e = base + (int64_t)j * kSeg + k0 * 8;
-                if (e < p.n) {
+                const int j = 4 * it + (lane >> 3);
+                const int k0 = 4 * (lane & 7);
+                const int e = j * kSeg + k0 * 8;
+                if (e < lim) {
                     const uint32_t* r = st + j * 32;
                     uint4 v;
                     v.x = r[(k0 + 0 + j) & 31];
@@ -158,19 +163,22 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
             }
         } else {
             // lane -> segment 2*it + lane/16, words 2*(lane%16), +1 (16 weights)
+            const uint32_t* vb = p.vbits + (base >> 11);          // 128 groups per task = 4 words
+            const uint8_t* smb = p.sm + base;
 #pragma unroll 2
             for (int it = 0; it < 16; it++) {
-                int j = 2 * it + (lane >> 4);
-                int k0 = 2 * (lane & 15);
-                int64_t e = base + (int64_t)j * kSeg + k0 * 8;
-                if (e >= p.n) continue;
+                const int j = 2 * it + (lane >> 4);
+                const int k0 = 2 * (lane & 15);
+                const int e = j * kSeg + k0 * 8;
+                if (e >= lim) continue;
                 const uint32_t* r = st + j * 32;
-                uint32_t w0 = r[(k0 + j) & 31], w1 = r[(k0 + 1 + j) & 31];
+                const uint32_t w0 = r[(k0 + j) & 31], w1 = r[(k0 + 1 + j) & 31];
                 uint4 ex;
-                int64_t g = e >> 6;
-                uint32_t vw = __ldg(&p.vbits[g >> 5]);
+                const int g = e >> 6;                               // group within the task
+                const uint32_t vw = __ldg(&vb[g >> 5]);
                 if ((vw >> (g & 31)) & 1u) {
-                    int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
+                    const int64_t gg = (base >> 6) + g;
+                    const int64_t rank = __ldg(&p.vpre[gg >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
                     ex = __ldg(reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + (e & 63)));
                 } else if (p.pal_small) {
                     const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
@@ -185,12 +193,12 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
                     ex.w = palette4(w1 >> 16, P0, P1, P2, P3);
                 }
                 if (MODE == kDecodeExponent) {
-                    reinterpret_cast<uint4*>(p.out)[e >> 4] = ex;
+                    reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) + base)[e >> 4] = ex;
                 } else {
-                    uint4 s = __ldg(reinterpret_cast<const uint4*>(p.sm + e));
-                    uint2 a = merge4(ex.x, s.x), b = merge4(ex.y, s.y);
-                    uint2 c = merge4(ex.z, s.z), d = merge4(ex.w, s.w);
-                    uint4* out = reinterpret_cast<uint4*>(p.out) + (e >> 3);
+                    const uint4 s = __ldg(reinterpret_cast<const uint4*>(smb + e));
+                    const uint2 a = merge4(ex.x, s.x), b = merge4(ex.y, s.y);
+                    const uint2 c = merge4(ex.z, s.z), d = merge4(ex.w, s.w);
+                    uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + base) + (e >> 3);
                     out[0] = make_uint4(a.x, a.y, b.x, b.y);
                     out[1] = make_uint4(c.x, c.y, d.x, d.y);
                 }

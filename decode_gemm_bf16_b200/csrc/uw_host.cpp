@@ -120,7 +120,10 @@ void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
             used += one_len[w];
             nsym++;
         }
-        lut[p] = syms | ((4 * nsym) << 16) | (used << 27);
+        if (nsym == 0)   // no valid code: progress by 12 bits, flag it
+            lut[p] = 12u | (4u << 5) | kLutInvalid;
+        else
+            lut[p] = used | ((4 * nsym) << 5) | (syms << 16);
     }
 }
 

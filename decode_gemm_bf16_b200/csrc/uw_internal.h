@@ -23,11 +23,14 @@ constexpr uint32_t kFormatVersion = 1;
 constexpr int64_t kMaxElems = (int64_t(1) << 31) - 256;
 
 // Decode-table entry (derived from the code lengths):
-//   bits  0..15  up to four symbols, symbol i in bits 4i..4i+3
-//   bits 16..20  4 x number of symbols decoded from the 12-bit window (0 = invalid)
-//   bits 27..31  bits consumed by those symbols
-__host__ __device__ constexpr uint32_t lut_nibble_bits(uint32_t e) { return (e >> 16) & 31u; }
-__host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return e >> 27; }
+//   bits  0..4   bits consumed by the decoded symbols (1..12)
+//   bits  5..9   4 x number of symbols decoded from the 12-bit window (4..16)
+//   bit  10      the window starts with no valid code (only in incomplete
+//                codes): decoded as one symbol 0 of 12 bits, and reported
+//   bits 16..31  up to four symbols, symbol i in bits 16+4i..19+4i
+__host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return e & 31u; }
+__host__ __device__ constexpr uint32_t lut_nibble_bits(uint32_t e) { return (e >> 5) & 31u; }
+constexpr uint32_t kLutInvalid = 1u << 10;
 
 struct Geometry {
     int64_t N = 0, K = 0, n = 0, G = 0, GW = 0, KG = 0, NW = 0, nseg = 0, nchunk = 0;
