@@ -22,7 +22,7 @@ namespace uw {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kBesideWarps = 4;                // decoder CTAs that share SMs with the GEMM
 constexpr int kTaskElems = 32 * kSeg;          // 8192 weights per warp task
 constexpr size_t kDecodeSmem = kLutSize * 4 + kWarps * 32 * 32 * 4;
 
@@ -41,11 +41,10 @@ struct DecodeParams {
     int64_t n;       // weights
     int64_t nseg;
     void* out;
+    unsigned long long* band_ready;   // optional: per-band finished-task counters
+    unsigned long long epoch;
+    int64_t band_tasks;               // tasks per band of 128 rows (= K/64)
 };
-
-__device__ __forceinline__ uint32_t ld_word(const uint32_t* s, int64_t i, int64_t nwords) {
-    return i < nwords ? __ldg(&s[i]) : 0u;
-}
 
 // Decodes segment `seg` (nsym symbols, a multiple of 64) into `row`: word k of
 // the segment (8 nibbles) is stored at row[(k + rot) & 31].
@@ -108,15 +107,15 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
     if (flags & kLutInvalid) raise_status(UW_ERR_DEVICE);
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
+template <int MODE, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 4) k_decode(const DecodeParams p) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     uint32_t* stage = smem + kLutSize;
     {
         const uint4* src = reinterpret_cast<const uint4*>(p.lut);
         uint4* dst = reinterpret_cast<uint4*>(lut);
-        for (int i = threadIdx.x; i < kLutSize / 4; i += kThreads) dst[i] = __ldg(&src[i]);
+        for (int i = threadIdx.x; i < kLutSize / 4; i += WARPS * 32) dst[i] = __ldg(&src[i]);
     }
     __syncthreads();
     // programmatic stream serialization: the table load above reads only the
@@ -128,8 +127,8 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
     const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
 
-    for (int64_t task = (int64_t)blockIdx.x * kWarps + warp; task < ntasks;
-         task += (int64_t)gridDim.x * kWarps) {
+    for (int64_t task = (int64_t)blockIdx.x * WARPS + warp; task < ntasks;
+         task += (int64_t)gridDim.x * WARPS) {
         const int64_t base = task * kTaskElems;
         // ---- phase 1: one segment per lane
         {
@@ -205,6 +204,12 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
             }
         }
         __syncwarp();
+        if (p.band_ready) {
+            // publish: this task's outputs are written
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) arrive_counter(p.band_ready + task / p.band_tasks, p.epoch);
+        }
     }
 }
 
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode(const DecodeParams p) {
 
 int decode_ctas_per_sm() { return 4; }
 
-cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s) {
+static DecodeParams decode_params(const uw_blob* b, void* out) {
     DecodeParams p;
     p.stream = (const uint32_t*)b->sec(UW_SEC_STREAM);
     p.nwords = b->nwords;
@@ -232,26 +237,29 @@ cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, 
     p.n = b->geo.n;
     p.nseg = b->geo.nseg;
     p.out = out;
-    int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
-    int64_t need = (ntasks + kWarps - 1) / kWarps;
-    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * decode_ctas_per_sm();
-    if (grid > need) grid = (int)need;
-    if (grid < 1) grid = 1;
-    void (*kern)(const DecodeParams) = mode == kDecodeFull       ? k_decode<kDecodeFull>
-                                       : mode == kDecodeExponent ? k_decode<kDecodeExponent>
-                                                                 : k_decode<kDecodeTranscode>;
+    p.band_ready = nullptr;
+    p.epoch = 0;
+    p.band_tasks = b->geo.KG;
+    return p;
+}
+
+template <int WARPS>
+static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid, size_t smem, cudaStream_t s) {
+    void (*kern)(const DecodeParams) = mode == kDecodeFull       ? k_decode<kDecodeFull, WARPS>
+                                       : mode == kDecodeExponent ? k_decode<kDecodeExponent, WARPS>
+                                                                 : k_decode<kDecodeTranscode, WARPS>;
     static bool attr_set[3][64] = {{false}};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[mode][dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[mode][dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kDecodeSmem;
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -261,6 +269,28 @@ cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, 
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s) {
+    DecodeParams p = decode_params(b, out);
+    const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
+    const int64_t need = (ntasks + kWarps - 1) / kWarps;
+    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * decode_ctas_per_sm();
+    if (grid > need) grid = (int)need;
+    if (grid < 1) grid = 1;
+    return launch_decode_impl<kWarps>(p, mode, grid, kDecodeSmem, s);
+}
+
+cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas, unsigned long long* band_ready,
+                                 unsigned long long epoch, cudaStream_t s) {
+    DecodeParams p = decode_params(b, out);
+    p.band_ready = band_ready;
+    p.epoch = epoch;
+    const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
+    const int64_t need = (ntasks + kBesideWarps - 1) / kBesideWarps;
+    int grid = ctas > need ? (int)need : ctas;
+    if (grid < 1) grid = 1;
+    return launch_decode_impl<kBesideWarps>(p, mode, grid, kDecodeBesideSmem, s);
 }
 
 int decode_status_take() { return unit_status_take(); }

@@ -71,6 +71,29 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// ---------------------------------------------------------------- tagged counters
+// A 64-bit counter word holds (tag << 16) | count, tag = 48-bit id of one
+// call.  A word carrying another tag (or stale bytes) counts as 0, so
+// counters living in caller workspace never need clearing.
+__device__ __forceinline__ unsigned arrive_counter(unsigned long long* cnt, unsigned long long tag) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+    for (;;) {
+        const unsigned long long base = (cur >> 16) == tag ? cur : (tag << 16);
+        const unsigned long long nxt = base + 1;
+        const unsigned long long prev = atomicCAS(cnt, cur, nxt);
+        if (prev == cur) return (unsigned)(nxt & 0xFFFFu);
+        cur = prev;
+    }
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+// Bounded wait until the counter shows `want` arrivals of call `tag`.
+__device__ __forceinline__ bool wait_counter(const unsigned long long* cnt, unsigned long long tag, unsigned want,
+                                             uint64_t timeout_ns, volatile int* abort);
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -119,11 +142,33 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
+__device__ __forceinline__ bool wait_counter(const unsigned long long* cnt, unsigned long long tag, unsigned want,
+                                             uint64_t timeout_ns, volatile int* abort) {
+    uint64_t deadline = 0;
+    for (uint32_t i = 0;; i++) {
+        const unsigned long long v = ld_acquire_u64(cnt);
+        if ((v >> 16) == tag && (unsigned)(v & 0xFFFFu) >= want) return true;
+        if (abort && *abort) return false;
+        const uint64_t now = globaltimer();
+        if (deadline == 0) {
+            deadline = now + timeout_ns;
+        } else if (now > deadline) {
+            if (abort) *abort = 1;
+            return false;
+        }
+        __nanosleep(200);
+    }
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Generic-proxy writes observed (acquire) -> visible to TMA (async proxy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- TMA

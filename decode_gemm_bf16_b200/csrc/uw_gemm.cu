@@ -81,23 +81,12 @@ struct GemmParams {
     float* partial;                // [2P][128][MG]
     unsigned long long* counters;  // [tiles][128]: (epoch << 16) | arrivals
     unsigned long long epoch;      // 48-bit tag of this call
+    // decoder running beside the GEMM: band b of 128 rows is ready when
+    // band_ready[b] shows band_tasks(b) finished decoder tasks of this call
+    const unsigned long long* band_ready;
+    int64_t band_tasks, ntasks;
     uint64_t timeout_ns;
 };
-
-// Counts one arrival at a stream-K fix-up counter and returns the number of
-// arrivals of this call so far.  The word holds (epoch << 16) | count; a word
-// carrying another call's tag (or any stale bytes left in the workspace) is
-// taken as a count of 0, so the workspace never needs clearing.
-__device__ __forceinline__ unsigned arrive_counter(unsigned long long* cnt, unsigned long long epoch) {
-    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
-    for (;;) {
-        unsigned long long base = (cur >> 16) == epoch ? cur : (epoch << 16);
-        unsigned long long nxt = base + 1;
-        unsigned long long prev = atomicCAS(cnt, cur, nxt);
-        if (prev == cur) return (unsigned)(nxt & 0xFFFFu);
-        cur = prev;
-    }
-}
 
 __host__ __device__ __forceinline__ int64_t iter_begin(int64_t b, int64_t total, int64_t P) {
     return b * total / P;
@@ -268,8 +257,18 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
             Segment sg;
             int64_t q = 0;
             bool ok = true;
+            int ready_band = -1;
             while (ok && wk.next(sg)) {
                 const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
+                if (p.band_ready && n_tile != ready_band) {
+                    // the rows of this tile come from the decoder running beside us
+                    const int64_t t0 = (int64_t)n_tile * p.band_tasks;
+                    const int64_t left = p.ntasks - t0;
+                    const unsigned want = (unsigned)(left < p.band_tasks ? left : p.band_tasks);
+                    if (!wait_counter(p.band_ready + n_tile, p.epoch, want, p.timeout_ns, abort_flag)) { ok = false; break; }
+                    fence_proxy_async_global();
+                    ready_band = n_tile;
+                }
                 for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
                     const int s = (int)(q % S);
                     const uint32_t ph = (uint32_t)((q / S) & 1);
@@ -545,6 +544,8 @@ uint64_t timeout_ns() {
 
 int gemm_default_grid() { return num_sms(); }
 
+unsigned long long gemm_next_epoch() { return next_epoch(); }
+
 int gemm_status_take() { return unit_status_take(); }
 
 size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
@@ -588,7 +589,10 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     size_t part = (size_t)2 * P * p.MG * kBlockN * 4;
     p.partial = (float*)a.ws;
     p.counters = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
-    p.epoch = next_epoch();
+    p.epoch = a.epoch ? a.epoch : next_epoch();
+    p.band_ready = a.band_ready;
+    p.band_tasks = a.band_tasks;
+    p.ntasks = a.ntasks;
     p.timeout_ns = timeout_ns();
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
@@ -616,7 +620,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     }
     p.stage_bytes = al1k(off);
     const size_t ctrl = 1024;
-    const size_t budget = 227 * 1024 - 1024 - ctrl;
+    size_t budget = 227 * 1024 - 1024 - ctrl;
+    if (a.smem_cap > 0 && (size_t)a.smem_cap < budget + 2048) budget = (size_t)a.smem_cap - 2048;
     int S = (int)(budget / p.stage_bytes);
     if (S > kMaxStages) S = kMaxStages;
     // TMEM: accumulator columns [0, MG); rebuilt-A stages of 32 columns after it

@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -640,14 +641,49 @@ static size_t decode_buffer_bytes(const uw_blob* b, int pipeline) {
     }
 }
 
+static bool runs_beside(const uw_gemm_opts* o) { return o->sm_dec > 0 && o->pipeline != UW_PIPE_DIRECT_PALETTE; }
+
+static size_t band_counter_bytes(const uw_blob* b) { return al256((uint64_t)((b->geo.N + 127) / 128) * 8); }
+
 extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gemm_opts* o, size_t* bytes) {
     uw_status st = check_committed(b);
     if (st) return st;
     if (!o || !bytes || M < 0) return UW_ERR_INVALID_ARG;
     if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
     if (M == 0) { *bytes = 0; return UW_OK; }
-    *bytes = decode_buffer_bytes(b, o->pipeline) + gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid);
+    *bytes = decode_buffer_bytes(b, o->pipeline) + al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid)) +
+             (runs_beside(o) ? band_counter_bytes(b) : 0);
     return UW_OK;
+}
+
+// Side stream and fork/join events per device for the decoder-beside-GEMM
+// launch (§解壓與運算資源共享).  Created once; calls on one device that run
+// beside each other must not overlap (they share these).
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+static SideStream* side_stream(uw_status* st) {
+    static std::mutex mu;
+    static SideStream per_dev[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        *st = UW_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    SideStream& ss = per_dev[dev];
+    if (!ss.s) {
+        if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            *st = UW_ERR_CUDA;
+            return nullptr;
+        }
+    }
+    return &ss;
 }
 
 extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, void* Y, const uw_gemm_opts* o,
@@ -662,7 +698,6 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     const bool needs_huff = o->pipeline != UW_PIPE_DIRECT_PALETTE;
     if (needs_huff && !(b->forms & UW_FORM_HUFFMAN)) return UW_ERR_UNSUPPORTED;
     if (!needs_huff && !(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
-    if (o->sm_dec > 0) return UW_ERR_UNSUPPORTED;
     size_t need = 0;
     uw_gemm_workspace(b, M, o, &need);
     if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
@@ -686,28 +721,43 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     a.vexp = b->sec(UW_SEC_VEXP);
     a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
     a.palette = b->palette;
+    const int mode = o->pipeline == UW_PIPE_FULL ? kDecodeFull : o->pipeline == UW_PIPE_EXPONENT ? kDecodeExponent
+                                                                                                : kDecodeTranscode;
     switch (o->pipeline) {
-        case UW_PIPE_FULL:
-            if (cuda_ok(launch_decode(b, kDecodeFull, ws, 0, s))) return UW_ERR_CUDA;
-            a.src = kSrcDense;
-            a.W = (const uint16_t*)ws;
-            break;
-        case UW_PIPE_EXPONENT:
-            if (cuda_ok(launch_decode(b, kDecodeExponent, ws, 0, s))) return UW_ERR_CUDA;
-            a.src = kSrcExponent;
-            a.ex = ws;
-            break;
-        case UW_PIPE_TRANSCODE:
-            if (cuda_ok(launch_decode(b, kDecodeTranscode, ws, 0, s))) return UW_ERR_CUDA;
-            a.src = kSrcPalette;
-            a.idx = ws;
-            break;
-        default:
-            a.src = kSrcPalette;
-            a.idx = b->sec(UW_SEC_IDX);
-            break;
+        case UW_PIPE_FULL: a.src = kSrcDense; a.W = (const uint16_t*)ws; break;
+        case UW_PIPE_EXPONENT: a.src = kSrcExponent; a.ex = ws; break;
+        case UW_PIPE_TRANSCODE: a.src = kSrcPalette; a.idx = ws; break;
+        default: a.src = kSrcPalette; a.idx = b->sec(UW_SEC_IDX); break;
     }
-    cudaError_t e = launch_gemm(a, s, &st);
+    if (o->pipeline == UW_PIPE_DIRECT_PALETTE) {
+        cudaError_t e = launch_gemm(a, s, &st);
+        if (st) return st;
+        return cuda_ok(e);
+    }
+    if (!runs_beside(o)) {
+        // decode, then GEMM
+        if (cuda_ok(launch_decode(b, mode, ws, 0, s))) return UW_ERR_CUDA;
+        cudaError_t e = launch_gemm(a, s, &st);
+        if (st) return st;
+        return cuda_ok(e);
+    }
+    // decoder beside the GEMM: the decoder's CTAs publish finished 128-row
+    // bands, the GEMM's producer waits for a band before loading its tiles.
+    // The GEMM keeps room for one decoder CTA on every SM.
+    SideStream* ss = side_stream(&st);
+    if (!ss) return st;
+    a.ws_bytes = al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid));
+    unsigned long long* band = (unsigned long long*)(ws + dbuf + a.ws_bytes);
+    a.epoch = gemm_next_epoch();
+    a.band_ready = band;
+    a.band_tasks = b->geo.KG;
+    a.ntasks = (b->geo.n + 8191) / 8192;
+    a.smem_cap = 228 * 1024 - kDecodeBesideSmem - 2048;
+    if (cuda_ok(cudaEventRecord(ss->fork, s)) || cuda_ok(cudaStreamWaitEvent(ss->s, ss->fork, 0))) return UW_ERR_CUDA;
+    if (cuda_ok(launch_decode_beside(b, mode, ws, o->sm_dec, band, a.epoch, s))) return UW_ERR_CUDA;
+    cudaError_t e = launch_gemm(a, ss->s, &st);
+    if (!st && e == cudaSuccess) e = cudaEventRecord(ss->join, ss->s);
+    if (!st && e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
     if (st) return st;
     return cuda_ok(e);
 }
@@ -763,6 +813,10 @@ extern "C" uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const 
     struct Cand { int pipe, sm_dec; };
     std::vector<Cand> cands;
     for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_DIRECT_PALETTE; pp++) cands.push_back({pp, 0});
+    // decoder beside the GEMM, with a few decoder CTA counts
+    const int sms = num_sms();
+    for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_TRANSCODE; pp++)
+        for (int f : {1, 2, 4}) cands.push_back({pp, f * sms / 2});
     uw_status result = UW_OK;
     for (int mi = 0; mi < nM && result == UW_OK; mi++) {
         const int64_t M = Ms[mi];

@@ -106,6 +106,11 @@ cudaError_t launch_encode(const uint16_t* W, const Geometry& g, const uint8_t in
 // ---- decoders (uw_decode.cu)
 enum DecodeMode { kDecodeFull = 0, kDecodeExponent = 1, kDecodeTranscode = 2 };
 cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s);
+// Decoder that runs beside the GEMM: `ctas` CTAs of 4 warps, each finished
+// 8192-weight task counted in band_ready[task / (K/64)] under call tag `epoch`.
+cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas, unsigned long long* band_ready,
+                                 unsigned long long epoch, cudaStream_t s);
+constexpr int kDecodeBesideSmem = (1 << 12) * 4 + 4 * 32 * 32 * 4;   // LUT + 4 warps of staging
 int decode_ctas_per_sm();
 
 // ---- GEMM (uw_gemm.cu)
@@ -128,9 +133,14 @@ struct GemmArgs {
     int grid = 0;
     void* ws = nullptr;               // partial sums + tile counters
     size_t ws_bytes = 0;
+    int smem_cap = 0;                 // >0: dynamic shared memory limit (room for a decoder CTA)
+    unsigned long long epoch = 0;     // 0: a fresh call tag
+    const unsigned long long* band_ready = nullptr;   // decoder-beside-GEMM readiness
+    int64_t band_tasks = 0, ntasks = 0;
 };
 size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid);
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st);
 int gemm_default_grid();
+unsigned long long gemm_next_epoch();
 
 }  // namespace uw

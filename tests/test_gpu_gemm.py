@@ -170,3 +170,58 @@ def test_workspace_contents_do_not_matter(fill):
             Y = uw.uw_gemm(Xd, blob, pipe, out_f32=True, ws=ws)
         check_gemm(_f32(Y), R, bf16_out=False)
     assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("pipe", ["full", "exponent", "transcode"])
+@pytest.mark.parametrize("sm_dec", [1, 37, 148, 300])
+def test_decoder_beside_gemm(pipe, sm_dec):
+    """Decoder CTAs running beside the GEMM (SM split): the GEMM waits for
+    each 128-row band; the result is the same as decode-then-GEMM."""
+    W, blob = _case("200x1408")
+    X = S.activations(24, 1408, seed=11)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    ref = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True))
+    for _ in range(2):
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True, sm_dec=sm_dec))
+        check_gemm(Y, R, bf16_out=False)
+        assert np.array_equal(Y, ref)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_decoder_beside_gemm_full_size():
+    W = S.gate_projection()
+    blob = uw.uw_compress(dev16(W))
+    X = S.activations(16, 4096, seed=12)
+    Xd = dev16(X)
+    for pipe in ["exponent", "transcode"]:
+        ref = _f32(uw.uw_gemm(Xd, blob, pipe))
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe, sm_dec=74))
+        assert np.array_equal(Y, ref)
+        _sampled(X, W, Y, 64, seed=5, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_autotune_plan(tmp_path):
+    """The autotuner returns one feasible, measured choice per projection
+    and batch size and writes the plan as JSON."""
+    import json
+    shapes = [(384, 512), (384, 512), (512, 384 + 128)]
+    Ws = [S.gaussian_weight(n, k, seed=60 + i) for i, (n, k) in enumerate(shapes)]
+    blobs = [uw.uw_compress(dev16(w)) for w in Ws]
+    Ms = [1, 64]
+    Xs = [dev16(S.activations(max(Ms), k, seed=70 + i)) for i, (n, k) in enumerate(shapes)]
+    Ys = [torch.empty(max(Ms), n, dtype=torch.bfloat16, device="cuda") for (n, k) in shapes]
+    need = max(uw.uw_gemm_workspace(b, max(Ms), p, sm_dec=sd) for b in blobs
+               for p in PIPES for sd in (0, 300))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    path = str(tmp_path / "plan.json")
+    plan = uw.uw_autotune(blobs, Ms, Xs, Ys, ws, reps=3, plan_json_path=path)
+    assert len(plan) == len(Ms) * len(blobs)
+    for i, e in enumerate(plan):
+        assert e["M"] == Ms[i // 3] and e["projection"] == i % 3
+        assert e["pipeline"] in PIPES and e["us"] > 0
+    saved = json.load(open(path))["plan"]
+    assert [(d["projection"], d["M"], d["pipeline"]) for d in saved] == \
+        [(e["projection"], e["M"], e["pipeline"]) for e in plan]
+    assert uw.uw_last_device_status() == 0
