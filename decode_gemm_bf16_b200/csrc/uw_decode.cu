@@ -253,6 +253,10 @@ static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid,
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[mode][dev]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        // SMs running decoder CTAs keep the largest shared-memory carveout, so
+        // a GEMM CTA can still be placed beside them
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[mode][dev] = true;
     }

@@ -195,10 +195,8 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
 }
 
 template <int SRC>
-__global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRecon, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
-           const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
-           const GemmParams p) {
+__device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_a, const CUtensorMap& tm_s2,
+                                          const CUtensorMap& tm_v, const GemmParams& p) {
     constexpr bool kRecon = SRC != kSrcDense;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -466,6 +464,24 @@ __global__ void __launch_bounds__(SRC == kSrcDense ? kThreadsDense : kThreadsRec
     }
 }
 
+// Dense source: 6 warps, registers unconstrained.
+__global__ void __launch_bounds__(kThreadsDense, 1)
+    k_gemm_dense(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                 const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+                 const GemmParams p) {
+    gemm_body<kSrcDense>(tm_x, tm_a, tm_s2, tm_v, p);
+}
+
+// Rebuilding sources: 22 warps held to 72 registers, which leaves one warp's
+// worth of registers per SM sub-partition for a decoder CTA running beside.
+template <int SRC>
+__global__ void __maxnreg__(72)
+    k_gemm_recon(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                 const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+                 const GemmParams p) {
+    gemm_body<SRC>(tm_x, tm_a, tm_s2, tm_v, p);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -515,6 +531,7 @@ cudaError_t set_smem_attr(const void* fn, int bytes) {
     for (auto& t : done)
         if (std::get<0>(t) == fn && std::get<1>(t) == dev && std::get<2>(t) >= bytes) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess) done.emplace_back(fn, dev, bytes);
     return e;
 }
@@ -670,7 +687,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
 
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams) =
-        a.src == kSrcDense ? k_gemm<kSrcDense> : a.src == kSrcExponent ? k_gemm<kSrcExponent> : k_gemm<kSrcPalette>;
+        a.src == kSrcDense ? k_gemm_dense : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent> : k_gemm_recon<kSrcPalette>;
     cudaError_t e = set_smem_attr((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
