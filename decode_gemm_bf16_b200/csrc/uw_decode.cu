@@ -51,7 +51,7 @@ struct DecodeParams {
 //
 // Bit reservoir in two 32-bit registers: `hi` holds the next 32 stream bits
 // (all valid whenever the table is read), `lo` the following ones, of which
-// the top `nlo` are valid.  One table read decodes up to four symbols from the
+// the top `nlo` are valid.  One table read decodes up to five symbols from the
 // 12-bit window hi >> 20; consuming them is a funnel shift.  When lo runs dry
 // the prefetched word `nxt` tops the reservoir up.  Word reads are clamped to
 // the stream, so a corrupt stream cannot read outside it; an undecodable
@@ -84,7 +84,7 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
         hi = __funnelshift_l(lo, hi, nb);
         lo <<= nb;
         nlo -= (int)nb;
-        const uint32_t sy = ent >> 16;
+        const uint32_t sy = ent >> kLutSymShift;
         const uint32_t accn2 = accn + lut_nibble_bits(ent);
         acc |= sy << accn;
         if (nlo < 0) {
@@ -98,7 +98,7 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
             row[kr] = acc;
             kr = (kr + 1) & 31;
             k++;
-            acc = sy >> (32u - accn);     // accn >= 16 here, so the shift is in [1, 16]
+            acc = sy >> (32u - accn);     // accn >= 12 here, so the shift is in [1, 20]
             accn = accn2 - 32u;
         } else {
             accn = accn2;
@@ -130,6 +130,14 @@ __global__ void __launch_bounds__(WARPS * 32, 4) k_decode(const DecodeParams p) 
     for (int64_t task = (int64_t)blockIdx.x * WARPS + warp; task < ntasks;
          task += (int64_t)gridDim.x * WARPS) {
         const int64_t base = task * kTaskElems;
+        if (MODE == kDecodeFull) {
+            // warm L2 with this task's sign+mantissa bytes, read in phase 2
+            const int64_t off = base + (int64_t)lane * 256;
+            if (off < p.n) {
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.sm + off));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.sm + off + 128));
+            }
+        }
         // ---- phase 1: one segment per lane
         {
             int64_t seg = task * 32 + lane;

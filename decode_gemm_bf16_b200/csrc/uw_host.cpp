@@ -104,7 +104,7 @@ void build_code(const uint64_t freq[16], uint8_t len[16], uint32_t code[16]) {
 }
 
 // 4096-entry multi-symbol table: entry p decodes as many whole codes (up to
-// four) as fit in the 12-bit window p, read MSB first.
+// five) as fit in the 12-bit window p, read MSB first.
 void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
     std::vector<int> one_sym(kLutSize, -1), one_len(kLutSize, 0);
     for (int s = 0; s < 16; s++) {
@@ -114,7 +114,7 @@ void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
     }
     for (uint32_t p = 0; p < (uint32_t)kLutSize; p++) {
         uint32_t syms = 0, nsym = 0, used = 0;
-        while (nsym < 4) {
+        while (nsym < (uint32_t)kLutMaxSymbols) {
             uint32_t w = (p << used) & (kLutSize - 1);
             if (one_sym[w] < 0 || used + one_len[w] > (uint32_t)kLmax) break;
             syms |= (uint32_t)one_sym[w] << (4 * nsym);
@@ -124,7 +124,7 @@ void build_lut(const uint8_t len[16], const uint32_t code[16], uint32_t* lut) {
         if (nsym == 0)   // no valid code: progress by 12 bits, flag it
             lut[p] = 12u | (4u << 5) | kLutInvalid;
         else
-            lut[p] = used | ((4 * nsym) << 5) | (syms << 16);
+            lut[p] = used | ((4 * nsym) << 5) | (syms << kLutSymShift);
     }
 }
 

@@ -24,10 +24,12 @@ constexpr int64_t kMaxElems = (int64_t(1) << 31) - 256;
 
 // Decode-table entry (derived from the code lengths):
 //   bits  0..4   bits consumed by the decoded symbols (1..12)
-//   bits  5..9   4 x number of symbols decoded from the 12-bit window (4..16)
+//   bits  5..9   4 x number of symbols decoded from the 12-bit window (4..20)
 //   bit  10      the window starts with no valid code (only in incomplete
 //                codes): decoded as one symbol 0 of 12 bits, and reported
-//   bits 16..31  up to four symbols, symbol i in bits 16+4i..19+4i
+//   bits 11..30  up to five symbols, symbol i in bits 11+4i..14+4i
+constexpr int kLutMaxSymbols = 5;
+constexpr int kLutSymShift = 11;
 __host__ __device__ constexpr uint32_t lut_bits(uint32_t e) { return e & 31u; }
 __host__ __device__ constexpr uint32_t lut_nibble_bits(uint32_t e) { return (e >> 5) & 31u; }
 constexpr uint32_t kLutInvalid = 1u << 10;
