@@ -90,6 +90,9 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
+// Bounded wait until *p == tag (a row published by another CTA of this call).
+__device__ __forceinline__ bool wait_tag(const unsigned long long* p, unsigned long long tag, uint64_t timeout_ns,
+                                         volatile int* abort);
 // Bounded wait until the counter shows `want` arrivals of call `tag`.
 __device__ __forceinline__ bool wait_counter(const unsigned long long* cnt, unsigned long long tag, unsigned want,
                                              uint64_t timeout_ns, volatile int* abort);
@@ -157,6 +160,23 @@ __device__ __forceinline__ bool wait_counter(const unsigned long long* cnt, unsi
             return false;
         }
         __nanosleep(200);
+    }
+}
+
+__device__ __forceinline__ bool wait_tag(const unsigned long long* p, unsigned long long tag, uint64_t timeout_ns,
+                                         volatile int* abort) {
+    uint64_t deadline = 0;
+    for (;;) {
+        if (ld_acquire_u64(p) == tag) return true;
+        if (abort && *abort) return false;
+        const uint64_t now = globaltimer();
+        if (deadline == 0) {
+            deadline = now + timeout_ns;
+        } else if (now > deadline) {
+            if (abort) *abort = 1;
+            return false;
+        }
+        __nanosleep(100);
     }
 }
 

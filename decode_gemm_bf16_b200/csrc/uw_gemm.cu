@@ -67,7 +67,7 @@ constexpr uint32_t kTileV = 16;                          // 128 verbatim flags
 struct GemmParams {
     int64_t M, N, K, KG;
     int MG, m_tiles, n_tiles, kt_count, P, stages;
-    int64_t total_iters;
+    uint32_t total_iters;
     uint32_t stage_bytes, off_a, off_b, off_sm, off_s2, off_v, tx_bytes;
     uint32_t tmem_cols;   // TMEM columns allocated (power of two)
     uint32_t a_col0;      // first TMEM column of the rebuilt-A stages (32 columns each)
@@ -79,7 +79,7 @@ struct GemmParams {
     void* Y;
     int out_f32;
     float* partial;                // [2P][128][MG]
-    unsigned long long* counters;  // [tiles][128]: (epoch << 16) | arrivals
+    unsigned long long* flags;     // [2P][128]: call tag once a slot's row is published
     unsigned long long epoch;      // 48-bit tag of this call
     // decoder running beside the GEMM: band b of 128 rows is ready when
     // band_ready[b] shows band_tasks(b) finished decoder tasks of this call
@@ -88,41 +88,49 @@ struct GemmParams {
     uint64_t timeout_ns;
 };
 
-__host__ __device__ __forceinline__ int64_t iter_begin(int64_t b, int64_t total, int64_t P) {
-    return b * total / P;
+// Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
+// the (tile, k step) sequence.  total * P < 2^32 is checked on the host.
+__host__ __device__ __forceinline__ uint32_t iter_begin(uint32_t b, uint32_t total, uint32_t P) {
+    return (uint32_t)(((uint64_t)b * total) / P);
 }
 // CTA that processes iteration i (the last b with iter_begin(b) <= i).
-__host__ __device__ __forceinline__ int64_t iter_owner(int64_t i, int64_t total, int64_t P) {
-    return ((i + 1) * P - 1) / total;
+__host__ __device__ __forceinline__ uint32_t iter_owner(uint32_t i, uint32_t total, uint32_t P) {
+    return (uint32_t)((((uint64_t)i + 1) * P - 1) / total);
+}
+// Partial-sum slot of CTA b's segment of `tile`: its first segment or its last.
+__device__ __forceinline__ uint32_t slot_of(uint32_t b, uint32_t tile, uint32_t total, uint32_t P, uint32_t kt) {
+    return 2u * b + ((iter_begin(b, total, P) / kt) == tile ? 0u : 1u);
 }
 
 struct Segment {
-    int64_t tile;
+    uint32_t tile;
     int kt0, kt1;
     bool first;   // first segment of this CTA's range
 };
 
 // Walks the segments of CTA b: [begin, end) cut at tile boundaries.
 struct SegWalker {
-    int64_t it, end;
-    int kt_count;
+    uint32_t it, end, kt_count;
     bool started = false;
-    __device__ SegWalker(int64_t b, const GemmParams& p)
+    __device__ SegWalker(uint32_t b, const GemmParams& p)
         : it(iter_begin(b, p.total_iters, p.P)), end(iter_begin(b + 1, p.total_iters, p.P)),
-          kt_count(p.kt_count) {}
+          kt_count((uint32_t)p.kt_count) {}
     __device__ bool next(Segment& s) {
         if (it >= end) return false;
         s.tile = it / kt_count;
-        s.kt0 = (int)(it % kt_count);
-        int64_t rest = end - it;
-        int64_t hi = (int64_t)s.kt0 + rest;
+        s.kt0 = (int)(it - s.tile * kt_count);
+        const uint32_t hi = (uint32_t)s.kt0 + (end - it);
         s.kt1 = (int)(hi < kt_count ? hi : kt_count);
         s.first = !started;
         started = true;
-        it += s.kt1 - s.kt0;
+        it += (uint32_t)(s.kt1 - s.kt0);
         return true;
     }
 };
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 // Offsets of 16-byte chunk c of row r in TMA tiles stored with a 64-byte
 // (rows of 64 B) or 32-byte (rows of 32 B) swizzle: chunk bits XOR address
@@ -365,33 +373,65 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         }
     } else if (warp < kEpiWarps) {
         // ------------------------------------------------------------ epilogue
+        // A tile cut between CTAs is finished by the CTA holding its first k
+        // steps (it reaches the tile last, at the end of its range): the other
+        // CTAs publish their fp32 partial rows with a per-row tag, the finisher
+        // waits for the tags, adds the partials to its own accumulator in k
+        // order and writes Y, then clears the tags for a replay of this call.
         SegWalker wk(blockIdx.x, p);
         Segment sg;
         int j = 0;
         const int r = warp * 32 + lane;
-        while (wk.next(sg)) {
-            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000)) break;
-            tc_fence_after();
+        bool ok = true;
+        while (ok && wk.next(sg)) {
             const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
             const int64_t n = (int64_t)n_tile * kBlockN + r;
             const int64_t m0 = (int64_t)m_tile * p.MG;
             const bool whole = sg.kt0 == 0 && sg.kt1 == p.kt_count;
-            const int64_t slot = 2 * (int64_t)blockIdx.x + (sg.first ? 0 : 1);
-            // partial sums: [slot][row][MG] so that a thread's row is contiguous
-            float* part = p.partial + (slot * kBlockN + r) * (int64_t)p.MG;
+            const bool finisher = !whole && sg.kt0 == 0;
+            const uint32_t kt = (uint32_t)p.kt_count;
+            const uint32_t b_last = finisher ? iter_owner(sg.tile * kt + kt - 1, p.total_iters, p.P) : 0u;
+            if (finisher) {
+                for (uint32_t b = blockIdx.x + 1; ok && b <= b_last; b++) {
+                    const uint32_t sl = slot_of(b, sg.tile, p.total_iters, p.P, kt);
+                    ok = wait_tag(p.flags + (size_t)sl * kBlockN + r, p.epoch, p.timeout_ns, abort_flag);
+                }
+                if (!ok) break;
+            }
+            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000)) break;
+            tc_fence_after();
+            const uint32_t slot = 2u * blockIdx.x + (sg.first ? 0u : 1u);
+            float* part = p.partial + ((size_t)slot * kBlockN + r) * p.MG;
             for (int c0 = 0; c0 < p.MG; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
                 tmem_wait_ld();
-                if (whole) {
+                if (whole || finisher) {
+                    float acc[16];
+#pragma unroll
+                    for (int i = 0; i < 16; i++) acc[i] = __uint_as_float(v[i]);
+                    for (uint32_t b = blockIdx.x + 1; finisher && b <= b_last; b++) {
+                        const uint32_t sl = slot_of(b, sg.tile, p.total_iters, p.P, kt);
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.partial + ((size_t)sl * kBlockN + r) * p.MG + c0);
+                        float4 q[4];
+#pragma unroll
+                        for (int i = 0; i < 4; i++) q[i] = __ldcg(src + i);
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            acc[4 * i] += q[i].x;
+                            acc[4 * i + 1] += q[i].y;
+                            acc[4 * i + 2] += q[i].z;
+                            acc[4 * i + 3] += q[i].w;
+                        }
+                    }
                     if (n < p.N) {
 #pragma unroll
                         for (int i = 0; i < 16; i++) {
-                            int64_t m = m0 + c0 + i;
+                            const int64_t m = m0 + c0 + i;
                             if (m < p.M) {
-                                float f = __uint_as_float(v[i]);
-                                if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = f;
-                                else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(f);
+                                if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc[i];
+                                else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc[i]);
                             }
                         }
                     }
@@ -406,51 +446,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(acce_bar));
-            if (!whole) {
-                // stream-K fix-up, one output row per thread: the last CTA to
-                // arrive sums every segment's partials in CTA order
-                const int64_t t0 = sg.tile * p.kt_count, t1 = t0 + p.kt_count - 1;
-                const int64_t b_first = iter_owner(t0, p.total_iters, p.P);
-                const int64_t b_last = iter_owner(t1, p.total_iters, p.P);
-                const int nsegs = (int)(b_last - b_first + 1);
-                __threadfence();
-                unsigned long long* cnt = p.counters + sg.tile * kBlockN + r;
-                if (arrive_counter(cnt, p.epoch) == (unsigned)nsegs) {
-                    __threadfence();
-                    for (int c0 = 0; c0 < p.MG; c0 += 16) {
-                        float acc[16];
-#pragma unroll
-                        for (int i = 0; i < 16; i++) acc[i] = 0.f;
-                        for (int64_t b = b_first; b <= b_last; b++) {
-                            const int64_t bs = iter_begin(b, p.total_iters, p.P);
-                            const int64_t sl = 2 * b + ((bs / p.kt_count) == sg.tile ? 0 : 1);
-                            const float4* src =
-                                reinterpret_cast<const float4*>(p.partial + (sl * kBlockN + r) * (int64_t)p.MG + c0);
-                            float4 q[4];
-#pragma unroll
-                            for (int i = 0; i < 4; i++) q[i] = __ldcg(src + i);
-#pragma unroll
-                            for (int i = 0; i < 4; i++) {
-                                acc[4 * i] += q[i].x;
-                                acc[4 * i + 1] += q[i].y;
-                                acc[4 * i + 2] += q[i].z;
-                                acc[4 * i + 3] += q[i].w;
-                            }
-                        }
-                        if (n < p.N) {
-#pragma unroll
-                            for (int i = 0; i < 16; i++) {
-                                int64_t m = m0 + c0 + i;
-                                if (m < p.M) {
-                                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc[i];
-                                    else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc[i]);
-                                }
-                            }
-                        }
-                    }
-                    *cnt = p.epoch << 16;   // count back to 0 for a replay of this call
-                }
-            }
+            if (!whole && !finisher) st_release_u64(p.flags + (size_t)slot * kBlockN + r, p.epoch);
+            if (finisher)
+                for (uint32_t b = blockIdx.x + 1; b <= b_last; b++)
+                    p.flags[(size_t)slot_of(b, sg.tile, p.total_iters, p.P, kt) * kBlockN + r] = 0ull;
             j++;
         }
     }
@@ -566,13 +565,13 @@ unsigned long long gemm_next_epoch() { return next_epoch(); }
 int gemm_status_take() { return unit_status_take(); }
 
 size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
+    (void)N;
     (void)K;
     int P = grid > 0 ? grid : gemm_default_grid();
     int MG = pick_mg(M);
-    int64_t m_tiles = (M + MG - 1) / MG, n_tiles = (N + kBlockN - 1) / kBlockN;
     size_t part = (size_t)2 * P * MG * kBlockN * 4;
-    size_t cnt = (size_t)m_tiles * n_tiles * kBlockN * 8;
-    return ((part + 255) & ~size_t(255)) + ((cnt + 255) & ~size_t(255));
+    size_t flags = (size_t)2 * P * kBlockN * 8;
+    return ((part + 255) & ~size_t(255)) + ((flags + 255) & ~size_t(255));
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
@@ -587,10 +586,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.m_tiles = (int)((a.M + p.MG - 1) / p.MG);
     p.n_tiles = (int)((a.N + kBlockN - 1) / kBlockN);
     p.kt_count = (int)(a.K / kBlockK);
-    int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
-    p.total_iters = tiles * p.kt_count;
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    const int64_t total = tiles * p.kt_count;
     int P = a.grid > 0 ? a.grid : gemm_default_grid();
-    if (P > p.total_iters) P = (int)p.total_iters;
+    if (P > total) P = (int)total;
+    if (total * (int64_t)P >= (int64_t(1) << 32)) { *st = UW_ERR_SHAPE; return cudaSuccess; }
+    p.total_iters = (uint32_t)total;
     p.P = P;
     p.vbits = a.vbits;
     p.vpre = a.vpre;
@@ -605,7 +606,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
     size_t part = (size_t)2 * P * p.MG * kBlockN * 4;
     p.partial = (float*)a.ws;
-    p.counters = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
+    p.flags = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
     p.epoch = a.epoch ? a.epoch : next_epoch();
     p.band_ready = a.band_ready;
     p.band_tasks = a.band_tasks;
@@ -717,7 +718,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
 // fix-up scratch (partial sums and per-row arrival tags) lives in the fixed
 // array below, compiled into the library: 4 MiB on every GPU that loads the
 // library, held until the process exits.  That covers batches up to 16 on a
-// 148-SM B200 for N up to about 200k rows.
+// 148-SM B200, for any N.
 // ===========================================================================
 namespace uw {
 namespace {

@@ -234,8 +234,7 @@ uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t
  *   X: device BF16 [M,K], 16-byte aligned; Y: device [M,N], BF16 or float32
  *   (out_f32), 16-byte aligned; the blob must hold the palette form.
  * Limits: returns UW_ERR_WORKSPACE, launching nothing, when the scratch this
- * call needs exceeds 4 MiB (on a 148-SM B200 that admits M <= 16 for N up to
- * about 200k rows).  The array's contents carry over from call to call; they
+ * call needs exceeds 4 MiB (on a 148-SM B200 that admits M <= 16, any N).  The array's contents carry over from call to call; they
  * need no clearing because every entry is tagged with its call.  All calls
  * share the one array, so calls that overlap on the GPU (other streams,
  * other threads) race: run them one at a time.  The first call on a device
