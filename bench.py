@@ -322,7 +322,7 @@ def run_gpu(args):
         "gemm_direct_palette": n + n // 2 + vstore + sec["vcol"][1] + xb + yb,
     }
     kernel_of = {"decode_full": "k_decode<full>", "decode_exponent": "k_decode<exponent>",
-                 "transcode": "k_decode<transcode>", "gemm_direct_palette": "k_gemm<palette>"}
+                 "transcode": "k_decode<transcode>", "gemm_direct_palette": "k_gemm_recon<palette>"}
     breakdown = {}
     for k, name in enumerate(OPS):
         d = {"us": 1e3 * per_op_ms[k], "eff_weight_gbs": 2.0 * n / (per_op_ms[k] / 1e3) / 1e9,
@@ -339,11 +339,16 @@ def run_gpu(args):
     dom = max(share, key=share.get)
     dom_ms = per_op_ms[OPS.index(dom)]
     achieved = alg[dom] / (dom_ms / 1e3) / 1e9
+    # DRAM bytes per launch from the committed ncu capture, only while the
+    # kernels are the ones that capture measured (same library sources)
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         try:
-            traffic = json.load(open(tp)).get(kernel_of[dom])
+            from decode_gemm_bf16_b200 import build as uwbuild
+            tj = json.load(open(tp))
+            if tj.get("source_hash") == uwbuild.source_hash():
+                traffic = tj["bytes_per_launch"].get(kernel_of[dom])
         except Exception:
             traffic = None
     launches_per_step = 3 + 2 + 2 + 2 + 1
