@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libunweight.so")
-SOURCES = ["uw_host.cpp", "uw_compress.cu", "uw_decode.cu", "uw_gemm.cu"]
+SOURCES = ["uw_host.cpp", "uw_compress.cu", "uw_decode.cu", "uw_gemm.cu", "uw_gemv.cu"]
 HEADERS = ["uw_internal.h", "uw_device.cuh", os.path.join("..", "..", "include", "unweight.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -6,12 +6,14 @@
 //   palette transcode -> 4-bit palette indices (a quarter).
 // §解壓與運算資源共享 gives the decoder a 16 KB Huffman table in shared
 // memory; here that table is a 4096-entry multi-symbol table (12-bit window ->
-// up to four symbols).
+// up to five symbols).
 //
 // Work split: a warp owns 32 consecutive 256-symbol segments (8192 weights).
 // Phase 1: lane l decodes segment l from its own start bit (chunk offset +
 // segment offset) into 32 words of packed nibbles in shared memory (rotated
-// by the lane index so that all lanes hit different banks).  Phase 2: the
+// by the lane index so that all lanes hit different banks).  The transcoder
+// first copies the task's stream words into shared memory (asynchronous
+// 16-byte copies, issued while the previous task writes its outputs).  Phase 2: the
 // warp walks its 8192 outputs in order, maps nibbles to exponents through the
 // palette (byte permutes), patches verbatim groups, merges the sign+mantissa
 // bytes and stores coalesced 16-byte vectors.
@@ -24,7 +26,18 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kBesideWarps = 4;                // decoder CTAs that share SMs with the GEMM
 constexpr int kTaskElems = 32 * kSeg;          // 8192 weights per warp task
-constexpr size_t kDecodeSmem = kLutSize * 4 + kWarps * 32 * 32 * 4;
+constexpr int kStreamCapW = 768;               // per-warp stream staging, words (3 KB)
+constexpr int kStageSmem = 32 * 32 * 4;        // per-warp decoded nibbles
+// The transcoder (the smallest output) is bound by its stream reads and
+// stages each task's stream bits in shared memory (3 CTAs per SM); the
+// other decoders keep 4 CTAs per SM and read the stream through L1.
+template <int MODE, int WARPS>
+constexpr bool kStaged = MODE == kDecodeTranscode && WARPS == kWarps;
+template <int MODE, int WARPS>
+constexpr size_t kWarpSmem = kStageSmem + (kStaged<MODE, WARPS> ? kStreamCapW * 4 : 0);
+template <int MODE, int WARPS>
+constexpr size_t kDecSmem = kLutSize * 4 + WARPS * kWarpSmem<MODE, WARPS>;
+static_assert(kDecodeBesideSmem == kLutSize * 4 + kBesideWarps * kStageSmem, "beside decoder smem");
 
 struct DecodeParams {
     const uint32_t* stream;
@@ -40,6 +53,7 @@ struct DecodeParams {
     int pal_small;   // all palette exponents < 128
     int64_t n;       // weights
     int64_t nseg;
+    uint64_t total_bits;
     void* out;
     unsigned long long* band_ready;   // optional: per-band finished-task counters
     unsigned long long epoch;
@@ -56,20 +70,28 @@ struct DecodeParams {
 // the prefetched word `nxt` tops the reservoir up.  Word reads are clamped to
 // the stream, so a corrupt stream cannot read outside it; an undecodable
 // window still advances (12 bits) and is reported once per segment.
-__device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint32_t* lut, int64_t seg, int nsym,
-                                               uint32_t* row, int rot) {
-    const uint64_t bitpos = __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
+template <bool SMEM>
+__device__ __forceinline__ uint32_t ldw(const uint32_t* sp, int64_t i) {
+    if (SMEM) return sp[i];
+    return __ldg(sp + i);
+}
+
+// `sp` = the stream words (global), or the warp's staged copy of them (SMEM);
+// `bitpos` counts from sp[0]; `last` = last readable word index.
+template <bool SMEM>
+__device__ __forceinline__ void decode_bits(const DecodeParams& p, const uint32_t* lut, const uint32_t* sp0,
+                                            int64_t last_word, uint64_t bitpos, int nsym, uint32_t* row, int rot) {
     const int64_t wi = (int64_t)(bitpos >> 5);
-    if (wi + 2 >= p.nwords) {
+    if (wi + 2 > last_word) {
         raise_status(UW_ERR_DEVICE);
         return;
     }
-    const uint32_t* __restrict__ sp = p.stream + wi;
-    const int64_t room = p.nwords - 1 - wi;
+    const uint32_t* __restrict__ sp = sp0 + wi;
+    const int64_t room = last_word - wi;
     const uint32_t last = room > 0x7FFFFFFF ? 0x7FFFFFFFu : (uint32_t)room;   // last readable index
     const uint32_t sh = (uint32_t)(bitpos & 31u);
-    const uint32_t w0 = __ldg(sp), w1 = __ldg(sp + 1);
-    uint32_t nxt = __ldg(sp + 2);                   // the bits right after lo's valid ones
+    const uint32_t w0 = ldw<SMEM>(sp, 0), w1 = ldw<SMEM>(sp, 1);
+    uint32_t nxt = ldw<SMEM>(sp, 2);                // the bits right after lo's valid ones
     uint32_t hi = __funnelshift_l(w1, w0, sh);      // stream bits [bitpos, bitpos + 32)
     uint32_t lo = w1 << sh;                         // rest of w1: 32 - sh valid bits
     int nlo = 32 - (int)sh;
@@ -91,7 +113,7 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
             hi |= nxt >> (32 + nlo);
             lo = nxt << (-nlo);
             nlo += 32;
-            nxt = __ldg(sp + min(idx, last));
+            nxt = ldw<SMEM>(sp, min(idx, last));
             idx++;
         }
         if (accn2 >= 32u) {
@@ -107,8 +129,41 @@ __device__ __forceinline__ void decode_segment(const DecodeParams& p, const uint
     if (flags & kLutInvalid) raise_status(UW_ERR_DEVICE);
 }
 
+__device__ __forceinline__ uint64_t segment_bitpos(const DecodeParams& p, int64_t seg) {
+    return seg < p.nseg ? __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]) : p.total_bits;
+}
+
+// Stream words of one warp task, staged into shared memory with 16-byte
+// asynchronous copies: [w0a, w0a + nw) with w0a a multiple of 4.  Copies never
+// leave the stream section (its allocation is rounded up to 256 bytes).
+struct Staging {
+    int64_t w0a;
+    int nw;
+    bool staged;
+};
+
+__device__ __forceinline__ Staging stage_stream(const DecodeParams& p, uint64_t first_bit, uint64_t end_bit,
+                                                uint32_t* sbuf, int lane) {
+    Staging g;
+    g.w0a = (int64_t)(first_bit >> 5) & ~int64_t(3);
+    int64_t wend = (int64_t)(end_bit >> 5) + 8;            // look-ahead of the bit reservoir
+    if (wend > p.nwords) wend = p.nwords;
+    wend = (wend + 3) & ~int64_t(3);
+    g.nw = (int)(wend - g.w0a);
+    g.staged = g.nw <= kStreamCapW;
+    if (g.staged) {
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(sbuf);
+        for (int i = lane * 4; i < g.nw; i += 128)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 4u * i), "l"(p.stream + g.w0a + i)
+                         : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    return g;
+}
+
 template <int MODE, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 4) k_decode(const DecodeParams p) {
+__global__ void __launch_bounds__(WARPS * 32, kStaged<MODE, WARPS> ? 3 : 4) k_decode(const DecodeParams p) {
+    constexpr bool STAGED = kStaged<MODE, WARPS>;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     uint32_t* stage = smem + kLutSize;
@@ -123,12 +178,25 @@ __global__ void __launch_bounds__(WARPS * 32, 4) k_decode(const DecodeParams p) 
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* st = stage + warp * 1024;
+    uint32_t* st = stage + warp * (kWarpSmem<MODE, WARPS> / 4);
+    uint32_t* sbuf = st + 32 * 32;
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
     const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
+    const int64_t stride = (int64_t)gridDim.x * WARPS;
 
-    for (int64_t task = (int64_t)blockIdx.x * WARPS + warp; task < ntasks;
-         task += (int64_t)gridDim.x * WARPS) {
+    // Staged (transcoder) software pipeline per warp: the stream bits of the
+    // next task are copied into shared memory (asynchronously) while this
+    // task's outputs are written; the next task's segment offsets load during
+    // this task's decode.
+    int64_t task = (int64_t)blockIdx.x * WARPS + warp;
+    uint64_t bitpos = 0;
+    Staging g = {0, 0, false};
+    if (STAGED && task < ntasks) {
+        bitpos = segment_bitpos(p, task * 32 + lane);
+        const uint64_t endb = lane == 31 ? segment_bitpos(p, task * 32 + 32) : 0;
+        g = stage_stream(p, __shfl_sync(0xFFFFFFFFu, bitpos, 0), __shfl_sync(0xFFFFFFFFu, endb, 31), sbuf, lane);
+    }
+    for (; task < ntasks; task += stride) {
         const int64_t base = task * kTaskElems;
         if (MODE == kDecodeFull) {
             // warm L2 with this task's sign+mantissa bytes, read in phase 2
@@ -138,15 +206,35 @@ __global__ void __launch_bounds__(WARPS * 32, 4) k_decode(const DecodeParams p) 
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(p.sm + off + 128));
             }
         }
+        const int64_t next = task + stride;
+        uint64_t nbit = 0, nend = 0;
+        if (STAGED && next < ntasks) {
+            nbit = segment_bitpos(p, next * 32 + lane);
+            if (lane == 31) nend = segment_bitpos(p, next * 32 + 32);
+        }
+        if (STAGED) {
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            __syncwarp();
+        }
         // ---- phase 1: one segment per lane
         {
-            int64_t seg = task * 32 + lane;
-            int64_t e0 = seg * kSeg;
-            int64_t left = p.n - e0;
-            int nsym = left <= 0 ? 0 : (left < kSeg ? (int)left : kSeg);
-            if (nsym > 0) decode_segment(p, lut, seg, nsym, st + lane * 32, lane);
+            const int64_t e0 = (task * 32 + lane) * (int64_t)kSeg;
+            const int64_t left = p.n - e0;
+            const int nsym = left <= 0 ? 0 : (left < kSeg ? (int)left : kSeg);
+            if (nsym > 0) {
+                if (STAGED && g.staged)
+                    decode_bits<true>(p, lut, sbuf, g.nw - 1, bitpos - (uint64_t)g.w0a * 32u, nsym, st + lane * 32, lane);
+                else {
+                    const int64_t seg = task * 32 + lane;
+                    const uint64_t bp = STAGED ? bitpos : __ldg(&p.chunk_off[seg >> 4]) + __ldg(&p.seg_rel[seg]);
+                    decode_bits<false>(p, lut, p.stream, p.nwords - 1, bp, nsym, st + lane * 32, lane);
+                }
+            }
         }
         __syncwarp();
+        if (STAGED && next < ntasks)
+            g = stage_stream(p, __shfl_sync(0xFFFFFFFFu, nbit, 0), __shfl_sync(0xFFFFFFFFu, nend, 31), sbuf, lane);
+        if (STAGED) bitpos = nbit;
         // ---- phase 2: ordered, coalesced output (offsets relative to the task)
         const int64_t left = p.n - base;
         const int lim = left < kTaskElems ? (int)left : kTaskElems;
@@ -244,6 +332,7 @@ static DecodeParams decode_params(const uw_blob* b, void* out) {
         if (b->palette[i] >= 128) p.pal_small = 0;
     p.n = b->geo.n;
     p.nseg = b->geo.nseg;
+    p.total_bits = b->total_bits;
     p.out = out;
     p.band_ready = nullptr;
     p.epoch = 0;
@@ -252,10 +341,13 @@ static DecodeParams decode_params(const uw_blob* b, void* out) {
 }
 
 template <int WARPS>
-static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid, size_t smem, cudaStream_t s) {
+static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid, cudaStream_t s) {
     void (*kern)(const DecodeParams) = mode == kDecodeFull       ? k_decode<kDecodeFull, WARPS>
                                        : mode == kDecodeExponent ? k_decode<kDecodeExponent, WARPS>
                                                                  : k_decode<kDecodeTranscode, WARPS>;
+    const size_t smem = mode == kDecodeFull       ? kDecSmem<kDecodeFull, WARPS>
+                        : mode == kDecodeExponent ? kDecSmem<kDecodeExponent, WARPS>
+                                                  : kDecSmem<kDecodeTranscode, WARPS>;
     static bool attr_set[3][64] = {{false}};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -287,10 +379,10 @@ cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, 
     DecodeParams p = decode_params(b, out);
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
     const int64_t need = (ntasks + kWarps - 1) / kWarps;
-    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * decode_ctas_per_sm();
+    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * (mode == kDecodeTranscode ? 3 : decode_ctas_per_sm());
     if (grid > need) grid = (int)need;
     if (grid < 1) grid = 1;
-    return launch_decode_impl<kWarps>(p, mode, grid, kDecodeSmem, s);
+    return launch_decode_impl<kWarps>(p, mode, grid, s);
 }
 
 cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas, unsigned long long* band_ready,
@@ -302,7 +394,7 @@ cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas
     const int64_t need = (ntasks + kBesideWarps - 1) / kBesideWarps;
     int grid = ctas > need ? (int)need : ctas;
     if (grid < 1) grid = 1;
-    return launch_decode_impl<kBesideWarps>(p, mode, grid, kDecodeBesideSmem, s);
+    return launch_decode_impl<kBesideWarps>(p, mode, grid, s);
 }
 
 int decode_status_take() { return unit_status_take(); }

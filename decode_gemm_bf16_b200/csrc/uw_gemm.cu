@@ -63,6 +63,7 @@ constexpr uint32_t kTileSM = kBlockN * kBlockK;          //  8 KB sign+mantissa
 constexpr uint32_t kTileE = kBlockN * kBlockK;           //  8 KB exponents
 constexpr uint32_t kTileIdx = kBlockN * kBlockK / 2;     //  4 KB palette indices
 constexpr uint32_t kTileV = 16;                          // 128 verbatim flags
+constexpr int kFinBufs = 4;                              // finisher staging rows in flight per warp
 
 struct GemmParams {
     int64_t M, N, K, KG;
@@ -78,7 +79,8 @@ struct GemmParams {
     uint32_t pal[4];
     void* Y;
     int out_f32;
-    float* partial;                // [2P][128][MG]
+    float* partial;                // [2P][MG/4][128][4]: float4 j of row r at (slot*MG/4 + j)*128 + r
+    int fin_cb;                    // finisher column block (16, 32 or 64)
     unsigned long long* flags;     // [2P][128]: call tag once a slot's row is published
     unsigned long long epoch;      // 48-bit tag of this call
     // decoder running beside the GEMM: band b of 128 rows is ready when
@@ -90,12 +92,13 @@ struct GemmParams {
 
 // Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
 // the (tile, k step) sequence.  total * P < 2^32 is checked on the host.
+// b <= P and i < total, so every product below is under 2^32.
 __host__ __device__ __forceinline__ uint32_t iter_begin(uint32_t b, uint32_t total, uint32_t P) {
-    return (uint32_t)(((uint64_t)b * total) / P);
+    return b * total / P;
 }
 // CTA that processes iteration i (the last b with iter_begin(b) <= i).
 __host__ __device__ __forceinline__ uint32_t iter_owner(uint32_t i, uint32_t total, uint32_t P) {
-    return (uint32_t)((((uint64_t)i + 1) * P - 1) / total);
+    return ((i + 1) * P - 1) / total;
 }
 // Partial-sum slot of CTA b's segment of `tile`: its first segment or its last.
 __device__ __forceinline__ uint32_t slot_of(uint32_t b, uint32_t tile, uint32_t total, uint32_t P, uint32_t kt) {
@@ -200,6 +203,111 @@ __device__ __forceinline__ void rebuild_row(const GemmParams& p, const uint8_t* 
 __device__ __forceinline__ uint16_t f2bf(float f) {
     __nv_bfloat16 h = __float2bfloat16_rn(f);
     return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// Y[m0 + i, n] for the 16 fp32 values v[i] (bit patterns) of output row n.
+__device__ __forceinline__ void store_y(void* Y, int64_t M, int64_t N, int out_f32, const uint32_t (&v)[16], int64_t n,
+                                        int64_t m0) {
+    if (n >= N || m0 >= M) return;
+    const int mv = M - m0 < 16 ? (int)(M - m0) : 16;
+    if (out_f32) {
+        float* y = reinterpret_cast<float*>(Y) + m0 * N + n;
+#pragma unroll
+        for (int i = 0; i < 16; i++, y += N)
+            if (i < mv) *y = __uint_as_float(v[i]);
+    } else {
+        uint16_t* y = reinterpret_cast<uint16_t*>(Y) + m0 * N + n;
+#pragma unroll
+        for (int i = 0; i < 16; i++, y += N)
+            if (i < mv) *y = f2bf(__uint_as_float(v[i]));
+    }
+}
+
+// Finisher of a split tile: own accumulator (TMEM) + the partial rows of
+// CTAs blockIdx.x + 1 .. b_last in that order, then Y.  Columns go in blocks
+// of CB; this warp's accumulator rows (32 x CB) and kFinBufs staging rows
+// live in `fin` (rows of CB + 4 floats: a 16-byte bank shift per lane), and
+// the (block, contributor) items stream in with asynchronous copies,
+// kFinBufs - 1 ahead.  Kept out of line: it runs once per CTA and would
+// otherwise set the register budget of the whole kernel.
+struct FinArgs {
+    const float* partial;
+    void* Y;
+    int64_t M, N;
+    int MG, CB, out_f32;
+    uint32_t total, P, kt;
+};
+
+__device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_t b_last, int64_t n, int64_t m0,
+                                         uint32_t trow, float* fin, int lane) {
+    const int CB = f.CB, RS = CB + 4;
+    const int MG4 = f.MG / 4;
+    const int r = (int)(threadIdx.x & 127);
+    const uint32_t nb = b_last - blockIdx.x;   // contributors, in k order after this CTA
+    const uint32_t nblk = (uint32_t)((f.MG + CB - 1) / CB);
+    const uint32_t items = nb * nblk;
+    float* facc = fin + lane * RS;
+    const uint32_t fbuf = smem_u32(fin + 32 * RS + lane * RS);   // staging rows, 32*RS floats apart
+    const float4* part4 = reinterpret_cast<const float4*>(f.partial);
+    // item t = (block t / nb, contributor t % nb) -> staging row t % kFinBufs;
+    // every call commits one group (possibly empty) so that groups count items
+    auto issue = [&](uint32_t t) {
+        if (t < items) {
+            const uint32_t blk = t / nb, i = t - blk * nb;
+            const int cb0 = (int)blk * CB;
+            const int cw = f.MG - cb0 < CB ? f.MG - cb0 : CB;
+            const uint32_t sl = slot_of(blockIdx.x + 1 + i, tile, f.total, f.P, f.kt);
+            const float4* src = part4 + ((size_t)sl * MG4 + cb0 / 4) * kBlockN + r;
+            const uint32_t dst = fbuf + (t % kFinBufs) * (uint32_t)(32 * RS * 4);
+            for (int q = 0; q < cw / 4; q++) cp_async16(dst + 16u * q, src + (size_t)q * kBlockN);
+        }
+        cp_async_commit();
+    };
+    for (uint32_t t = 0; t + 1 < (uint32_t)kFinBufs; t++) issue(t);
+    uint32_t t = 0;
+    for (uint32_t blk = 0; blk < nblk; blk++) {
+        const int cb0 = (int)blk * CB;
+        const int cw = f.MG - cb0 < CB ? f.MG - cb0 : CB;
+        for (int c = 0; c < cw; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(trow + (uint32_t)(cb0 + c), v);
+            tmem_wait_ld();
+            float4* a4 = reinterpret_cast<float4*>(facc + c);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                a4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+        for (uint32_t i = 0; i < nb; i++, t++) {
+            issue(t + kFinBufs - 1);
+            cp_async_wait<kFinBufs - 1>();   // item t has landed
+            const float4* b4 = reinterpret_cast<const float4*>(fin + (1 + t % kFinBufs) * 32 * RS + lane * RS);
+            float4* a4 = reinterpret_cast<float4*>(facc);
+            for (int q = 0; q < cw / 4; q++) {
+                float4 x = a4[q];
+                const float4 y = b4[q];
+                x.x += y.x;
+                x.y += y.y;
+                x.z += y.z;
+                x.w += y.w;
+                a4[q] = x;
+            }
+        }
+        for (int c = 0; c < cw; c += 16) {
+            uint32_t v[16];
+            const uint4* a4 = reinterpret_cast<const uint4*>(facc + c);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const uint4 x = a4[i];
+                v[4 * i] = x.x;
+                v[4 * i + 1] = x.y;
+                v[4 * i + 2] = x.z;
+                v[4 * i + 3] = x.w;
+            }
+            store_y(f.Y, f.M, f.N, f.out_f32, v, n, m0 + cb0 + c);
+        }
+    }
+    cp_async_wait<0>();
 }
 
 template <int SRC>
@@ -378,10 +486,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // CTAs publish their fp32 partial rows with a per-row tag, the finisher
         // waits for the tags, adds the partials to its own accumulator in k
         // order and writes Y, then clears the tags for a replay of this call.
+        // Partials are stored float4-interleaved across rows, so every warp
+        // access covers 512 contiguous bytes.  The finisher's segment is its
+        // CTA's last, so the stage ring is idle by then: it stages partial
+        // rows there with asynchronous copies (one round trip per block of
+        // columns and contributor instead of one per 16 columns).
         SegWalker wk(blockIdx.x, p);
         Segment sg;
         int j = 0;
         const int r = warp * 32 + lane;
+        const uint32_t trow = tacc + ((uint32_t)(warp * 32) << 16);
+        // finisher staging: this warp's 1 + kFinBufs rows-of-32 of fin_cb + 4 floats
+        float* fin = reinterpret_cast<float*>(smem) + (size_t)warp * (1 + kFinBufs) * 32 * (p.fin_cb + 4);
+        const int MG4 = p.MG / 4;
         bool ok = true;
         while (ok && wk.next(sg)) {
             const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
@@ -401,47 +518,28 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000)) break;
             tc_fence_after();
             const uint32_t slot = 2u * blockIdx.x + (sg.first ? 0u : 1u);
-            float* part = p.partial + ((size_t)slot * kBlockN + r) * p.MG;
-            for (int c0 = 0; c0 < p.MG; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-                tmem_wait_ld();
-                if (whole || finisher) {
-                    float acc[16];
-#pragma unroll
-                    for (int i = 0; i < 16; i++) acc[i] = __uint_as_float(v[i]);
-                    for (uint32_t b = blockIdx.x + 1; finisher && b <= b_last; b++) {
-                        const uint32_t sl = slot_of(b, sg.tile, p.total_iters, p.P, kt);
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.partial + ((size_t)sl * kBlockN + r) * p.MG + c0);
-                        float4 q[4];
-#pragma unroll
-                        for (int i = 0; i < 4; i++) q[i] = __ldcg(src + i);
-#pragma unroll
-                        for (int i = 0; i < 4; i++) {
-                            acc[4 * i] += q[i].x;
-                            acc[4 * i + 1] += q[i].y;
-                            acc[4 * i + 2] += q[i].z;
-                            acc[4 * i + 3] += q[i].w;
-                        }
-                    }
-                    if (n < p.N) {
-#pragma unroll
-                        for (int i = 0; i < 16; i++) {
-                            const int64_t m = m0 + c0 + i;
-                            if (m < p.M) {
-                                if (p.out_f32) reinterpret_cast<float*>(p.Y)[m * p.N + n] = acc[i];
-                                else reinterpret_cast<uint16_t*>(p.Y)[m * p.N + n] = f2bf(acc[i]);
-                            }
-                        }
-                    }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(part + c0);
+            if (whole) {
+                for (int c0 = 0; c0 < p.MG; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(trow + (uint32_t)c0, v);
+                    tmem_wait_ld();
+                    store_y(p.Y, p.M, p.N, p.out_f32, v, n, m0 + c0);
+                }
+            } else if (!finisher) {
+                // publish the partial rows
+                float4* dst = reinterpret_cast<float4*>(p.partial) + (size_t)slot * MG4 * kBlockN + r;
+                for (int c0 = 0; c0 < p.MG; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(trow + (uint32_t)c0, v);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; i++)
-                        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                        dst[(size_t)(c0 / 4 + i) * kBlockN] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
                 }
+            } else {
+                const FinArgs fa = {p.partial, p.Y, p.M, p.N, p.MG, p.fin_cb, p.out_f32, p.total_iters, (uint32_t)p.P, kt};
+                finish_tile(fa, sg.tile, b_last, n, m0, trow, fin, lane);
             }
             tc_fence_before();
             __syncwarp();
@@ -577,6 +675,7 @@ size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     *st = UW_OK;
     if (a.M == 0) return cudaSuccess;
+    if (a.M <= kGemvMaxM && !a.band_ready) return launch_gemv(a, s, st);
     GemmParams p{};
     p.M = a.M;
     p.N = a.N;
@@ -651,6 +750,14 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.stages = S;
+    // finisher staging in the idle ring: 4 warps x (1 + kFinBufs) rows-of-32 x (CB + 4) floats
+    p.fin_cb = 0;
+    for (int cb = 64; cb >= 16; cb >>= 1)
+        if (cb <= p.MG && (size_t)4 * (1 + kFinBufs) * 32 * (cb + 4) * 4 <= (size_t)S * p.stage_bytes) {
+            p.fin_cb = cb;
+            break;
+        }
+    if (p.fin_cb == 0) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.a_col0 = acc_cols;
     uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + 32u * (uint32_t)S;
     p.tmem_cols = 32;

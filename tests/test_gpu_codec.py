@@ -24,6 +24,17 @@ def _constructed():
     return ((ex.astype(np.uint16) << 7) | rng.integers(0, 128, N * K).astype(np.uint16)).reshape(N, K)
 
 
+def _high_entropy(N, K):
+    """Rows 0-31: sixteen exponents drawn uniformly (4 bits a symbol, more
+    stream bits per 8192-weight block than typical weights need); the rest
+    Gaussian.  Decoders see both dense and sparse stretches of the stream."""
+    rng = np.random.default_rng(12)
+    W = S.gaussian_weight(N, K, seed=24)
+    ex = rng.integers(112, 128, 32 * K).astype(np.uint16)
+    W[:32] = ((ex << 7) | rng.integers(0, 0x8080, 32 * K).astype(np.uint16) & 0x807F).reshape(32, K)
+    return W
+
+
 MATRICES = {
     "small_512x2048": lambda: S.small_matrix()[0],
     "every_pattern_1024x64": S.all_bf16_patterns,
@@ -34,6 +45,7 @@ MATRICES = {
     "ragged_37x320": lambda: S.gaussian_weight(37, 320, seed=21),
     "ragged_300x1408": lambda: S.weight_with_verbatim_rows(300, 1408, seed=22, frac_groups=0.02),
     "no_verbatim_16x4096": lambda: S.gaussian_weight(16, 4096, seed=23, std=0.5),
+    "high_entropy_96x4096": lambda: _high_entropy(96, 4096),
 }
 
 _cache = {}
