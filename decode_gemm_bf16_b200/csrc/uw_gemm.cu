@@ -105,6 +105,19 @@ __device__ __forceinline__ uint32_t slot_of(uint32_t b, uint32_t tile, uint32_t 
     return 2u * b + ((iter_begin(b, total, P) / kt) == tile ? 0u : 1u);
 }
 
+// Position in the stage ring: slot and phase parity of iteration q, advanced
+// one iteration at a time (no division in the per-stage loops).
+struct RingPos {
+    int s = 0;
+    uint32_t ph = 0;
+    __device__ __forceinline__ void advance(int S) {
+        if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+};
+
 struct Segment {
     uint32_t tile;
     int kt0, kt1;
@@ -370,6 +383,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             SegWalker wk(blockIdx.x, p);
             Segment sg;
             int64_t q = 0;
+            RingPos rp;
             bool ok = true;
             int ready_band = -1;
             while (ok && wk.next(sg)) {
@@ -383,10 +397,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     fence_proxy_async_global();
                     ready_band = n_tile;
                 }
-                for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
-                    const int s = (int)(q % S);
-                    const uint32_t ph = (uint32_t)((q / S) & 1);
-                    if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
+                for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
+                    const int s = rp.s;
+                    if (!mbar_wait(smem_u32(&empty_bar[s]), rp.ph ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
@@ -416,28 +429,31 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             const uint32_t idesc = mma_idesc_bf16(kBlockN, p.MG);
             SegWalker wk(blockIdx.x, p);
             Segment sg;
-            int64_t q = 0;
+            RingPos rp;
             int j = 0;
             bool ok = true;
             while (ok && wk.next(sg)) {
                 if (!mbar_wait(smem_u32(acce_bar), (uint32_t)(j & 1) ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
-                    const int s = (int)(q % S);
-                    const uint32_t ph = (uint32_t)((q / S) & 1);
+                for (int kt = sg.kt0; kt < sg.kt1; kt++, rp.advance(S)) {
+                    const int s = rp.s;
                     const uint32_t wb = kRecon ? smem_u32(&recon_bar[s]) : smem_u32(&full_bar[s]);
-                    if (!mbar_wait(wb, ph, p.timeout_ns, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(wb, rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_base + s * p.stage_bytes;
+                    // 16 k = 32 bytes further along a swizzled row: +2 in the
+                    // descriptor's start-address field (16-byte units)
+                    const uint64_t bd0 = sw128_desc(st + p.off_b);
+                    const uint64_t ad0 = sw128_desc(st + p.off_a);
+                    const uint32_t ta0 = tacc + p.a_col0 + 32u * (uint32_t)s;
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; kk++) {
-                        const uint64_t bd = sw128_desc(st + p.off_b + kk * 32);
                         const uint32_t acc = (kt > sg.kt0 || kk > 0) ? 1u : 0u;
                         if (kRecon) {
                             // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
-                            tc_mma_tmem_a(tacc, tacc + p.a_col0 + 32u * (uint32_t)s + 8u * kk, bd, idesc, acc);
+                            tc_mma_tmem_a(tacc, ta0 + 8u * kk, bd0 + 2u * kk, idesc, acc);
                         } else {
-                            tc_mma(tacc, sw128_desc(st + p.off_a + kk * 32), bd, idesc, acc);
+                            tc_mma(tacc, ad0 + 2u * kk, bd0 + 2u * kk, idesc, acc);
                         }
                     }
                     tc_commit(smem_u32(&empty_bar[s]));
@@ -462,15 +478,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0 + 16u * (uint32_t)h;
         SegWalker wk(blockIdx.x, p);
         Segment sg;
-        int64_t q = 0;
+        uint32_t q = 0;
+        RingPos rp;
         bool ok = true;
         while (ok && wk.next(sg)) {
             const int64_t n0 = (sg.tile / p.m_tiles) * kBlockN;
-            for (int kt = sg.kt0; kt < sg.kt1; kt++, q++) {
+            for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
                 if ((int)(q & 1) != group) continue;
-                const int s = (int)(q % S);
-                const uint32_t ph = (uint32_t)((q / S) & 1);
-                if (!mbar_wait(smem_u32(&full_bar[s]), ph, p.timeout_ns, abort_flag)) { ok = false; break; }
+                const int s = rp.s;
+                if (!mbar_wait(smem_u32(&full_bar[s]), rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
                 rebuild_row<SRC>(p, smem + (size_t)s * p.stage_bytes, n0, kt, quarter, h, lane,
                                  tlane + 32u * (uint32_t)s);
                 tmem_wait_st();
