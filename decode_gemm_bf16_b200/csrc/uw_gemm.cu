@@ -48,7 +48,7 @@ namespace uw {
 namespace {
 
 constexpr int kBlockN = 128;   // weight rows per tile (MMA M)
-constexpr int kBlockK = 64;    // k per stage: one 128-byte swizzle row of BF16
+constexpr int kBoxK = 64;      // k per TMA box of BF16: one 128-byte swizzle row
 constexpr int kEpiWarps = 4;
 constexpr int kProdWarp = 4;
 constexpr int kMmaWarp = 5;
@@ -58,11 +58,10 @@ constexpr int kReconGroupWarps = 8;
 constexpr int kMaxStages = 8;
 constexpr int kThreadsDense = 6 * 32;
 constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
-constexpr uint32_t kTileA = kBlockN * kBlockK * 2;       // 16 KB BF16 weight tile (dense source)
-constexpr uint32_t kTileSM = kBlockN * kBlockK;          //  8 KB sign+mantissa
-constexpr uint32_t kTileE = kBlockN * kBlockK;           //  8 KB exponents
-constexpr uint32_t kTileIdx = kBlockN * kBlockK / 2;     //  4 KB palette indices
-constexpr uint32_t kTileV = 16;                          // 128 verbatim flags
+// Per stage of KB k (KB = 64 or 128): BF16 weight tile 128 x KB (dense
+// source), sign+mantissa 128 x KB bytes, exponents 128 x KB bytes or palette
+// indices 128 x KB/2 bytes, and KB/64 words of 128 verbatim flags.
+constexpr uint32_t kTileA64 = kBlockN * kBoxK * 2;       // 16 KB: one 64-k box of BF16 weights
 constexpr int kFinBufs = 4;                              // finisher staging rows in flight per warp
 
 struct GemmParams {
@@ -148,56 +147,61 @@ __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned l
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Offsets of 16-byte chunk c of row r in TMA tiles stored with a 64-byte
-// (rows of 64 B) or 32-byte (rows of 32 B) swizzle: chunk bits XOR address
-// bits 7 and up.
+// Offsets of 16-byte chunk c of row r in TMA tiles stored with a 128-byte,
+// 64-byte or 32-byte swizzle (rows of that many bytes): chunk bits XOR
+// address bits 7 and up.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 __device__ __forceinline__ uint32_t sw64_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 __device__ __forceinline__ uint32_t sw32_off(int r, int c) { return r * 32 + ((c ^ ((r >> 2) & 1)) << 4); }
 
-// Rebuilds weight row r = 32q + lane, k = 32h .. 32h+31 of the stage's tile
-// and writes it to TMEM lane r, columns taddr_cols .. +15 (one BF16 pair per
-// column).
-template <int SRC>
+// Rebuilds weight row r = 32q + lane, k = 32j .. 32j+31 of the stage's tile
+// (stage of KB k at stage index kt) and writes it to TMEM lane r, columns
+// taddr .. +15 (one BF16 pair per column).  Sign+mantissa and exponent
+// tiles have rows of KB bytes (swizzle KB), index tiles rows of KB/2 bytes.
+template <int SRC, int KB>
 __device__ __forceinline__ void rebuild_row(const GemmParams& p, const uint8_t* stage, int64_t n0, int kt,
-                                            int q, int h, int lane, uint32_t taddr) {
+                                            int q, int j, int lane, uint32_t taddr) {
     const int r = 32 * q + lane;
+    auto row_off = [&](int c) { return KB == 128 ? sw128_off(r, c) : sw64_off(r, c); };
     const uint8_t* SM = stage + p.off_sm;
-    const uint4 s0 = *reinterpret_cast<const uint4*>(SM + sw64_off(r, 2 * h));
-    const uint4 s1 = *reinterpret_cast<const uint4*>(SM + sw64_off(r, 2 * h + 1));
+    const uint4 s0 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j));
+    const uint4 s1 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j + 1));
     uint32_t E[8];
     if (SRC == kSrcExponent) {
         const uint8_t* EX = stage + p.off_s2;
-        const uint4 e0 = *reinterpret_cast<const uint4*>(EX + sw64_off(r, 2 * h));
-        const uint4 e1 = *reinterpret_cast<const uint4*>(EX + sw64_off(r, 2 * h + 1));
+        const uint4 e0 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j));
+        const uint4 e1 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j + 1));
         E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
         E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
     } else {
-        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + p.off_v + 4 * q);
+        const int grp = j >> 1;   // 64-weight group within the stage
+        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + p.off_v + 16 * grp + 4 * q);
         if ((vw >> lane) & 1u) {
             // verbatim group: raw exponents from the verbatim store
-            const int64_t g = (n0 + r) * p.KG + kt;
+            const int64_t g = (n0 + r) * p.KG + (int64_t)kt * (KB / kGroup) + grp;
             const uint32_t w = __ldg(&p.vbits[g >> 5]);
             const int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
-            const uint4* src = reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + 32 * h);
+            const uint4* src = reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + 32 * (j & 1));
             const uint4 e0 = __ldg(src), e1 = __ldg(src + 1);
             E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
             E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
         } else {
-            const uint4 ix = *reinterpret_cast<const uint4*>(stage + p.off_s2 + sw32_off(r, h));
+            const uint4 ix = *reinterpret_cast<const uint4*>(
+                stage + p.off_s2 + (KB == 128 ? sw64_off(r, j) : sw32_off(r, j)));
             const uint32_t w[4] = {ix.x, ix.y, ix.z, ix.w};
             const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
             if (p.pal_small) {
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const uint32_t xs = w[j] ^ 0x88888888u;
-                    E[2 * j] = palette4_small(w[j], xs, P0, P1, P2, P3);
-                    E[2 * j + 1] = palette4_small(w[j] >> 16, xs >> 16, P0, P1, P2, P3);
+                for (int i = 0; i < 4; i++) {
+                    const uint32_t xs = w[i] ^ 0x88888888u;
+                    E[2 * i] = palette4_small(w[i], xs, P0, P1, P2, P3);
+                    E[2 * i + 1] = palette4_small(w[i] >> 16, xs >> 16, P0, P1, P2, P3);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    E[2 * j] = palette4(w[j], P0, P1, P2, P3);
-                    E[2 * j + 1] = palette4(w[j] >> 16, P0, P1, P2, P3);
+                for (int i = 0; i < 4; i++) {
+                    E[2 * i] = palette4(w[i], P0, P1, P2, P3);
+                    E[2 * i + 1] = palette4(w[i] >> 16, P0, P1, P2, P3);
                 }
             }
         }
@@ -205,10 +209,10 @@ __device__ __forceinline__ void rebuild_row(const GemmParams& p, const uint8_t* 
     const uint32_t S[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
     uint32_t out[16];
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const uint2 m = merge4(E[j], S[j]);
-        out[2 * j] = m.x;
-        out[2 * j + 1] = m.y;
+    for (int i = 0; i < 8; i++) {
+        const uint2 m = merge4(E[i], S[i]);
+        out[2 * i] = m.x;
+        out[2 * i + 1] = m.y;
     }
     tmem_st16(taddr, out);
 }
@@ -323,9 +327,11 @@ __device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_
     cp_async_wait<0>();
 }
 
-template <int SRC>
+template <int SRC, int KB>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_a, const CUtensorMap& tm_s2,
                                           const CUtensorMap& tm_v, const GemmParams& p) {
+    static_assert(KB == 64 || KB == 128, "stage k");
+    constexpr int kHalves = KB / kBoxK;   // 64-k boxes of X (and of dense W) per stage
     constexpr bool kRecon = SRC != kSrcDense;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -403,16 +409,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
-                    tma_load_2d(st + p.off_b, &tm_x, kt * kBlockK, m_tile * p.MG, fb);
+#pragma unroll
+                    for (int hb = 0; hb < kHalves; hb++)
+                        tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, fb);
                     if (SRC == kSrcDense) {
-                        tma_load_2d(st + p.off_a, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
+#pragma unroll
+                        for (int hb = 0; hb < kHalves; hb++)
+                            tma_load_2d(st + p.off_a + hb * kTileA64, &tm_a, kt * KB + hb * kBoxK, n_tile * kBlockN, fb);
                     } else {
-                        tma_load_2d(st + p.off_sm, &tm_a, kt * kBlockK, n_tile * kBlockN, fb);
+                        tma_load_2d(st + p.off_sm, &tm_a, kt * KB, n_tile * kBlockN, fb);
                         if (SRC == kSrcExponent)
-                            tma_load_2d(st + p.off_s2, &tm_s2, kt * kBlockK, n_tile * kBlockN, fb);
+                            tma_load_2d(st + p.off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
                         else {
-                            tma_load_2d(st + p.off_s2, &tm_s2, kt * (kBlockK / 2), n_tile * kBlockN, fb);
-                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt, fb);
+                            tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
+                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
                         }
                     }
                 }
@@ -443,17 +453,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     // 16 k = 32 bytes further along a swizzled row: +2 in the
                     // descriptor's start-address field (16-byte units)
-                    const uint64_t bd0 = sw128_desc(st + p.off_b);
-                    const uint64_t ad0 = sw128_desc(st + p.off_a);
-                    const uint32_t ta0 = tacc + p.a_col0 + 32u * (uint32_t)s;
+                    const uint32_t ta0 = tacc + p.a_col0 + (uint32_t)(KB / 2) * (uint32_t)s;
 #pragma unroll
-                    for (int kk = 0; kk < kBlockK / 16; kk++) {
-                        const uint32_t acc = (kt > sg.kt0 || kk > 0) ? 1u : 0u;
-                        if (kRecon) {
-                            // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
-                            tc_mma_tmem_a(tacc, ta0 + 8u * kk, bd0 + 2u * kk, idesc, acc);
-                        } else {
-                            tc_mma(tacc, ad0 + 2u * kk, bd0 + 2u * kk, idesc, acc);
+                    for (int hb = 0; hb < kHalves; hb++) {
+                        const uint64_t bd0 = sw128_desc(st + p.off_b + hb * p.MG * 128);
+                        const uint64_t ad0 = sw128_desc(st + p.off_a + hb * kTileA64);
+#pragma unroll
+                        for (int kk = 0; kk < kBoxK / 16; kk++) {
+                            const uint32_t acc = (kt > sg.kt0 || hb > 0 || kk > 0) ? 1u : 0u;
+                            if (kRecon) {
+                                // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
+                                tc_mma_tmem_a(tacc, ta0 + 8u * (uint32_t)(hb * 4 + kk), bd0 + 2u * kk, idesc, acc);
+                            } else {
+                                tc_mma(tacc, ad0 + 2u * kk, bd0 + 2u * kk, idesc, acc);
+                            }
                         }
                     }
                     tc_commit(smem_u32(&empty_bar[s]));
@@ -471,11 +484,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // ------------------------------------------------------------ reconstruct
         // warp w may only touch TMEM lanes 32(w%4)..+31.  Two groups of 8
         // warps take alternate stages (two stages rebuilt at once); inside a
-        // group, two warps per lane quarter, one per half of the k step.
+        // group, two warps per lane quarter, one per half of the stage's k
+        // (one or two 32-k pieces each).
+        constexpr int kPieces = KB / 64;   // 32-k pieces per warp and stage
         const int rw = warp - kReconWarp0;
         const int group = rw / kReconGroupWarps;
         const int quarter = warp & 3, h = (rw % kReconGroupWarps) >> 2;
-        const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0 + 16u * (uint32_t)h;
+        const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0;
         SegWalker wk(blockIdx.x, p);
         Segment sg;
         uint32_t q = 0;
@@ -487,8 +502,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 if ((int)(q & 1) != group) continue;
                 const int s = rp.s;
                 if (!mbar_wait(smem_u32(&full_bar[s]), rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
-                rebuild_row<SRC>(p, smem + (size_t)s * p.stage_bytes, n0, kt, quarter, h, lane,
-                                 tlane + 32u * (uint32_t)s);
+#pragma unroll
+                for (int pc = 0; pc < kPieces; pc++) {
+                    const int j = h * kPieces + pc;
+                    rebuild_row<SRC, KB>(p, smem + (size_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
+                                         tlane + (uint32_t)(KB / 2) * (uint32_t)s + 16u * (uint32_t)j);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -578,21 +597,22 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 }
 
 // Dense source: 6 warps, registers unconstrained.
+template <int KB>
 __global__ void __launch_bounds__(kThreadsDense, 1)
     k_gemm_dense(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
                  const GemmParams p) {
-    gemm_body<kSrcDense>(tm_x, tm_a, tm_s2, tm_v, p);
+    gemm_body<kSrcDense, KB>(tm_x, tm_a, tm_s2, tm_v, p);
 }
 
 // Rebuilding sources: 22 warps held to 72 registers, which leaves one warp's
 // worth of registers per SM sub-partition for a decoder CTA running beside.
-template <int SRC>
+template <int SRC, int KB>
 __global__ void __maxnreg__(72)
     k_gemm_recon(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
                  const GemmParams p) {
-    gemm_body<SRC>(tm_x, tm_a, tm_s2, tm_v, p);
+    gemm_body<SRC, KB>(tm_x, tm_a, tm_s2, tm_v, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -696,11 +716,15 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.M = a.M;
     p.N = a.N;
     p.K = a.K;
-    p.KG = a.K / kBlockK;
+    p.KG = a.K / kGroup;
     p.MG = pick_mg(a.M);
+    // stage k: 128 for small batch tiles (halves the per-stage TMA, barrier
+    // and MMA-issue overhead per weight byte), 64 where a stage is already
+    // large (batch tiles above 64 rows)
+    const int KB = (p.MG <= 64 && a.K % 128 == 0) ? 128 : 64;
     p.m_tiles = (int)((a.M + p.MG - 1) / p.MG);
     p.n_tiles = (int)((a.N + kBlockN - 1) / kBlockN);
-    p.kt_count = (int)(a.K / kBlockK);
+    p.kt_count = (int)(a.K / KB);
     const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
     const int64_t total = tiles * p.kt_count;
     int P = a.grid > 0 ? a.grid : gemm_default_grid();
@@ -729,26 +753,28 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.timeout_ns = timeout_ns();
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
-    const uint32_t b_bytes = (uint32_t)p.MG * 128;
+    const int halves = KB / kBoxK;
+    const uint32_t b_bytes = (uint32_t)p.MG * 128 * halves;
     auto al1k = [](uint32_t x) { return (x + 1023u) & ~1023u; };
     uint32_t off = 0;
     p.tx_bytes = b_bytes;
     if (a.src == kSrcDense) {
         p.off_a = 0;
-        p.off_b = kTileA;
-        off = kTileA + b_bytes;
-        p.tx_bytes += kTileA;
+        p.off_b = kTileA64 * halves;
+        off = p.off_b + b_bytes;
+        p.tx_bytes += kTileA64 * halves;
     } else {
+        const uint32_t sm_bytes = kBlockN * KB, idx_bytes = kBlockN * KB / 2, v_bytes = 16 * halves;
         p.off_b = 0;
         p.off_sm = al1k(b_bytes);
-        p.off_s2 = p.off_sm + kTileSM;
+        p.off_s2 = p.off_sm + sm_bytes;
         if (a.src == kSrcExponent) {
-            off = p.off_s2 + kTileE;
-            p.tx_bytes += kTileSM + kTileE;
+            off = p.off_s2 + sm_bytes;
+            p.tx_bytes += 2 * sm_bytes;
         } else {
-            p.off_v = al1k(p.off_s2 + kTileIdx);
-            off = p.off_v + kTileV;
-            p.tx_bytes += kTileSM + kTileIdx + kTileV;
+            p.off_v = al1k(p.off_s2 + idx_bytes);
+            off = p.off_v + v_bytes;
+            p.tx_bytes += sm_bytes + idx_bytes + v_bytes;
         }
     }
     p.stage_bytes = al1k(off);
@@ -761,7 +787,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     uint32_t acc_cols = 32;
     while (acc_cols < (uint32_t)p.MG) acc_cols <<= 1;
     if (a.src != kSrcDense) {
-        const int s_tmem = (int)((512u - acc_cols) / 32u);
+        const int s_tmem = (int)((512u - acc_cols) / (uint32_t)(KB / 2));
         if (S > s_tmem) S = s_tmem;
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
@@ -775,7 +801,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
         }
     if (p.fin_cb == 0) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.a_col0 = acc_cols;
-    uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + 32u * (uint32_t)S;
+    uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + (uint32_t)(KB / 2) * (uint32_t)S;
     p.tmem_cols = 32;
     while (p.tmem_cols < need_cols) p.tmem_cols <<= 1;
     if (p.tmem_cols > 512) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
@@ -786,32 +812,42 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     size_t smem = (size_t)S * p.stage_bytes + ctrl + 1024;
 
     CUtensorMap tx{}, ta{}, ts2{}, tv{};
-    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBlockK, p.MG,
+    bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBoxK, p.MG,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (a.src == kSrcDense) {
-        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, a.K, a.N, a.K * 2, kBlockK, kBlockN,
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, a.K, a.N, a.K * 2, kBoxK, kBlockN,
                                CU_TENSOR_MAP_SWIZZLE_128B);
         ts2 = ta;
         tv = ta;
     } else {
-        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, kBlockK, kBlockN,
-                               CU_TENSOR_MAP_SWIZZLE_64B);
+        // byte planes: rows of KB bytes (swizzle KB), index rows of KB/2 bytes
+        const CUtensorMapSwizzle swz = KB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+        const CUtensorMapSwizzle swz_i = KB == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, KB, kBlockN, swz);
         if (a.src == kSrcExponent) {
-            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, kBlockK, kBlockN,
-                                   CU_TENSOR_MAP_SWIZZLE_64B);
+            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, KB, kBlockN, swz);
             tv = ts2;
         } else {
             int64_t NW = 4 * ((a.N + 127) / 128);
-            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.idx, a.K / 2, a.N, a.K / 2, kBlockK / 2,
-                                   kBlockN, CU_TENSOR_MAP_SWIZZLE_32B);
-            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kBlockK, NW * 4, 4, 1,
-                                   CU_TENSOR_MAP_SWIZZLE_NONE);
+            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.idx, a.K / 2, a.N, a.K / 2, KB / 2,
+                                   kBlockN, swz_i);
+            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kGroup, NW * 4, 4,
+                                   KB / kGroup, CU_TENSOR_MAP_SWIZZLE_NONE);
         }
     }
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
 
-    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams) =
-        a.src == kSrcDense ? k_gemm_dense : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent> : k_gemm_recon<kSrcPalette>;
+    typedef void (*GemmKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                               const GemmParams);
+    GemmKernel kern;
+    if (KB == 128)
+        kern = a.src == kSrcDense      ? k_gemm_dense<128>
+               : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent, 128>
+                                       : k_gemm_recon<kSrcPalette, 128>;
+    else
+        kern = a.src == kSrcDense      ? k_gemm_dense<64>
+               : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent, 64>
+                                       : k_gemm_recon<kSrcPalette, 64>;
     cudaError_t e = set_smem_attr((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
