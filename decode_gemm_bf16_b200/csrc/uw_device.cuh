@@ -61,6 +61,17 @@ __device__ __forceinline__ uint2 merge4(uint32_t E, uint32_t S) {
     return make_uint2(prmt(lo, hi, 0x5140u), prmt(lo, hi, 0x7362u));
 }
 
+// One lane of a converged warp (the others get false).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

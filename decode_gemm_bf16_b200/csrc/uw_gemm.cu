@@ -385,7 +385,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 
     if (warp == kProdWarp) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // The whole warp walks the loop (its state stays warp-uniform); one
+        // elected lane issues the transfers.
+        {
+            const bool leader = elect_one();
             SegWalker wk(blockIdx.x, p);
             Segment sg;
             int64_t q = 0;
@@ -408,6 +411,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     if (!mbar_wait(smem_u32(&empty_bar[s]), rp.ph ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
+                    if (!leader) continue;
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
 #pragma unroll
                     for (int hb = 0; hb < kHalves; hb++)
@@ -435,7 +439,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp walks the loop; one elected lane issues the MMAs
+        // and commits.
+        {
+            const bool leader = elect_one();
             const uint32_t idesc = mma_idesc_bf16(kBlockN, p.MG);
             SegWalker wk(blockIdx.x, p);
             Segment sg;
@@ -454,6 +461,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     // 16 k = 32 bytes further along a swizzled row: +2 in the
                     // descriptor's start-address field (16-byte units)
                     const uint32_t ta0 = tacc + p.a_col0 + (uint32_t)(KB / 2) * (uint32_t)s;
+                    if (!leader) continue;
 #pragma unroll
                     for (int hb = 0; hb < kHalves; hb++) {
                         const uint64_t bd0 = sw128_desc(st + p.off_b + hb * p.MG * 128);
@@ -472,11 +480,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     tc_commit(smem_u32(&empty_bar[s]));
                 }
                 if (!ok) break;
-                tc_commit(smem_u32(accf_bar));
+                if (leader) tc_commit(smem_u32(accf_bar));
                 j++;
             }
             // drain the tensor core before TMEM is released
-            tc_commit(smem_u32(final_bar));
+            if (leader) tc_commit(smem_u32(final_bar));
             mbar_wait(smem_u32(final_bar), 0, p.timeout_ns, nullptr);
         }
         __syncwarp();
