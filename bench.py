@@ -7,6 +7,9 @@ One step = the whole per-call hot path over one batch:
   palette) with x[1, 4096].
 value = effective BF16 weight bytes delivered per second over the step
 (7 x 2*N*K bytes per step / step time), whole job (all ranks).
+The line also carries a batch sweep outside the timed step: the tensor-core
+GEMM (direct palette, exponent pipeline, dense BF16) at M = 16 ... 1024 on
+the same projection, each timed alone over rotated copies.
 
 Inputs larger than L2: four compressed copies of W (~110 MB each) are
 rotated so that an op never finds its inputs left in L2 by the previous use.
@@ -175,6 +178,61 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def uw_gemv_serves():
+    """Whether batch 1 on this projection runs the CUDA-core GEMV (the
+    library's rule: fewer than half as many 128-row tiles as GEMM CTAs)."""
+    import torch
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return 2 * ((N_W + 127) // 128) < sms
+
+
+def batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak):
+    """Tensor-core GEMM at larger batches on the same projection (outside the
+    timed step): per M and pipeline, device time of one call (graph replays
+    over the rotated copies), TFLOP/s against the measured dense BF16 peak
+    and effective BF16 weight GB/s."""
+    import numpy as np
+    n = N_W * K_W
+    Wd = torch.from_numpy(S.gate_projection().view(np.int16)).to(dev).view(torch.bfloat16)
+    dense = [Wd] + [Wd.clone() for _ in range(3)]
+    out = {}
+    for M in (16, 64, 256, 1024):
+        X = torch.from_numpy(S.activations(M, K_W, seed=M + S.X_SEED_OFFSET).view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty(M, N_W, dtype=torch.bfloat16, device=dev)
+        wsb = max([uw.uw_gemm_workspace(copies[0], M, p) for p in ("direct_palette", "exponent")] +
+                  [uw.uw_dense_gemm_workspace(M, N_W, K_W)])
+        ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+        row = {}
+        for name in ("direct_palette", "exponent", "dense"):
+            if name == "dense":
+                fns = [lambda w=w: uw.uw_dense_gemm(X, w, out=Y, ws=ws) for w in dense]
+            else:
+                fns = [lambda b=b, name=name: uw.uw_gemm(X, b, name, out=Y, ws=ws) for b in copies]
+            with torch.cuda.stream(cap):
+                for f in fns:
+                    f()
+            torch.cuda.synchronize()
+            gs = [capture(f) for f in fns]
+            for i in range(8):
+                gs[i % len(gs)].replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 40
+            a.record()
+            for i in range(reps):
+                gs[i % len(gs)].replay()
+            b.record()
+            torch.cuda.synchronize()
+            us = 1e3 * a.elapsed_time(b) / reps
+            tflops = 2.0 * M * n / (us / 1e6) / 1e12
+            row[name] = {"us": us, "tflops": tflops, "tensor_frac": tflops / tc_peak,
+                         "eff_weight_gbs": 2.0 * n / (us / 1e6) / 1e9}
+            del gs
+        out[str(M)] = row
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during the batch sweep")
+    return out
+
+
 def run_gpu(args):
     import numpy as np
     import torch
@@ -280,6 +338,7 @@ def run_gpu(args):
         per_op_ms.append(a.elapsed_time(b) / reps)
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
+    sweep = batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak) if not args.no_sweep else None
 
     # ---- end to end: host x (pinned) -> device, the step, Y -> host (pinned)
     xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -319,10 +378,11 @@ def run_gpu(args):
         "decode_full": stream_b + vstore + n + 2 * n,
         "decode_exponent": stream_b + vstore + n,
         "transcode": stream_b + n // 2,
-        "gemm_direct_palette": n + n // 2 + vstore + sec["vcol"][1] + xb + yb,
+        "gemm_direct_palette": n + n // 2 + vstore + xb + yb + (0 if uw_gemv_serves() else sec["vcol"][1]),
     }
     kernel_of = {"decode_full": "k_decode<full>", "decode_exponent": "k_decode<exponent>",
-                 "transcode": "k_decode<transcode>", "gemm_direct_palette": "k_gemm_recon<palette>"}
+                 "transcode": "k_decode<transcode>",
+                 "gemm_direct_palette": "k_gemv<palette, M=1>" if uw_gemv_serves() else "k_gemm_recon<palette>"}
     breakdown = {}
     for k, name in enumerate(OPS):
         d = {"us": 1e3 * per_op_ms[k], "eff_weight_gbs": 2.0 * n / (per_op_ms[k] / 1e3) / 1e9,
@@ -365,6 +425,7 @@ def run_gpu(args):
                      "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic},
         "breakdown": breakdown,
+        "batch_sweep": sweep,
         "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": xb, "d2h_bytes_per_step": 4 * yb},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -385,6 +446,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the larger-batch GEMM sweep")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

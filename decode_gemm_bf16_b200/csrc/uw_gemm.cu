@@ -702,6 +702,17 @@ uint64_t timeout_ns() {
 
 int gemm_default_grid() { return num_sms(); }
 
+// Batch 1 on a projection with fewer than half as many 128-row tiles as
+// GEMM CTAs (every tile would be cut several ways along k) runs the GEMV;
+// the choice depends only on the shape, never on the weight source, so the
+// pipelines and the dense baseline keep identical summation orders.
+bool gemv_serves(const GemmArgs& a) {
+    if (a.M != 1 || a.band_ready) return false;
+    const int64_t n_tiles = (a.N + kBlockN - 1) / kBlockN;
+    const int64_t P = a.grid > 0 ? a.grid : gemm_default_grid();
+    return 2 * n_tiles < P;
+}
+
 unsigned long long gemm_next_epoch() { return next_epoch(); }
 
 int gemm_status_take() { return unit_status_take(); }
@@ -719,7 +730,7 @@ size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     *st = UW_OK;
     if (a.M == 0) return cudaSuccess;
-    if (a.M <= kGemvMaxM && !a.band_ready) return launch_gemv(a, s, st);
+    if (gemv_serves(a)) return launch_gemv(a, s, st);
     GemmParams p{};
     p.M = a.M;
     p.N = a.N;

@@ -1,6 +1,7 @@
-// uw_gemv.cu -- Y[M,N] = X[M,K] . W[N,K]^T for batches of 1 to 4 rows on the
-// CUDA cores, with W plain BF16 or rebuilt in registers from its compressed
-// form.
+// uw_gemv.cu -- y[N] = W[N,K] . x[K] (batch 1) on the CUDA cores, with W
+// plain BF16 or rebuilt in registers from its compressed form.  The GEMM
+// entry points route batch 1 here when the projection has few 128-row tiles
+// (the tensor-core kernel would cut every tile several ways along k).
 //
 // "Cloudflare推出Unweight無損壓縮系統" (easyvibecoding.app),
 // §重建矩陣乘法核心運作 and §四種執行管道: at batch 1 the matmul is a
@@ -16,9 +17,9 @@
 //     one 64-weight group), so every plane is read in 512-byte (sign+
 //     mantissa, exponents) or 256-byte (indices) coalesced warp accesses,
 //     streaming (evict-first); BF16 weights take two 16-byte loads a lane;
-//   * a batch of one row issues four steps of loads before using them (two
-//     for larger batches), and 32 warps per SM keep well over the ~45 KB per
-//     SM in flight that HBM3e needs at this latency;
+//   * each warp issues four steps of loads before using them, and 32 warps
+//     per SM keep well over the ~45 KB per SM in flight that HBM3e needs at
+//     this latency;
 //   * the palette lookup is two byte permutes per four weights, verbatim
 //     64-weight groups (rare) read their raw exponents from the verbatim
 //     store; the merged BF16 pairs widen to fp32 with a shift or a mask;
@@ -225,8 +226,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) k_gemv(const GemvParams p)
 
 template <int SRC, bool XS>
 static const void* gemv_kernel_xs(int mb) {
-    return mb == 1 ? (const void*)k_gemv<SRC, 1, XS> : mb == 2 ? (const void*)k_gemv<SRC, 2, XS>
-                                                                : (const void*)k_gemv<SRC, 4, XS>;
+    (void)mb;
+    return (const void*)k_gemv<SRC, 1, XS>;
 }
 template <int SRC>
 static const void* gemv_kernel(int mb, bool xs) {

@@ -141,10 +141,12 @@ struct GemmArgs {
     int64_t band_tasks = 0, ntasks = 0;
 };
 size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid);
-// Tensor-core GEMM; batches of at most kGemvMaxM rows (without a decoder
-// running beside) go to the CUDA-core GEMV instead.
+// Tensor-core GEMM; the shapes gemv_serves() accepts (batch 1 on a
+// projection with few 128-row tiles, no decoder beside) go to the CUDA-core
+// GEMV instead.
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st);
-constexpr int kGemvMaxM = 4;
+bool gemv_serves(const GemmArgs& a);
+constexpr int kGemvMaxM = 1;   // batches the GEMV kernel supports
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, uw_status* st);
 int gemm_default_grid();
 unsigned long long gemm_next_epoch();

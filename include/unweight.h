@@ -109,9 +109,8 @@ typedef struct {
     int32_t pipeline;        /* uw_pipeline                                               */
     int32_t sm_dec;          /* >0: the Huffman decoder runs on sm_dec SMs beside the GEMM
                                 in one launch (§解壓與運算資源共享); 0: decode, then GEMM */
-    int32_t grid;            /* tensor-core GEMM CTAs; 0 = one per SM.  Batches of 1-4
-                                rows (with sm_dec = 0) run the CUDA-core GEMV, which
-                                ignores it                                                 */
+    int32_t grid;            /* tensor-core GEMM CTAs; 0 = one per SM.  It also decides
+                                whether batch 1 runs the CUDA-core GEMV (see uw_gemm)      */
     int32_t out_f32;         /* 0: Y is BF16 (round to nearest even); 1: Y is float32      */
     void* workspace;         /* device, 256-byte aligned, any contents; a call owns it
                                 until it completes (one workspace per stream)              */
@@ -208,11 +207,13 @@ uw_status uw_transcode_palette(const uw_blob* blob, uint8_t* idx_out, void* stre
 /* ---------------------------------------------------------------- GEMM
  * Y[M,N] = X[M,K] . W^T with W given compressed (§重建矩陣乘法核心運作).
  * X: device BF16 [M,K], 16-byte aligned; Y: device [M,N] BF16 or float32.
- * M = 0 is a no-op.  Accumulation is float32: on the tensor cores for M > 4
- * (and whenever sm_dec > 0), on the CUDA cores (a GEMV that rebuilds the
- * weights in registers) for M <= 4.  All pipelines and uw_dense_gemm take
- * the same summation order for a given M, N, K and grid, so their results
- * agree bit for bit. */
+ * M = 0 is a no-op.  Accumulation is float32 on the tensor cores, except
+ * for M = 1 on a projection with fewer than grid/2 tiles of 128 rows (grid:
+ * the GEMM CTA count, one per SM by default) and sm_dec = 0: that runs on
+ * the CUDA cores (a GEMV that rebuilds the weights in registers).  The
+ * choice depends on the shape only, so all pipelines and uw_dense_gemm take
+ * the same summation order for a given M, N, K and grid and agree bit for
+ * bit. */
 
 /* Workspace bytes for uw_gemm with these options and M. */
 uw_status uw_gemm_workspace(const uw_blob* blob, int64_t M, const uw_gemm_opts* opts, size_t* bytes);
@@ -220,8 +221,8 @@ uw_status uw_gemm_workspace(const uw_blob* blob, int64_t M, const uw_gemm_opts* 
 uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* blob, void* Y,
                   const uw_gemm_opts* opts, void* stream);
 
-/* The uncompressed baseline: the same GEMM (tensor cores, or the GEMV for
- * M <= 4) on a plain BF16 W. */
+/* The uncompressed baseline: the same GEMM (tensor cores, or the GEMV where
+ * uw_gemm would use it) on a plain BF16 W. */
 uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int grid, size_t* bytes);
 
 uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K,
