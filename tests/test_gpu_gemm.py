@@ -23,6 +23,8 @@ SHAPES = {
     # N x K: several 128-row tiles and 64-wide k steps, ragged N, verbatim rows
     "384x512": lambda: S.weight_with_verbatim_rows(384, 512, seed=31, frac_groups=0.01),
     "200x1408": lambda: S.weight_with_verbatim_rows(200, 1408, seed=32, frac_groups=0.01),
+    # K an odd multiple of 64: small batches fall back to 64-k stages
+    "136x576": lambda: S.weight_with_verbatim_rows(136, 576, seed=33, frac_groups=0.01),
 }
 MS = [1, 3, 16, 17, 64, 100, 256, 300]
 
@@ -138,14 +140,39 @@ def test_full_size_gate_sampled(M):
     assert uw.uw_last_device_status() == 0
 
 
-def test_full_size_down_sampled():
+@pytest.fixture(scope="module")
+def down_case():
     W = S.down_projection()
-    blob = uw.uw_compress(dev16(W))
+    return W, uw.uw_compress(dev16(W))
+
+
+def test_full_size_down_sampled(down_case):
+    W, blob = down_case
     X = S.activations(256, 14336, seed=4 + S.X_SEED_OFFSET)
     Xd = dev16(X)
     for pipe in ["exponent", "direct_palette"]:
         Y = _f32(uw.uw_gemm(Xd, blob, pipe))
         _sampled(X, W, Y, 128, seed=3, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_full_size_down_small_batch(down_case, M):
+    """Down projection (32 row tiles, K = 14336) at batch 1 (the CUDA-core
+    GEMV serves it) and 16 (tensor cores, 128-k stages, each tile cut ~4-5
+    ways): every pipeline and the dense baseline agree bit for bit and match
+    sampled oracle outputs."""
+    W, blob = down_case
+    X = S.activations(M, 14336, seed=40 + M)
+    Xd = dev16(X)
+    ref = None
+    for pipe in PIPES:
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
+        if ref is None:
+            ref = Y
+            _sampled(X, W, Y, 128, seed=M, bf16_out=True)
+        assert np.array_equal(Y, ref), pipe
+    assert np.array_equal(_f32(uw.uw_dense_gemm(Xd, dev16(W))), ref)
     assert uw.uw_last_device_status() == 0
 
 
