@@ -34,6 +34,7 @@ N_W, K_W, M_X = 14336, 4096, 1
 OPS = ["decode_full", "decode_exponent", "transcode", "gemm_full", "gemm_exponent", "gemm_transcode",
        "gemm_direct_palette"]
 WORKLOAD = "gate projection W[14336,4096] bf16 N(0,0.02)+0.1% t3 tail, x[1,4096]; decode x3 + 4 pipelines"
+OP_BURST = 8      # launches per graph when one op is timed alone
 
 
 def _peaks():
@@ -212,21 +213,21 @@ def batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak):
                 for f in fns:
                     f()
             torch.cuda.synchronize()
-            gs = [capture(f) for f in fns]
-            for i in range(8):
-                gs[i % len(gs)].replay()
+            g = capture(lambda: [fns[i % len(fns)]() for i in range(OP_BURST)])
+            for i in range(2):
+                g.replay()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 40
+            reps = 8
             a.record()
             for i in range(reps):
-                gs[i % len(gs)].replay()
+                g.replay()
             b.record()
             torch.cuda.synchronize()
-            us = 1e3 * a.elapsed_time(b) / reps
+            us = 1e3 * a.elapsed_time(b) / (reps * OP_BURST)
             tflops = 2.0 * M * n / (us / 1e6) / 1e12
             row[name] = {"us": us, "tflops": tflops, "tensor_frac": tflops / tc_peak,
                          "eff_weight_gbs": 2.0 * n / (us / 1e6) / 1e9}
-            del gs
+            del g
         out[str(M)] = row
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the batch sweep")
@@ -288,7 +289,9 @@ def run_gpu(args):
     torch.cuda.synchronize()
     step_graphs = [capture(lambda r=r: [op(k, copies[(r + k) % ncopy], xd) for k in range(nops)])
                    for r in range(ncopy)]
-    op_graphs = [[capture(lambda k=k, c=c: op(k, copies[c], xd)) for c in range(ncopy)] for k in range(nops)]
+    # per-op graphs: OP_BURST launches of one op over the rotated copies, so the
+    # per-launch time is not inflated by the gap between graph launches
+    op_graphs = [capture(lambda k=k: [op(k, copies[i % ncopy], xd) for i in range(OP_BURST)]) for k in range(nops)]
 
     # warm-up: W steps, and at least half a second of work so the clocks settle
     t_w = time.time()
@@ -324,18 +327,18 @@ def run_gpu(args):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
     # per-op device time: each op alone, rotated over the copies
-    reps = max(40, min(400, args.steps // 5))
+    reps = max(10, min(100, args.steps // 20))
     per_op_ms = []
     for k in range(nops):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for i in range(8):
-            op_graphs[k][i % ncopy].replay()
+        for i in range(2):
+            op_graphs[k].replay()
         a.record(stream)
         for i in range(reps):
-            op_graphs[k][i % ncopy].replay()
+            op_graphs[k].replay()
         b.record(stream)
         torch.cuda.synchronize()
-        per_op_ms.append(a.elapsed_time(b) / reps)
+        per_op_ms.append(a.elapsed_time(b) / (reps * OP_BURST))
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
     sweep = batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak) if not args.no_sweep else None
