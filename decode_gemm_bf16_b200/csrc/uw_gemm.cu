@@ -87,6 +87,7 @@ struct GemmParams {
     const unsigned long long* band_ready;
     int64_t band_tasks, ntasks;
     uint64_t timeout_ns;
+    int static_a;                  // weight planes are not written by any kernel that may still run
 };
 
 // Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
@@ -378,8 +379,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     tc_fence_after();
     const uint32_t tacc = *tmem_slot;
     // launched with programmatic stream serialization: the prologue above may
-    // overlap the previous kernel; global memory is touched only after it ends
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // overlap the previous kernel; global memory it may write is touched only
+    // after it ends (the producer warp waits inside its role, below)
+    if (warp != kProdWarp) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t smem_base = smem_u32(smem);
 
@@ -389,6 +391,28 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // elected lane issues the transfers.
         {
             const bool leader = elect_one();
+            // Static weight planes (direct palette from the committed blob):
+            // the first ring's worth of weight tiles is requested before the
+            // wait on the previous kernel, so it streams in during that
+            // kernel's tail; activations follow after the wait.
+            int npre = 0;
+            if (SRC == kSrcPalette && p.static_a && !p.band_ready) {
+                SegWalker wk0(blockIdx.x, p);
+                Segment sg0;
+                while (npre < S && wk0.next(sg0)) {
+                    const int n_tile = (int)(sg0.tile / p.m_tiles);
+                    for (int kt = sg0.kt0; kt < sg0.kt1 && npre < S; kt++, npre++) {
+                        if (!leader) continue;
+                        const uint32_t st = smem_base + npre * p.stage_bytes;
+                        const uint32_t fb = smem_u32(&full_bar[npre]);
+                        mbar_arrive_expect_tx(fb, p.tx_bytes);
+                        tma_load_2d(st + p.off_sm, &tm_a, kt * KB, n_tile * kBlockN, fb);
+                        tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
+                        tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
+                    }
+                }
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             SegWalker wk(blockIdx.x, p);
             Segment sg;
             int64_t q = 0;
@@ -408,6 +432,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 }
                 for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
                     const int s = rp.s;
+                    if (q < npre) {
+                        // weight tiles already requested: the activations only
+                        if (leader) {
+                            const uint32_t st = smem_base + s * p.stage_bytes;
+#pragma unroll
+                            for (int hb = 0; hb < kHalves; hb++)
+                                tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG,
+                                            smem_u32(&full_bar[s]));
+                        }
+                        continue;
+                    }
                     if (!mbar_wait(smem_u32(&empty_bar[s]), rp.ph ^ 1u, p.timeout_ns, abort_flag)) { ok = false; break; }
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
@@ -775,6 +810,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.band_tasks = a.band_tasks;
     p.ntasks = a.ntasks;
     p.timeout_ns = timeout_ns();
+    p.static_a = a.static_a;
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
     const int halves = KB / kBoxK;
@@ -955,6 +991,7 @@ extern "C" uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M
     a.K = b->geo.K;
     a.sm = b->sec(UW_SEC_SM);
     a.idx = b->sec(UW_SEC_IDX);
+    a.static_a = 1;
     a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
     a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
     a.vexp = b->sec(UW_SEC_VEXP);

@@ -727,7 +727,11 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
         case UW_PIPE_FULL: a.src = kSrcDense; a.W = (const uint16_t*)ws; break;
         case UW_PIPE_EXPONENT: a.src = kSrcExponent; a.ex = ws; break;
         case UW_PIPE_TRANSCODE: a.src = kSrcPalette; a.idx = ws; break;
-        default: a.src = kSrcPalette; a.idx = b->sec(UW_SEC_IDX); break;
+        default:   // the committed blob's index plane: no kernel writes it
+            a.src = kSrcPalette;
+            a.idx = b->sec(UW_SEC_IDX);
+            a.static_a = 1;
+            break;
     }
     if (o->pipeline == UW_PIPE_DIRECT_PALETTE) {
         cudaError_t e = launch_gemm(a, s, &st);

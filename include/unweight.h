@@ -215,7 +215,13 @@ uw_status uw_transcode_palette(const uw_blob* blob, uint8_t* idx_out, void* stre
  * the CUDA cores (a GEMV that rebuilds the weights in registers).  The
  * choice depends on the shape only, so all pipelines and uw_dense_gemm take
  * the same summation order for a given M, N, K and grid and agree bit for
- * bit. */
+ * bit.
+ * Kernels are launched with programmatic dependent launch.  The direct-palette
+ * pipeline requests its first weight tiles from the blob's device image
+ * before waiting for the preceding kernel on the stream to finish, so that
+ * image must not be written by device work that may still be running when
+ * the call is enqueued (the library never writes a committed blob; ordinary
+ * kernels and copies finish before a dependent kernel starts). */
 
 /* Workspace bytes for uw_gemm with these options and M. */
 uw_status uw_gemm_workspace(const uw_blob* blob, int64_t M, const uw_gemm_opts* opts, size_t* bytes);
