@@ -87,7 +87,8 @@ struct GemmParams {
     const unsigned long long* band_ready;
     int64_t band_tasks, ntasks;
     uint64_t timeout_ns;
-    int static_a;                  // weight planes are not written by any kernel that may still run
+    int static_sm;                 // sign+mantissa plane and verbatim flags come from the committed blob
+    int static_s2;                 // so does the second plane (the stored index plane)
 };
 
 // Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
@@ -391,12 +392,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // elected lane issues the transfers.
         {
             const bool leader = elect_one();
-            // Static weight planes (direct palette from the committed blob):
-            // the first ring's worth of weight tiles is requested before the
+            // Weight planes read from the committed blob (the sign+mantissa
+            // plane and verbatim flags of every rebuilding pipeline, the index
+            // plane of the direct-palette one) are not written by any kernel:
+            // the first ring's worth of those tiles is requested before the
             // wait on the previous kernel, so it streams in during that
-            // kernel's tail; activations follow after the wait.
+            // kernel's tail; activations and decoded planes follow the wait.
             int npre = 0;
-            if (SRC == kSrcPalette && p.static_a && !p.band_ready) {
+            if (kRecon && p.static_sm && !p.band_ready) {
                 SegWalker wk0(blockIdx.x, p);
                 Segment sg0;
                 while (npre < S && wk0.next(sg0)) {
@@ -407,8 +410,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                         const uint32_t fb = smem_u32(&full_bar[npre]);
                         mbar_arrive_expect_tx(fb, p.tx_bytes);
                         tma_load_2d(st + p.off_sm, &tm_a, kt * KB, n_tile * kBlockN, fb);
-                        tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
-                        tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
+                        if (SRC == kSrcPalette) {
+                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
+                            if (p.static_s2) tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
+                        }
                     }
                 }
             }
@@ -433,13 +438,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
                     const int s = rp.s;
                     if (q < npre) {
-                        // weight tiles already requested: the activations only
+                        // static tiles already requested: activations and the
+                        // decoded plane only
                         if (leader) {
                             const uint32_t st = smem_base + s * p.stage_bytes;
+                            const uint32_t fb = smem_u32(&full_bar[s]);
 #pragma unroll
                             for (int hb = 0; hb < kHalves; hb++)
-                                tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG,
-                                            smem_u32(&full_bar[s]));
+                                tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, fb);
+                            if (SRC == kSrcExponent)
+                                tma_load_2d(st + p.off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
+                            else if (!p.static_s2)
+                                tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
                         }
                         continue;
                     }
@@ -810,7 +820,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.band_tasks = a.band_tasks;
     p.ntasks = a.ntasks;
     p.timeout_ns = timeout_ns();
-    p.static_a = a.static_a;
+    p.static_sm = a.static_sm;
+    p.static_s2 = a.static_s2;
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
     const int halves = KB / kBoxK;
@@ -991,7 +1002,8 @@ extern "C" uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M
     a.K = b->geo.K;
     a.sm = b->sec(UW_SEC_SM);
     a.idx = b->sec(UW_SEC_IDX);
-    a.static_a = 1;
+    a.static_sm = 1;
+    a.static_s2 = 1;
     a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
     a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
     a.vexp = b->sec(UW_SEC_VEXP);

@@ -721,6 +721,7 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     a.vexp = b->sec(UW_SEC_VEXP);
     a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
     a.palette = b->palette;
+    a.static_sm = 1;   // the sign+mantissa plane and verbatim flags are the committed blob's
     const int mode = o->pipeline == UW_PIPE_FULL ? kDecodeFull : o->pipeline == UW_PIPE_EXPONENT ? kDecodeExponent
                                                                                                 : kDecodeTranscode;
     switch (o->pipeline) {
@@ -730,7 +731,7 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
         default:   // the committed blob's index plane: no kernel writes it
             a.src = kSrcPalette;
             a.idx = b->sec(UW_SEC_IDX);
-            a.static_a = 1;
+            a.static_s2 = 1;
             break;
     }
     if (o->pipeline == UW_PIPE_DIRECT_PALETTE) {

@@ -139,7 +139,8 @@ struct GemmArgs {
     unsigned long long epoch = 0;     // 0: a fresh call tag
     const unsigned long long* band_ready = nullptr;   // decoder-beside-GEMM readiness
     int64_t band_tasks = 0, ntasks = 0;
-    int static_a = 0;                 // palette source read from the committed blob (no kernel writes it)
+    int static_sm = 0;                // sm plane and verbatim flags read from the committed blob (no kernel writes it)
+    int static_s2 = 0;                // second plane too (the stored index plane)
 };
 size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid);
 // Tensor-core GEMM; the shapes gemv_serves() accepts (batch 1 on a
