@@ -106,14 +106,28 @@ class Clocks:
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(sel)}
 
 
-def _dist():
+def _dist(backend: str = "nccl"):
+    """One process per GPU under torchrun: (dist module or None, rank, world,
+    local rank).  The path does not shard, so ranks are independent replicas
+    that meet only for the barriers around the timed region and the
+    max-over-ranks reduction of its device time."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
         import torch.distributed as dist
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return dist, int(os.environ["RANK"]), ws, int(os.environ.get("LOCAL_RANK", "0"))
     return None, 0, 1, 0
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's value (every rank gets it)."""
+    if not dist:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -153,7 +167,9 @@ def cpu_baseline(rows: int = 256):
 
 
 def run_reference(args):
-    dist, rank, world, _ = _dist()
+    # the oracle runs on rank 0 only; other ranks exit at once (no process
+    # group: they exchange nothing)
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     rows = 256
@@ -323,9 +339,7 @@ def run_gpu(args):
         dist.barrier()
     ms = t0.elapsed_time(t1)
     if dist:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, dev)
     # per-op device time: each op alone, rotated over the copies
     reps = max(10, min(100, args.steps // 20))
     per_op_ms = []
@@ -364,9 +378,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if dist:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
 
     # ---- numbers
     eff_bytes_step = nops * 2.0 * n
