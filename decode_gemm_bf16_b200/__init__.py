@@ -267,7 +267,8 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 def uw_gemm(X: torch.Tensor, blob: Blob, pipeline="direct_palette", out: Optional[torch.Tensor] = None,
             out_f32: bool = False, ws: Optional[torch.Tensor] = None, sm_dec: int = 0, grid: int = 0,
             stream=None) -> torch.Tensor:
-    """Y[M, N] = X[M, K] . W^T with W compressed in `blob`."""
+    """Y[M, N] = X[M, K] . W^T with W compressed in `blob` (tensor cores; batch 1
+    on a projection with few 128-row tiles runs the library's CUDA-core GEMV)."""
     X = _bits16(X)
     M = X.shape[0]
     if out is None:
@@ -302,7 +303,8 @@ def uw_dense_gemm_workspace(M: int, N: int, K: int, grid: int = 0) -> int:
 
 def uw_dense_gemm(X: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = None, out_f32: bool = False,
                   ws: Optional[torch.Tensor] = None, grid: int = 0, stream=None) -> torch.Tensor:
-    """The uncompressed baseline: same tensor-core GEMM on plain BF16 W[N, K]."""
+    """The uncompressed baseline: the same GEMM (tensor cores, or the GEMV where
+    uw_gemm would use it) on plain BF16 W[N, K]."""
     X = _bits16(X)
     W = _bits16(W)
     M, K = X.shape
