@@ -415,14 +415,15 @@ def run_gpu(args):
     dom_ms = per_op_ms[OPS.index(dom)]
     achieved = alg[dom] / (dom_ms / 1e3) / 1e9
     # DRAM bytes per launch from the committed ncu capture, only while the
-    # kernels are the ones that capture measured (same library sources)
+    # kernels are the ones that capture measured (same code hash: library
+    # sources without comments, plus build flags)
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         try:
             from decode_gemm_bf16_b200 import build as uwbuild
             tj = json.load(open(tp))
-            if tj.get("source_hash") == uwbuild.source_hash():
+            if tj.get("code_hash") == uwbuild.code_hash():
                 traffic = tj["bytes_per_launch"].get(kernel_of[dom])
         except Exception:
             traffic = None

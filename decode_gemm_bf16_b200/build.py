@@ -12,6 +12,8 @@ LIB = os.path.join(HERE, "libunweight.so")
 SOURCES = ["uw_host.cpp", "uw_compress.cu", "uw_decode.cu", "uw_gemm.cu", "uw_gemv.cu"]
 HEADERS = ["uw_internal.h", "uw_device.cuh", os.path.join("..", "..", "include", "unweight.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+BUILD_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-Xcompiler",
+               "-fvisibility=default", "--expt-relaxed-constexpr"]
 
 
 def _nvcc():
@@ -30,6 +32,41 @@ def source_hash() -> str:
     return h.hexdigest()
 
 
+def _strip_comments(text: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed
+    (string and character literals kept verbatim)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def code_hash() -> str:
+    """Hash of what the compiler sees (sources without comments, plus the
+    build flags): measurements keyed to it stay valid across comment edits."""
+    h = hashlib.sha256(" ".join(ARCH + BUILD_FLAGS).encode())
+    for f in SOURCES + HEADERS:
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            h.update(_strip_comments(fh.read()).encode())
+    return h.hexdigest()
+
+
 def stale() -> bool:
     """True when the library is missing or was built from other sources."""
     if not os.path.exists(LIB) or not os.path.exists(STAMP):
@@ -42,9 +79,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=default", "--expt-relaxed-constexpr",
-           *extra, *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp]
+    cmd = [_nvcc(), *ARCH, *BUILD_FLAGS, *extra, *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)

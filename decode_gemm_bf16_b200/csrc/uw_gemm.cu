@@ -17,20 +17,28 @@
 //     tensor memory (TMEM) -- no register-file accumulators, so shared memory
 //     holds only the stage ring;
 //   * warp roles: warps 0-3 epilogue (TMEM lanes 32w..32w+31), warp 4 TMA
-//     producer, warp 5 allocates TMEM and issues tcgen05.mma (one thread),
-//     warps 6-13 rebuild BF16 rows;
+//     producer, warp 5 allocates TMEM and issues tcgen05.mma, warps 6-21
+//     rebuild BF16 rows (two groups of eight, alternate stages); the producer
+//     and MMA warps walk their loops as whole warps and one elected lane
+//     issues;
+//   * a stage covers 128 k for batch tiles up to 64 rows (64 k above), so the
+//     per-stage barrier, TMA and commit costs are paid once per 128 k;
 //   * the rebuilt tile never touches shared memory: each rebuild thread owns
-//     one weight row (one TMEM lane) and half of the 64-wide k step, reads its
-//     sign+mantissa and index bytes from TMA tiles staged with a 64/32-byte
-//     swizzle (conflict-free row-per-lane reads), and writes 16 columns of BF16
-//     pairs into tensor memory with tcgen05.st; the MMA reads A from TMEM.
-//     Shared memory then carries 3 bytes per weight (TMA write + one read)
-//     instead of 7, and holds no A tiles;
-//   * stream-K: the (tile, 64-wide k step) iterations are split evenly over one
-//     CTA per SM; tiles cut between CTAs are finished by the last CTA to
-//     arrive, per output row, summing fp32 partials in CTA order
-//     (deterministic).  This covers batch 1-64 (HBM bound, K split) and the
-//     long-K down projection with the same kernel;
+//     one weight row (one TMEM lane) and one or two 32-k pieces of the stage,
+//     reads its sign+mantissa and index (or exponent) bytes from TMA tiles
+//     staged with a swizzle matching their row length (conflict-free
+//     row-per-lane reads), and writes 16 columns of BF16 pairs per piece into
+//     tensor memory with tcgen05.st; the MMA reads A from TMEM.  Shared memory
+//     then carries 3 bytes per weight (TMA write + one read) instead of 7,
+//     and holds no A tiles;
+//   * stream-K: the (tile, stage) iterations are split evenly over one CTA
+//     per SM (or one CTA per tile when that is cheaper, see launch_gemm); a
+//     tile cut between CTAs is finished by the CTA holding its first k steps,
+//     which reaches it last and adds the others' fp32 partial rows in k order
+//     (deterministic).  This covers batch 1-1024 and the long-K down
+//     projection with the same kernel;
+//   * weight planes that come from the committed blob are requested before
+//     the wait on the previous kernel (programmatic dependent launch);
 //   * every wait is bounded (globaltimer deadline); on expiry the CTA raises
 //     UW_ERR_TIMEOUT, drains its own TMA and MMA work, frees TMEM and exits.
 #include <atomic>

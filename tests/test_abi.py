@@ -133,3 +133,15 @@ def test_corrupt_headers_rejected(L, what):
 def test_header_layout_size():
     # the size the library expects: 4+4+8+8+4+4+8+8+8+16+16+128+2048+80
     assert len(serialize_oracle(O.compress(np.zeros((1, 64), np.uint16) | 0x3F80), forms=3)) > 2344
+
+
+def test_code_hash_ignores_comments_only():
+    """Measurements (profiles/traffic.json) are keyed to the code hash: it must
+    ignore comments and whitespace but not code, strings or build flags."""
+    from decode_gemm_bf16_b200 import build as B
+    strip = B._strip_comments
+    assert strip("a /* x */ b // y\n c") == strip("a b\n\n   c")
+    assert strip('s = "//not a comment"; // gone') == 's = "//not a comment";'
+    assert strip("x = '/'; /* multi\nline */ y") == "x = '/'; y"
+    assert strip("a + b") != strip("a - b")
+    assert len(B.code_hash()) == 64
