@@ -195,6 +195,56 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def run_stack(args):
+    """The 32-layer stack of Llama-3.1-8B-shaped MLP weights (synthetic, a
+    per-layer seed and std): every gate, up and down matrix compressed and
+    kept resident, the total footprint per form against BF16, and the
+    autotuner's plan (pipeline and decoder SM split per projection and batch
+    size, measured on layer 0) with the measured time of one layer's MLP
+    matmuls.  Prints one JSON line; not part of the timed benchmark."""
+    import numpy as np
+    import torch
+    import decode_gemm_bf16_b200 as uw
+    import synthetic as S
+
+    dev = torch.device("cuda", 0)
+    Ms = [1, 8, 64, 256, 1024]
+    t_start = time.time()
+    blobs, bf16_bytes, huff, pal, devb = [], 0, 0, 0, 0
+    for layer in range(args.layers):
+        for W in S.stack_layer(layer):
+            Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+            b = uw.uw_compress(Wd)
+            del Wd
+            info = b.info
+            bf16_bytes += 2 * W.size
+            huff += info["bytes_huffman_form"]
+            pal += info["bytes_palette_form"]
+            devb += info["device_bytes"]
+            blobs.append(b)
+    torch.cuda.synchronize()
+    t_compress = time.time() - t_start
+    proj = blobs[:3]
+    Xs = [torch.from_numpy(S.activations(max(Ms), b.info["K"], seed=7 + i).view(np.int16)).to(dev).view(torch.bfloat16)
+          for i, b in enumerate(proj)]
+    Ys = [torch.empty(max(Ms), b.info["N"], dtype=torch.bfloat16, device=dev) for b in proj]
+    need = max(uw.uw_gemm_workspace(b, max(Ms), p, sm_dec=sd) for b in proj for p in uw.PIPELINES for sd in (0, 296))
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    plan = uw.uw_autotune(proj, Ms, Xs, Ys, ws, reps=5)
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during the stack run")
+    layer_us = {str(M): sum(e["us"] for e in plan if e["M"] == M) for M in Ms}
+    flops = {str(M): 2.0 * M * sum(b.info["N"] * b.info["K"] for b in proj) for M in Ms}
+    line = {"stack": {"layers": args.layers, "matrices": len(blobs), "weights": bf16_bytes // 2,
+                      "bf16_bytes": bf16_bytes, "huffman_form_bytes": huff, "palette_form_bytes": pal,
+                      "device_image_bytes": devb, "ratio_huffman_form": huff / bf16_bytes,
+                      "ratio_palette_form": pal / bf16_bytes, "compress_s_incl_host_generation": t_compress},
+            "plan_layer0": plan,
+            "layer_mlp_us": layer_us,
+            "layer_mlp_tflops": {M: flops[M] / (layer_us[M] * 1e-6) / 1e12 for M in layer_us}}
+    print(json.dumps(line), flush=True)
+
+
 def uw_gemv_serves():
     """Whether batch 1 on this projection runs the CUDA-core GEMV (the
     library's rule: fewer than half as many 128-row tiles as GEMM CTAs)."""
@@ -463,9 +513,14 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-sweep", action="store_true", help="skip the larger-batch GEMM sweep")
+    ap.add_argument("--stack", action="store_true",
+                    help="compress the synthetic 32-layer MLP stack, report footprint and the autotuned plan")
+    ap.add_argument("--layers", type=int, default=32, help="layers for --stack")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.stack:
+        run_stack(args)
     else:
         run_gpu(args)
 
