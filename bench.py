@@ -52,7 +52,10 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        # raw samples: $UW_CLOCKS_DIR if set, else the system temp directory
+        import tempfile
+        d = os.environ.get("UW_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"uw_bench_clocks_gpu{index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
