@@ -468,16 +468,17 @@ def run_gpu(args):
     dom_ms = per_op_ms[OPS.index(dom)]
     achieved = alg[dom] / (dom_ms / 1e3) / 1e9
     # DRAM bytes per launch from the committed ncu capture, only while the
-    # kernels are the ones that capture measured (same code hash: library
-    # sources without comments, plus build flags)
+    # kernel is the one that capture measured (same code hash of its
+    # translation unit: sources without comments, plus build flags)
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         try:
             from decode_gemm_bf16_b200 import build as uwbuild
             tj = json.load(open(tp))
-            if tj.get("code_hash") == uwbuild.code_hash():
-                traffic = tj["bytes_per_launch"].get(kernel_of[dom])
+            ent = tj["bytes_per_launch"].get(kernel_of[dom])
+            if ent and ent.get("code_hash") == uwbuild.kernel_code_hash(kernel_of[dom]):
+                traffic = ent["bytes"]
         except Exception:
             traffic = None
     launches_per_step = 3 + 2 + 2 + 2 + 1

@@ -57,14 +57,29 @@ def _strip_comments(text: str) -> str:
     return " ".join("".join(out).split())
 
 
-def code_hash() -> str:
+def code_hash(unit: str | None = None) -> str:
     """Hash of what the compiler sees (sources without comments, plus the
-    build flags): measurements keyed to it stay valid across comment edits."""
+    build flags): measurements keyed to it stay valid across comment edits.
+    With `unit` (a source file name), only that translation unit and the
+    headers count, so a measurement of its kernels survives changes to the
+    other units."""
     h = hashlib.sha256(" ".join(ARCH + BUILD_FLAGS).encode())
-    for f in SOURCES + HEADERS:
+    for f in ([unit] if unit else SOURCES) + HEADERS:
         with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
             h.update(_strip_comments(fh.read()).encode())
     return h.hexdigest()
+
+
+# translation unit of each measured kernel family
+KERNEL_UNITS = {"k_decode": "uw_decode.cu", "k_gemm": "uw_gemm.cu", "k_gemv": "uw_gemv.cu"}
+
+
+def kernel_code_hash(kernel: str) -> str:
+    """code_hash of the unit that defines `kernel` (a profile short name)."""
+    for prefix, unit in KERNEL_UNITS.items():
+        if kernel.startswith(prefix):
+            return code_hash(unit)
+    return code_hash()
 
 
 def stale() -> bool:

@@ -145,3 +145,5 @@ def test_code_hash_ignores_comments_only():
     assert strip("x = '/'; /* multi\nline */ y") == "x = '/'; y"
     assert strip("a + b") != strip("a - b")
     assert len(B.code_hash()) == 64
+    assert B.kernel_code_hash("k_decode<full>") == B.code_hash("uw_decode.cu")
+    assert B.kernel_code_hash("k_gemm_recon<palette>") != B.kernel_code_hash("k_decode<full>")
