@@ -800,11 +800,13 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
     const int64_t total = tiles * p.kt_count;
     int P = a.grid > 0 ? a.grid : gemm_default_grid();
-    // Default grid: with batch tiles of 64+ rows and between half and all of
-    // a CTA per SM's worth of output tiles, one CTA per tile (no split, no
-    // fix-up) beats cutting tiles along k: the fix-up moves 32-128 KB of
-    // fp32 partials per cut tile and stalls the MMA while they are written.
-    if (a.grid == 0 && p.MG >= 64 && tiles <= P && 2 * tiles >= P) P = (int)tiles;
+    // Default grid: with batch tiles of 64+ rows and no more output tiles
+    // than SMs, every tile is cut into the same whole number of k ranges,
+    // one CTA each (one CTA per tile when the tiles number half the SMs or
+    // more): each CTA then holds a single segment, instead of a tail and a
+    // head whose fix-ups move 32-128 KB of fp32 partials per cut and stall
+    // the MMA while they are written.
+    if (a.grid == 0 && p.MG >= 64 && tiles <= P) P = (int)(tiles * (P / tiles));
     if (P > total) P = (int)total;
     if (total * (int64_t)P >= (int64_t(1) << 32)) { *st = UW_ERR_SHAPE; return cudaSuccess; }
     p.total_iters = (uint32_t)total;

@@ -109,10 +109,11 @@ typedef struct {
     int32_t pipeline;        /* uw_pipeline                                               */
     int32_t sm_dec;          /* >0: the Huffman decoder runs on sm_dec SMs beside the GEMM
                                 in one launch (§解壓與運算資源共享); 0: decode, then GEMM */
-    int32_t grid;            /* tensor-core GEMM CTAs; 0 = one per SM (or one per output
-                                tile, when batch tiles have 64+ rows and the tiles number
-                                between half and all of the SMs).  It also decides whether
-                                batch 1 runs the CUDA-core GEMV (see uw_gemm)              */
+    int32_t grid;            /* tensor-core GEMM CTAs; 0 = one per SM, or, when batch
+                                tiles have 64+ rows and there are no more output tiles than
+                                SMs, the largest whole multiple of the tile count that
+                                fits.  It also decides whether batch 1 runs the CUDA-core
+                                GEMV (see uw_gemm)                                         */
     int32_t out_f32;         /* 0: Y is BF16 (round to nearest even); 1: Y is float32      */
     void* workspace;         /* device, 256-byte aligned, any contents; a call owns it
                                 until it completes (one workspace per stream)              */
