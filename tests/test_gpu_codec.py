@@ -42,6 +42,7 @@ MATRICES = {
     "one_exponent_3x128": lambda: (np.full((3, 128), 127, np.uint16) << 7)
     | (np.arange(384, dtype=np.uint16).reshape(3, 128) % 128),
     "tiny_1x64": lambda: (np.array([120] * 32 + [121] * 16 + [122] * 8 + [123] * 8, np.uint16) << 7).reshape(1, 64),
+    "nibble_order_1x64": lambda: (np.array([120 + (k % 4) for k in range(64)], np.uint16) << 7).reshape(1, 64),
     "ragged_37x320": lambda: S.gaussian_weight(37, 320, seed=21),
     "ragged_300x1408": lambda: S.weight_with_verbatim_rows(300, 1408, seed=22, frac_groups=0.02),
     "no_verbatim_16x4096": lambda: S.gaussian_weight(16, 4096, seed=23, std=0.5),
@@ -98,6 +99,19 @@ def test_decoders_match_oracle(name):
     assert np.array_equal(host8(E), e_oracle)
     assert np.array_equal(host8(idx), O.transcode(ob))
     assert np.array_equal(host8(idx), ob["idx"])
+    assert uw.uw_last_device_status() == 0
+
+
+def test_index_plane_nibble_order_golden():
+    """The library's index plane and transcoder against the hand-derived
+    bytes of tests/golden/nibble_order_1x64.txt (0x10, 0x32 repeating:
+    element 2j in the low nibble), not only against the oracle."""
+    W = MATRICES["nibble_order_1x64"]()
+    blob = uw.uw_compress(dev16(W))
+    assert section_view(blob, "idx", np.uint8).tolist() == [0x10, 0x32] * 16
+    assert host8(uw.uw_transcode_palette(blob)).tolist() == [0x10, 0x32] * 16
+    assert [format(int(x), "08X") for x in section_view(blob, "stream", np.uint32)] == \
+        ["1B1B1B1B"] * 4 + ["00000000"] * 2
     assert uw.uw_last_device_status() == 0
 
 

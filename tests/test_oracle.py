@@ -225,6 +225,79 @@ def test_length_limit_binds_on_fibonacci():
     assert _cost(freq, lim) > _cost(freq, free)
 
 
+def _package_merge_py(freq, lmax, leaf_first):
+    """Independent package-merge in Python with a switchable tie rule: on
+    equal weight a leaf goes before a package (leaf_first) or after it."""
+    used = sorted([s for s in range(len(freq)) if freq[s] > 0], key=lambda s: (freq[s], s))
+    leaves = [(int(freq[s]), {s: 1}) for s in used]
+    lst = list(leaves)
+    for _ in range(2, lmax + 1):
+        pk = []
+        for i in range(len(lst) // 2):
+            (wa, ca), (wb, cb) = lst[2 * i], lst[2 * i + 1]
+            c = dict(ca)
+            for k, v in cb.items():
+                c[k] = c.get(k, 0) + v
+            pk.append((wa + wb, c))
+        out, i, j = [], 0, 0
+        while i < len(leaves) or j < len(pk):
+            if i >= len(leaves):
+                take_leaf = False
+            elif j >= len(pk):
+                take_leaf = True
+            else:
+                take_leaf = leaves[i][0] <= pk[j][0] if leaf_first else leaves[i][0] < pk[j][0]
+            if take_leaf:
+                out.append(leaves[i])
+                i += 1
+            else:
+                out.append(pk[j])
+                j += 1
+        lst = out
+    lengths = [0] * len(freq)
+    for _, c in lst[:2 * (len(used) - 1)]:
+        for k, v in c.items():
+            lengths[k] += v
+    return lengths
+
+
+def test_package_merge_tie_rule_hand_derived():
+    """tests/golden/package_merge_tie.txt: a leaf and a package of equal
+    weight meet; leaf-first gives 2,2,2,2 and package-first 3,3,2,1 at the
+    same cost, so this pins the tie rule (cost-only checks cannot)."""
+    rows = _read_golden("package_merge_tie.txt")
+    lmax = int([r for r in rows if r[0] == "lmax"][0][1])
+    cost = int([r for r in rows if r[0] == "cost"][0][1])
+    syms = [r for r in rows if r[0] not in ("lmax", "cost")]
+    freq = np.zeros(16, np.uint64)
+    leaf_first = np.zeros(16, np.uint8)
+    pkg_first = np.zeros(16, np.uint8)
+    for s, f, a, b in syms:
+        freq[int(s)], leaf_first[int(s)], pkg_first[int(s)] = int(f), int(a), int(b)
+    ln = O.code_lengths(freq, lmax)
+    assert ln.tolist() == leaf_first.tolist()
+    assert ln.tolist() != pkg_first.tolist()
+    assert _cost(freq, leaf_first) == _cost(freq, pkg_first) == cost
+    assert _kraft(pkg_first) == 1 and _kraft(leaf_first) == 1
+    # the independent implementation reproduces both hand-derived columns
+    assert _package_merge_py(freq.tolist(), lmax, True) == leaf_first.tolist()
+    assert _package_merge_py(freq.tolist(), lmax, False) == pkg_first.tolist()
+
+
+def test_package_merge_tie_rule_fibonacci():
+    """Fibonacci frequencies at the 12-bit limit: the two tie rules give
+    different optimal length vectors; the oracle gives the leaf-first one."""
+    fib = [1, 1]
+    while len(fib) < 16:
+        fib.append(fib[-1] + fib[-2])
+    leaf_first = [12, 12, 11, 10, 9, 8, 7, 6, 5, 4, 4, 4, 3, 3, 2, 2]
+    pkg_first = [12, 12, 12, 12, 11, 11, 10, 10, 8, 7, 6, 5, 4, 3, 2, 1]
+    assert _package_merge_py(fib, 12, True) == leaf_first
+    assert _package_merge_py(fib, 12, False) == pkg_first
+    assert _cost(fib, leaf_first) == _cost(fib, pkg_first)
+    assert O.code_lengths(np.array(fib, np.uint64), 12).tolist() == leaf_first
+
+
 def test_degenerate_alphabets():
     f = np.zeros(16, np.uint64)
     f[9] = 1000
@@ -264,6 +337,28 @@ def test_tiny_hand_derived_stream():
     assert b["idx"].tolist() == expect_idx
     assert b["chunk_off"].tolist() == [0] and b["seg_rel"].tolist() == [0]
     assert b["V"] == 0
+    assert np.array_equal(O.decode_full(b), W)
+
+
+def test_nibble_order_hand_derived():
+    """tests/golden/nibble_order_1x64.txt: symbols 0,1,2,3 repeating give
+    index bytes 0x10, 0x32 (element 2j in the low nibble); the swapped order
+    would give 0x01, 0x23."""
+    rows = {r[0]: r[1:] for r in _read_golden("nibble_order_1x64.txt")}
+    ex = [120 + (k % 4) for k in range(64)]
+    W = (np.array(ex, np.uint16) << 7).reshape(1, 64)
+    b = O.compress(W)
+    assert b["palette"].tolist() == [int(x) for x in rows["palette"]]
+    assert b["code_len"].tolist() == [int(x) for x in rows["code_len"]]
+    assert b["total_bits"] == int(rows["total_bits"][0])
+    assert [format(int(x), "08X") for x in b["stream"]] == rows["stream"]
+    expect_idx = []
+    for tok in rows["idx"]:
+        byte, rep = tok.split("x")
+        expect_idx += [int(byte, 16)] * int(rep)
+    assert b["idx"].tolist() == expect_idx
+    assert b["idx"][:2].tolist() == [0x10, 0x32]
+    assert np.array_equal(O.transcode(b), b["idx"])
     assert np.array_equal(O.decode_full(b), W)
 
 
