@@ -1,20 +1,28 @@
-"""Benchmark of the fused decode-GEMM path on one Llama-3.1-8B-shaped gate
-projection W[14336, 4096] (BF16, N(0, 0.02) with a 0.1% t_3 tail) at batch 1.
+"""Benchmark of the fused decode-GEMM path on the 32-layer stack of
+Llama-3.1-8B-shaped MLP weights (synthetic: gate/up W[14336,4096], down
+W[4096,14336] per layer, BF16 N(0, sigma_l) with a 0.1% t_3 tail, sigma_l ~
+U(0.015, 0.03)), every matrix compressed and resident on the GPU.
 
-One step = the whole per-call hot path over one batch:
-  uw_decode_full, uw_decode_exponent, uw_transcode_palette, and
-  uw_gemm through the four pipelines (full, exponent, transcode, direct
-  palette) with x[1, 4096].
-value = effective BF16 weight bytes delivered per second over the step
-(7 x 2*N*K bytes per step / step time), whole job (all ranks).
-The line also carries a batch sweep outside the timed step: the tensor-core
-GEMM (direct palette, exponent pipeline, dense BF16) at M = 16 ... 1024 on
-the same projection, each timed alone over rotated copies.
+One step = one pass over all 96 matrices at each batch size M in
+{1, 8, 64, 256, 1024}: Y = X . W^T through uw_gemm with UW_PIPE_AUTO, i.e.
+the pipeline, matmul variant and decoder split the autotuner (§自動調優機制)
+chose for that projection and batch on this GPU.  The activations are fixed
+synthetic X[M, 4096] (gate, up) and X[M, 14336] (down).
+value = effective BF16 weight bytes per second over the step (5 x 96
+matrices x 2*N*K bytes per step / step time), whole job (all ranks).
 
-Inputs larger than L2: four compressed copies of W (~110 MB each) are
-rotated so that an op never finds its inputs left in L2 by the previous use.
+Inputs are larger than L2: consecutive calls use different matrices, so no
+weight is read from L2 left by the previous use.
+
+The line also carries, outside the timed step: per (projection, M) the time
+of one call (the plan's choice, rotated over the layers) with its compressed
+GB/s, TFLOP/s, roofline fraction and slowdown against the library's own
+dense BF16 GEMM; the compressed footprint of the stack per form; the
+decoders and the four pipelines at batch 1 on the gate projection; and the
+decoder/matmul SM split swept on the down projection at M = 256 and 1024.
+
 --impl reference times the CPU oracle (plain C) on a bounded row sample of the
-same workload and prints the same metric.
+same step and prints the same metric.
 """
 from __future__ import annotations
 
@@ -30,11 +38,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fused decode-GEMM eff. weight GB/s & TFLOP/s, % roofline, batch 1–1024"
-N_W, K_W, M_X = 14336, 4096, 1
-OPS = ["decode_full", "decode_exponent", "transcode", "gemm_full", "gemm_exponent", "gemm_transcode",
-       "gemm_direct_palette"]
-WORKLOAD = "gate projection W[14336,4096] bf16 N(0,0.02)+0.1% t3 tail, x[1,4096]; decode x3 + 4 pipelines"
+MS = [1, 8, 64, 256, 1024]
+PROJ = ["gate", "up", "down"]
+SHAPES = {"gate": (14336, 4096), "up": (14336, 4096), "down": (4096, 14336)}
+WORKLOAD = ("32-layer Llama-3.1-8B-shaped MLP stack (gate/up W[14336,4096], down W[4096,14336]; bf16 "
+            "N(0,s_l)+0.1% t3 tail, s_l~U(0.015,0.03)); one step = all 96 matrices at each batch "
+            "M in {1,8,64,256,1024}, autotuned plan (UW_PIPE_AUTO)")
 OP_BURST = 8      # launches per graph when one op is timed alone
+ORACLE_ROWS_CPU = 256      # rows per projection in the CPU baseline sample
+ORACLE_ROWS_REF = 16       # rows per projection in one step of --impl reference
 
 
 def _peaks():
@@ -42,8 +54,9 @@ def _peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d.get("hbm_gbs", 6650.0)), float(d.get("bf16_tflops", 1590.0)), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (float(d.get("hbm_gbs", 6650.0)), float(d.get("bf16_tflops", 1590.0)),
+                float(d.get("bf16_tflops_sustained", 1400.0)), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 class Clocks:
@@ -66,7 +79,7 @@ class Clocks:
                  "--query-gpu=timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         return self
@@ -106,7 +119,13 @@ class Clocks:
         mx = max(float(r[2]) for r in sel)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in sel for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(sel)}
+        try:
+            pw = sorted(float(r[3]) for r in sel)
+            power = pw[len(pw) // 2]
+        except Exception:
+            power = None
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(sel),
+                "power_w_median": power}
 
 
 def _dist(backend: str = "nccl"):
@@ -139,34 +158,73 @@ def max_over_ranks(x: float, dist, device) -> float:
 _sample_cache = {}
 
 
-def oracle_step_sample(rows: int = 256):
-    """Runs the oracle's version of one step on `rows` rows of the workload:
-    Huffman decode -> full / exponent / transcode, then the reference product
-    for each of the four pipelines.  Returns (seconds, weights processed)."""
-    import synthetic as S
-    from oracle import oracle as O
+def _oracle_sample(rows: int):
+    """`rows` rows of each projection of layer 0's shape and distribution
+    (host recipe), compressed by the oracle; activations per projection and M."""
     if rows not in _sample_cache:
-        _sample_cache[rows] = S.gate_projection()[:rows].copy()
-    W = _sample_cache[rows]
-    x = S.activations(M_X, K_W, seed=1 + S.X_SEED_OFFSET)
-    b = O.compress(W)
+        import synthetic as S
+        from oracle import oracle as O
+        sd = float(S.layer_stds()[0])
+        sample = []
+        for j, name in enumerate(PROJ):
+            K = SHAPES[name][1]
+            Wr = S.weight_with_tail(rows, K, seed=1000 + j, std=sd)
+            X = {M: S.activations(M, K, seed=7 + j + M) for M in MS}
+            sample.append((name, O.compress(Wr), X))
+        _sample_cache[rows] = sample
+    return _sample_cache[rows]
+
+
+def oracle_step_sample(rows: int, threads: int):
+    """The oracle's version of one step on `rows` rows of every projection of
+    layer 0, at each batch size: rebuild the rows from their compressed form
+    (direct palette: palette lookup, verbatim groups, merge) and form
+    X . W^T, in `threads` threads over row blocks.  Returns (seconds,
+    weights processed, flops)."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as O
+    sample = _oracle_sample(rows)
+    blocks = []
+    for name, b, X in sample:
+        for M in MS:
+            blocks.append((b, X[M]))
+    nw = sum(b["N"] * b["K"] for _, b, _ in sample) * len(MS)
+    flops = sum(2.0 * M * b["N"] * b["K"] for _, b, _ in sample for M in MS)
+
+    def one(item):
+        b, x = item
+        W = O.decode_full(b)
+        O.gemm(x, W, "f32")
+
     t0 = time.perf_counter()
-    Wd = O.decode_full(b)                 # decode_full
-    O.decode_exponent(b)                  # decode_exponent
-    O.transcode(b)                        # transcode
-    for _ in range(4):                    # four pipelines: decode form + product
-        O.decode_exponent(b)
-        O.gemm(x, Wd, "f32")
+    if threads <= 1:
+        for it in blocks:
+            one(it)
+    else:
+        # split every block's rows so all threads have work
+        parts = []
+        import numpy as np
+        for b, x in blocks:
+            W = O.decode_full(b)
+            step = max(1, -(-W.shape[0] // threads))
+            for r0 in range(0, W.shape[0], step):
+                parts.append((x, np.ascontiguousarray(W[r0:r0 + step])))
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda p: O.gemm(p[0], p[1], "f32"), parts))
     dt = time.perf_counter() - t0
-    return dt, W.size
+    return dt, nw, flops
 
 
-def cpu_baseline(rows: int = 256):
-    dt, nw = oracle_step_sample(rows)
-    eff = len(OPS) * 2.0 * nw / dt / 1e9
-    return {"value": eff, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} of 14336 rows ({nw} weights), one step: decode x3 + 4 x (decode + GEMV), "
-                      f"single thread, {dt:.3f} s"}
+def cpu_baseline():
+    cores = os.cpu_count() or 1
+    _oracle_sample(ORACLE_ROWS_CPU)
+    dt1, nw, fl = oracle_step_sample(ORACLE_ROWS_CPU, 1)
+    dtn, _, _ = oracle_step_sample(ORACLE_ROWS_CPU, cores)
+    return {"value": 2.0 * nw / dtn / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "single_thread_value": 2.0 * nw / dt1 / 1e9, "tflops_all_cores": fl / dtn / 1e12,
+            "sample": f"{ORACLE_ROWS_CPU} rows of each of gate, up and down (layer 0 shapes and std), at each M in {MS}: "
+                      f"rebuild rows from the palette form + X.W^T in fp32 ({nw} weights x batch); "
+                      f"{cores} threads {dtn:.2f} s, 1 thread {dt1:.2f} s"}
 
 
 def run_reference(args):
@@ -175,22 +233,24 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    rows = 256
+    cores = os.cpu_count() or 1
+    rows = ORACLE_ROWS_REF
+    _oracle_sample(rows)
     for _ in range(args.warmup):
-        oracle_step_sample(rows)
-    tot = 0.0
-    nw = 0
+        oracle_step_sample(rows, cores)
+    tot, nw = 0.0, 0
     for _ in range(args.steps):
-        dt, nw = oracle_step_sample(rows)
+        dt, nw, _ = oracle_step_sample(rows, cores)
         tot += dt
-    value = len(OPS) * 2.0 * nw * args.steps / tot / 1e9
+    value = 2.0 * nw * args.steps / tot / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "oracle_rows_per_step": rows, "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} of 14336 rows per step, single thread"},
+            "config": {"workload": WORKLOAD, "oracle_rows_per_projection_per_step": rows, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} rows of each of gate, up and down at each M in {MS} "
+                                       f"per step, {cores} threads"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -198,109 +258,30 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def run_stack(args):
-    """The 32-layer stack of Llama-3.1-8B-shaped MLP weights (synthetic, a
-    per-layer seed and std): every gate, up and down matrix compressed and
-    kept resident, the total footprint per form against BF16, and the
-    autotuner's plan (pipeline and decoder SM split per projection and batch
-    size, measured on layer 0) with the measured time of one layer's MLP
-    matmuls.  Prints one JSON line; not part of the timed benchmark."""
-    import numpy as np
-    import torch
-    import decode_gemm_bf16_b200 as uw
-    import synthetic as S
-
-    dev = torch.device("cuda", 0)
-    Ms = [1, 8, 64, 256, 1024]
-    t_start = time.time()
-    blobs, bf16_bytes, huff, pal, devb = [], 0, 0, 0, 0
-    for layer in range(args.layers):
-        for W in S.stack_layer(layer):
-            Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
-            b = uw.uw_compress(Wd)
-            del Wd
-            info = b.info
-            bf16_bytes += 2 * W.size
-            huff += info["bytes_huffman_form"]
-            pal += info["bytes_palette_form"]
-            devb += info["device_bytes"]
-            blobs.append(b)
-    torch.cuda.synchronize()
-    t_compress = time.time() - t_start
-    proj = blobs[:3]
-    Xs = [torch.from_numpy(S.activations(max(Ms), b.info["K"], seed=7 + i).view(np.int16)).to(dev).view(torch.bfloat16)
-          for i, b in enumerate(proj)]
-    Ys = [torch.empty(max(Ms), b.info["N"], dtype=torch.bfloat16, device=dev) for b in proj]
-    need = max(uw.uw_gemm_workspace(b, max(Ms), p, sm_dec=sd) for b in proj for p in uw.PIPELINES for sd in (0, 296))
-    ws = torch.empty(need, dtype=torch.uint8, device=dev)
-    plan = uw.uw_autotune(proj, Ms, Xs, Ys, ws, reps=5)
-    if uw.uw_last_device_status() != 0:
-        raise RuntimeError("device status set during the stack run")
-    layer_us = {str(M): sum(e["us"] for e in plan if e["M"] == M) for M in Ms}
-    flops = {str(M): 2.0 * M * sum(b.info["N"] * b.info["K"] for b in proj) for M in Ms}
-    line = {"stack": {"layers": args.layers, "matrices": len(blobs), "weights": bf16_bytes // 2,
-                      "bf16_bytes": bf16_bytes, "huffman_form_bytes": huff, "palette_form_bytes": pal,
-                      "device_image_bytes": devb, "ratio_huffman_form": huff / bf16_bytes,
-                      "ratio_palette_form": pal / bf16_bytes, "compress_s_incl_host_generation": t_compress},
-            "plan_layer0": plan,
-            "layer_mlp_us": layer_us,
-            "layer_mlp_tflops": {M: flops[M] / (layer_us[M] * 1e-6) / 1e12 for M in layer_us}}
-    print(json.dumps(line), flush=True)
+def _alg_bytes(info, pipeline, M, gemv):
+    """Bytes the method must move for one call (what a perfect kernel reads
+    and writes): the compressed planes it reads, intermediate planes written
+    and read back, activations and outputs."""
+    sec = info["sections"]
+    n = info["N"] * info["K"]
+    stream_b = sec["stream"][1] + sec["chunk_off"][1] + sec["seg_rel"][1]
+    vstore = sec["vbits"][1] + sec["vpre"][1] + sec["vexp"][1]
+    vcol = 0 if gemv else sec["vcol"][1]
+    xy = 2 * M * (info["N"] + info["K"])
+    if pipeline == "direct_palette":
+        return n + n // 2 + vstore + vcol + xy
+    if pipeline == "transcode":
+        return (stream_b + n // 2) + (n + n // 2 + vstore + vcol + xy)
+    if pipeline == "exponent":
+        return (stream_b + vstore + n) + (2 * n + xy)
+    return (stream_b + vstore + n + 2 * n) + (2 * n + xy)   # full
 
 
-def uw_gemv_serves():
-    """Whether batch 1 on this projection runs the CUDA-core GEMV (the
-    library's rule: fewer than half as many 128-row tiles as GEMM CTAs)."""
-    import torch
-    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    return 2 * ((N_W + 127) // 128) < sms
-
-
-def batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak):
-    """Tensor-core GEMM at larger batches on the same projection (outside the
-    timed step): per M and pipeline, device time of one call (graph replays
-    over the rotated copies), TFLOP/s against the measured dense BF16 peak
-    and effective BF16 weight GB/s."""
-    import numpy as np
-    n = N_W * K_W
-    Wd = torch.from_numpy(S.gate_projection().view(np.int16)).to(dev).view(torch.bfloat16)
-    dense = [Wd] + [Wd.clone() for _ in range(3)]
-    out = {}
-    for M in (16, 64, 256, 1024):
-        X = torch.from_numpy(S.activations(M, K_W, seed=M + S.X_SEED_OFFSET).view(np.int16)).to(dev).view(torch.bfloat16)
-        Y = torch.empty(M, N_W, dtype=torch.bfloat16, device=dev)
-        wsb = max([uw.uw_gemm_workspace(copies[0], M, p) for p in ("direct_palette", "exponent")] +
-                  [uw.uw_dense_gemm_workspace(M, N_W, K_W)])
-        ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
-        row = {}
-        for name in ("direct_palette", "exponent", "dense"):
-            if name == "dense":
-                fns = [lambda w=w: uw.uw_dense_gemm(X, w, out=Y, ws=ws) for w in dense]
-            else:
-                fns = [lambda b=b, name=name: uw.uw_gemm(X, b, name, out=Y, ws=ws) for b in copies]
-            with torch.cuda.stream(cap):
-                for f in fns:
-                    f()
-            torch.cuda.synchronize()
-            g = capture(lambda: [fns[i % len(fns)]() for i in range(OP_BURST)])
-            for i in range(2):
-                g.replay()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 8
-            a.record()
-            for i in range(reps):
-                g.replay()
-            b.record()
-            torch.cuda.synchronize()
-            us = 1e3 * a.elapsed_time(b) / (reps * OP_BURST)
-            tflops = 2.0 * M * n / (us / 1e6) / 1e12
-            row[name] = {"us": us, "tflops": tflops, "tensor_frac": tflops / tc_peak,
-                         "eff_weight_gbs": 2.0 * n / (us / 1e6) / 1e9}
-            del g
-        out[str(M)] = row
-    if uw.uw_last_device_status() != 0:
-        raise RuntimeError("device status set during the batch sweep")
-    return out
+def _kernel_name(pipeline, gemv):
+    if pipeline == "full":
+        return "k_gemv<dense, M=1>" if gemv else "k_gemm_dense"
+    src = "exponent" if pipeline == "exponent" else "palette"
+    return f"k_gemv<{src}, M=1>" if gemv else f"k_gemm_recon<{src}>"
 
 
 def run_gpu(args):
@@ -312,36 +293,73 @@ def run_gpu(args):
     dist, rank, world, local = _dist()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    hbm_peak, tc_peak, peak_kind = _peaks()
+    hbm_peak, tc_burst, tc_sust, peak_kind = _peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    L = args.layers
+    t_start = time.time()
 
-    W = S.gate_projection()
-    x = S.activations(M_X, K_W, seed=1 + S.X_SEED_OFFSET)
-    Wd = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
-    copies = [uw.uw_compress(Wd) for _ in range(4)]
-    del Wd
-    info = copies[0].info
-    n = N_W * K_W
-    xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
-    wsb = max(uw.uw_gemm_workspace(copies[0], M_X, p) for p in uw.PIPELINES)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
-    out_full = torch.empty(N_W, K_W, dtype=torch.bfloat16, device=dev)
-    out_e = torch.empty(n, dtype=torch.uint8, device=dev)
-    out_i = torch.empty(n // 2, dtype=torch.uint8, device=dev)
-    Ys = [torch.empty(M_X, N_W, dtype=torch.bfloat16, device=dev) for _ in range(4)]
-    stream = torch.cuda.current_stream()
+    # ---- the stack: draw, compress, keep resident (dense copies of the first
+    # few layers stay too, for the dense baseline)
+    n_dense = min(4, L)
+    blobs = [[None] * 3 for _ in range(L)]
+    dense = [[None] * 3 for _ in range(n_dense)]
+    foot = {"bf16": 0, "huffman_form": 0, "palette_form": 0, "device_image": 0}
+    per_proj_ratio = {p: [0, 0, 0] for p in PROJ}
+    for layer in range(L):
+        mats = S.stack_layer_device(layer, dev)
+        for j, W in enumerate(mats):
+            b = uw.uw_compress(W)
+            blobs[layer][j] = b
+            info = b.info
+            nbytes = 2 * W.numel()
+            foot["bf16"] += nbytes
+            foot["huffman_form"] += info["bytes_huffman_form"]
+            foot["palette_form"] += info["bytes_palette_form"]
+            foot["device_image"] += info["device_bytes"]
+            r = per_proj_ratio[PROJ[j]]
+            r[0] += nbytes
+            r[1] += info["bytes_huffman_form"]
+            r[2] += info["bytes_palette_form"]
+            if layer < n_dense:
+                dense[layer][j] = W
+        del mats
+    torch.cuda.synchronize()
+    t_compress = time.time() - t_start
 
-    def op(k, blob, xin):
-        if k == 0:
-            uw.uw_decode_full(blob, out_full)
-        elif k == 1:
-            uw.uw_decode_exponent(blob, out_e)
-        elif k == 2:
-            uw.uw_transcode_palette(blob, out_i)
-        else:
-            uw.uw_gemm(xin, blob, k - 3, out=Ys[k - 3], ws=ws)
+    # activations per (projection input width, M); outputs per (projection, M)
+    Xg = {M: S.activations_device(M, 4096, seed=17 + M, device=dev) for M in MS}
+    Xd = {M: S.activations_device(M, 14336, seed=29 + M, device=dev) for M in MS}
+    Xof = {"gate": Xg, "up": Xg, "down": Xd}
+    Y = {(p, M): torch.empty(M, SHAPES[p][0], dtype=torch.bfloat16, device=dev) for p in PROJ for M in MS}
 
-    nops = len(OPS)
-    ncopy = len(copies)
+    # ---- autotune on the first layers (each layer is a copy of the shapes)
+    n_copies = min(4, L)
+    tune_blobs = [blobs[c][j] for c in range(n_copies) for j in range(3)]
+    Mmax = max(MS)
+    tX = [Xg[Mmax], Xg[Mmax], Xd[Mmax]]
+    tY = [Y[(p, Mmax)] for p in PROJ]
+    need = max(uw.uw_gemm_workspace(b, Mmax, p, sm_dec=sd) for b in blobs[0] for p in uw.PIPELINES
+               for sd in (0, sms // 2, sms, 2 * sms))
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    t_tune = time.time()
+    plan_entries = uw.uw_autotune(tune_blobs, MS, tX, tY, ws, reps=3, copies=n_copies)
+    t_tune = time.time() - t_tune
+    plan = uw.Plan(plan_entries)
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during autotuning")
+    choice = {(PROJ[e["projection"]], e["M"]): e for e in plan_entries}
+
+    def call(p, M, layer, xin=None, yout=None):
+        j = PROJ.index(p)
+        uw.uw_gemm(xin if xin is not None else Xof[p][M], blobs[layer][j], "auto",
+                   out=yout if yout is not None else Y[(p, M)], ws=ws, plan=plan, projection=j)
+
+    def step():
+        for M in MS:
+            for layer in range(L):
+                for p in PROJ:
+                    call(p, M, layer)
+
     cap = torch.cuda.Stream(device=dev)
 
     def capture(fn):
@@ -350,31 +368,29 @@ def run_gpu(args):
             fn()
         return g
 
-    # every op once eagerly (sets kernel attributes), then one graph per
-    # rotation of the weight copies: step r runs op k on copy (r + k) % 4
     with torch.cuda.stream(cap):
-        for k in range(nops):
-            op(k, copies[k % ncopy], xd)
+        step()                       # eager once: kernel attributes, side streams
     torch.cuda.synchronize()
-    step_graphs = [capture(lambda r=r: [op(k, copies[(r + k) % ncopy], xd) for k in range(nops)])
-                   for r in range(ncopy)]
-    # per-op graphs: OP_BURST launches of one op over the rotated copies, so the
-    # per-launch time is not inflated by the gap between graph launches
-    op_graphs = [capture(lambda k=k: [op(k, copies[i % ncopy], xd) for i in range(OP_BURST)]) for k in range(nops)]
+    step_graph = capture(step)
+    launches_per_step = 0
+    for M in MS:
+        for p in PROJ:
+            e = choice[(p, M)]
+            per_call = 1 + (0 if e["pipeline"] == "direct_palette" else 1)
+            launches_per_step += L * per_call
 
-    # warm-up: W steps, and at least half a second of work so the clocks settle
+    # warm-up: W steps, and at least a second of work so the clocks settle
     t_w = time.time()
     i = 0
-    while i < max(3, args.warmup) or time.time() - t_w < 0.5:
-        step_graphs[i % ncopy].replay()
+    while i < max(3, args.warmup) or time.time() - t_w < 1.0:
+        step_graph.replay()
         i += 1
-        if i % 50 == 0:
-            torch.cuda.synchronize()
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
     # ---- timed region: K steps (graph replays), device time with CUDA events
+    stream = torch.cuda.current_stream()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -384,7 +400,7 @@ def run_gpu(args):
         clk.mark("t0")
         t0.record(stream)
         for i in range(args.steps):
-            step_graphs[i % ncopy].replay()
+            step_graph.replay()
         t1.record(stream)
         torch.cuda.synchronize()
         clk.mark("t1")
@@ -393,112 +409,190 @@ def run_gpu(args):
     ms = t0.elapsed_time(t1)
     if dist:
         ms = max_over_ranks(ms, dist, dev)
-    # per-op device time: each op alone, rotated over the copies
-    reps = max(10, min(100, args.steps // 20))
-    per_op_ms = []
-    for k in range(nops):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for i in range(2):
-            op_graphs[k].replay()
-        a.record(stream)
-        for i in range(reps):
-            op_graphs[k].replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        per_op_ms.append(a.elapsed_time(b) / (reps * OP_BURST))
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the timed region")
-    sweep = batch_sweep(uw, torch, S, copies, dev, cap, capture, tc_peak, hbm_peak) if not args.no_sweep else None
+    del step_graph
 
-    # ---- end to end: host x (pinned) -> device, the step, Y -> host (pinned)
-    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = [torch.empty(M_X, N_W, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
-    xdev = torch.empty_like(xd)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for k in range(nops):
-        op(k, copies[k % ncopy], xdev)
+    def time_graph(g, launches, reps=5):
+        for _ in range(2):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * a.elapsed_time(b) / (reps * launches)   # microseconds per launch
+
+    # ---- per (projection, M): the plan's call alone, over all layers; the
+    # dense baseline over the dense copies
+    dense_ws = torch.zeros(max(uw.uw_dense_gemm_workspace(M, *SHAPES[p]) for p in PROJ for M in MS),
+                           dtype=torch.uint8, device=dev)
+    per = {}
+    for p in PROJ:
+        N, K = SHAPES[p]
+        info = blobs[0][PROJ.index(p)].info
+        for M in MS:
+            g = capture(lambda p=p, M=M: [call(p, M, layer) for layer in range(L)])
+            us = time_graph(g, L)
+            del g
+            nd = n_dense * max(1, OP_BURST // n_dense)
+            gd = capture(lambda p=p, M=M: [uw.uw_dense_gemm(Xof[p][M], dense[i % n_dense][PROJ.index(p)],
+                                                            out=Y[(p, M)], ws=dense_ws) for i in range(nd)])
+            us_dense = time_graph(gd, nd)
+            del gd
+            e = choice[(p, M)]
+            gemv = (e["variant"] == 2) or (e["variant"] == 0 and M == 1 and e["sm_dec"] == 0 and
+                                            2 * ((N + 127) // 128) < (e["grid"] or sms))
+            alg = _alg_bytes(info, e["pipeline"], M, gemv)
+            flops = 2.0 * M * N * K
+            gbs = alg / (us * 1e-6) / 1e9
+            tfl = flops / (us * 1e-6) / 1e12
+            per[f"{p}/M={M}"] = {
+                "us": us, "pipeline": e["pipeline"], "variant": e["variant"], "sm_dec": e["sm_dec"],
+                "grid": e["grid"], "split_k": e["split_k"], "kernel": _kernel_name(e["pipeline"], gemv),
+                "alg_bytes": alg, "compressed_gbs": gbs, "eff_weight_gbs": 2.0 * N * K / (us * 1e-6) / 1e9,
+                "tflops": tfl, "hbm_frac": gbs / hbm_peak, "tensor_frac": tfl / tc_burst,
+                "roofline_frac": max(gbs / hbm_peak, tfl / tc_burst),
+                "bound": "tensor" if tfl / tc_burst > gbs / hbm_peak else "hbm",
+                "dense_us": us_dense, "slowdown_vs_dense": us / us_dense,
+                "share_of_step": L * us / (1e3 * ms / args.steps)}
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set while timing single calls")
+
+    # ---- the decoders and the four pipelines at batch 1 on the gate
+    # projection (layers 0..3 rotated), and the SM split on the down projection
+    ops = {}
+    gate_blobs = [blobs[c][0] for c in range(n_copies)]
+    ginfo = gate_blobs[0].info
+    n = 14336 * 4096
+    out_full = torch.empty(14336, 4096, dtype=torch.bfloat16, device=dev)
+    out_e = torch.empty(n, dtype=torch.uint8, device=dev)
+    out_i = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    sec = ginfo["sections"]
+    stream_b = sec["stream"][1] + sec["chunk_off"][1] + sec["seg_rel"][1]
+    vstore = sec["vbits"][1] + sec["vpre"][1] + sec["vexp"][1]
+    dec_alg = {"decode_full": stream_b + vstore + 3 * n, "decode_exponent": stream_b + vstore + n,
+               "transcode": stream_b + n // 2}
+    dec_fn = {"decode_full": lambda b: uw.uw_decode_full(b, out_full),
+              "decode_exponent": lambda b: uw.uw_decode_exponent(b, out_e),
+              "transcode": lambda b: uw.uw_transcode_palette(b, out_i)}
+    for name, fn in dec_fn.items():
+        g = capture(lambda fn=fn: [fn(gate_blobs[i % n_copies]) for i in range(OP_BURST)])
+        us = time_graph(g, OP_BURST)
+        del g
+        ops[name] = {"us": us, "alg_bytes": dec_alg[name], "alg_gbs": dec_alg[name] / (us * 1e-6) / 1e9,
+                     "hbm_frac": dec_alg[name] / (us * 1e-6) / 1e9 / hbm_peak}
+    for pipe in ["full", "exponent", "transcode", "direct_palette"]:
+        g = capture(lambda pipe=pipe: [uw.uw_gemm(Xg[1], gate_blobs[i % n_copies], pipe, out=Y[("gate", 1)], ws=ws)
+                                       for i in range(OP_BURST)])
+        us = time_graph(g, OP_BURST)
+        del g
+        gemv = 2 * 112 < sms
+        alg = _alg_bytes(ginfo, pipe, 1, gemv)
+        ops[f"gemm_{pipe}"] = {"us": us, "alg_bytes": alg, "alg_gbs": alg / (us * 1e-6) / 1e9,
+                               "hbm_frac": alg / (us * 1e-6) / 1e9 / hbm_peak,
+                               "eff_weight_gbs": 2.0 * n / (us * 1e-6) / 1e9}
+    sm_split = {}
+    down_blobs = [blobs[c][2] for c in range(n_copies)]
+    for M in (256, 1024):
+        row = {}
+        for pipe, sds in (("direct_palette", (0,)), ("exponent", (0, sms // 4, sms // 2, sms, 2 * sms))):
+            for sd in sds:
+                g = capture(lambda pipe=pipe, sd=sd, M=M: [
+                    uw.uw_gemm(Xd[M], down_blobs[i % n_copies], pipe, out=Y[("down", M)], ws=ws, sm_dec=sd)
+                    for i in range(n_copies)])
+                us = time_graph(g, n_copies, reps=3)
+                del g
+                row[f"{pipe}/sm_dec={sd}"] = {"us": us, "tflops": 2.0 * M * 4096 * 14336 / (us * 1e-6) / 1e12}
+        sm_split[f"M={M}"] = row
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set during the breakdowns")
+
+    # ---- end to end: every step, the activations of every batch size are
+    # copied from pinned host memory, the step runs through the public API
+    # (eager calls, no graph), and every batch's last down-projection output
+    # is copied back to pinned host memory
+    xh = {(w, M): (Xg if w == 4096 else Xd)[M].cpu().pin_memory() for w in (4096, 14336) for M in MS}
+    yh = {M: torch.empty(M, 4096, dtype=torch.bfloat16).pin_memory() for M in MS}
+    xdev = {k: torch.empty_like(v, device=dev) for k, v in xh.items()}
+    h2d = sum(v.numel() * 2 for v in xh.values())
+    d2h = sum(v.numel() * 2 for v in yh.values())
+
+    def e2e_step():
+        for (w, M), t in xh.items():
+            xdev[(w, M)].copy_(t, non_blocking=True)
+        for M in MS:
+            for layer in range(L):
+                for p in PROJ:
+                    call(p, M, layer, xin=xdev[(4096 if p != "down" else 14336, M)])
+            yh[M].copy_(Y[("down", M)], non_blocking=True)
+
+    e2e_step()
     torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    ctr = 0
-    for i in range(args.steps):
-        xdev.copy_(xh, non_blocking=True)
-        for k in range(nops):
-            op(k, copies[ctr % ncopy], xdev)
-            ctr += 1
-        for j in range(4):
-            yh[j].copy_(Ys[j], non_blocking=True)
+    for _ in range(e2e_steps):
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if dist:
         e2e_ms = max_over_ranks(e2e_ms, dist, dev)
 
     # ---- numbers
-    eff_bytes_step = nops * 2.0 * n
-    value = world * eff_bytes_step * args.steps / (ms / 1e3) / 1e9
-    e2e = world * eff_bytes_step * args.steps / (e2e_ms / 1e3) / 1e9
-    sec = info["sections"]
-    stream_b = sec["stream"][1] + sec["chunk_off"][1] + sec["seg_rel"][1]
-    vstore = sec["vbits"][1] + sec["vpre"][1] + sec["vexp"][1]
-    xb, yb = M_X * K_W * 2, M_X * N_W * 2
-    # algorithmic bytes per launch of each single-kernel op (what must move)
-    alg = {
-        "decode_full": stream_b + vstore + n + 2 * n,
-        "decode_exponent": stream_b + vstore + n,
-        "transcode": stream_b + n // 2,
-        "gemm_direct_palette": n + n // 2 + vstore + xb + yb + (0 if uw_gemv_serves() else sec["vcol"][1]),
-    }
-    kernel_of = {"decode_full": "k_decode<full>", "decode_exponent": "k_decode<exponent>",
-                 "transcode": "k_decode<transcode>",
-                 "gemm_direct_palette": "k_gemv<palette, M=1>" if uw_gemv_serves() else "k_gemm_recon<palette>"}
-    breakdown = {}
-    for k, name in enumerate(OPS):
-        d = {"us": 1e3 * per_op_ms[k], "eff_weight_gbs": 2.0 * n / (per_op_ms[k] / 1e3) / 1e9,
-             "tflops": (2.0 * M_X * n / (per_op_ms[k] / 1e3) / 1e12) if name.startswith("gemm") else None}
-        if name in alg:
-            d["alg_bytes"] = alg[name]
-            d["alg_gbs"] = alg[name] / (per_op_ms[k] / 1e3) / 1e9
-            d["hbm_frac"] = d["alg_gbs"] / hbm_peak
-        breakdown[name] = d
-    # dominant single-kernel op: the decode_full kernel also runs inside the
-    # full pipeline, the palette GEMM inside the transcode pipeline
-    share = {"decode_full": per_op_ms[0] * 2, "decode_exponent": per_op_ms[1] * 2,
-             "transcode": per_op_ms[2] * 2, "gemm_direct_palette": per_op_ms[6] * 2}
-    dom = max(share, key=share.get)
-    dom_ms = per_op_ms[OPS.index(dom)]
-    achieved = alg[dom] / (dom_ms / 1e3) / 1e9
-    # DRAM bytes per launch from the committed ncu capture, only while the
-    # kernel is the one that capture measured (same code hash of its
-    # translation unit: sources without comments, plus build flags)
-    traffic = None
+    weight_bytes_pass = sum(2 * SHAPES[p][0] * SHAPES[p][1] for p in PROJ) * L
+    eff_bytes_step = weight_bytes_pass * len(MS)
+    flops_step = sum(2.0 * M * SHAPES[p][0] * SHAPES[p][1] for p in PROJ for M in MS) * L
+    ms_step = ms / args.steps
+    value = world * eff_bytes_step / (ms_step / 1e3) / 1e9
+    e2e = world * eff_bytes_step / (e2e_ms / 1e3) / 1e9
+    # dominant kernel: the (projection, M) call with the largest share of the step
+    dom_key = max(per, key=lambda k: per[k]["share_of_step"])
+    d = per[dom_key]
+    if d["bound"] == "tensor":
+        roof = {"bound": "tensor", "kernel": d["kernel"], "call": dom_key, "achieved": d["tflops"],
+                "peak": tc_burst, "peak_kind": f"{peak_kind} bf16_tflops (cuBLAS, burst; call timed alone)",
+                "unit": "TFLOP/s", "frac": d["tflops"] / tc_burst,
+                "frac_of_sustained": d["tflops"] / tc_sust}
+    else:
+        roof = {"bound": "hbm", "kernel": d["kernel"], "call": dom_key, "achieved": d["compressed_gbs"],
+                "peak": hbm_peak, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",
+                "frac": d["compressed_gbs"] / hbm_peak}
+    roof["traffic"] = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         try:
             from decode_gemm_bf16_b200 import build as uwbuild
             tj = json.load(open(tp))
-            ent = tj["bytes_per_launch"].get(kernel_of[dom])
-            if ent and ent.get("code_hash") == uwbuild.kernel_code_hash(kernel_of[dom]):
-                traffic = ent["bytes"]
+            ent = tj["bytes_per_launch"].get(f"{d['kernel']} {dom_key}")
+            if ent and ent.get("code_hash") == uwbuild.kernel_code_hash(d["kernel"]):
+                roof["traffic"] = ent["bytes"]
         except Exception:
-            traffic = None
-    launches_per_step = 3 + 2 + 2 + 2 + 1
+            roof["traffic"] = None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M_X, "N": N_W, "K": K_W, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2: 4 rotating compressed copies",
-                   "ratio_huffman_form": info["bytes_huffman_form"] / (2 * n),
-                   "ratio_palette_form": info["bytes_palette_form"] / (2 * n),
-                   "mean_code_bits": info["mean_code_len"]},
-        "roofline": {"bound": "hbm", "kernel": kernel_of[dom], "achieved": achieved, "peak": hbm_peak,
-                     "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": traffic},
-        "breakdown": breakdown,
-        "batch_sweep": sweep,
-        "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": xb, "d2h_bytes_per_step": 4 * yb},
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (device-drawn, seeded)",
+        "tflops": world * flops_step / (ms_step / 1e3) / 1e12,
+        "config": {"workload": WORKLOAD, "layers": L, "batches": MS, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: consecutive calls read different matrices (96 resident)",
+                   "plan": {k: {kk: v[kk] for kk in ("pipeline", "variant", "sm_dec", "grid", "split_k")}
+                            for k, v in per.items()}},
+        "roofline": roof,
+        "per_call": per,
+        "footprint": dict(foot, ratio_huffman_form=foot["huffman_form"] / foot["bf16"],
+                          ratio_palette_form=foot["palette_form"] / foot["bf16"],
+                          per_projection={p: {"ratio_huffman_form": r[1] / r[0], "ratio_palette_form": r[2] / r[0]}
+                                          for p, r in per_proj_ratio.items()}),
+        "ops_gate_M1": ops,
+        "sm_split_down": sm_split,
+        "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "path": "eager uw_gemm calls (ctypes C ABI), UW_PIPE_AUTO"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "setup_s": {"draw_and_compress": t_compress, "autotune": t_tune},
     }
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline()
@@ -512,19 +606,15 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--no-sweep", action="store_true", help="skip the larger-batch GEMM sweep")
-    ap.add_argument("--stack", action="store_true",
-                    help="compress the synthetic 32-layer MLP stack, report footprint and the autotuned plan")
-    ap.add_argument("--layers", type=int, default=32, help="layers for --stack")
+    ap.add_argument("--layers", type=int, default=32, help="layers of the stack (32 = Llama-3.1-8B)")
+    ap.add_argument("--stack", action="store_true", help="same as the default run (kept for old command lines)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
-    elif args.stack:
-        run_stack(args)
     else:
         run_gpu(args)
 

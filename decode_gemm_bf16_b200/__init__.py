@@ -24,8 +24,10 @@ UW_OK = 0
 STATUS = {0: "UW_OK", 1: "UW_ERR_INVALID_ARG", 2: "UW_ERR_SHAPE", 3: "UW_ERR_CORRUPT",
           4: "UW_ERR_UNSUPPORTED", 5: "UW_ERR_WORKSPACE", 6: "UW_ERR_CUDA", 7: "UW_ERR_TIMEOUT",
           8: "UW_ERR_DEVICE"}
-UW_PIPE_FULL, UW_PIPE_EXPONENT, UW_PIPE_TRANSCODE, UW_PIPE_DIRECT_PALETTE = 0, 1, 2, 3
+UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXPONENT, UW_PIPE_TRANSCODE, UW_PIPE_DIRECT_PALETTE = -1, 0, 1, 2, 3
 PIPELINES = {"full": 0, "exponent": 1, "transcode": 2, "direct_palette": 3}
+UW_VARIANT_AUTO, UW_VARIANT_TENSOR, UW_VARIANT_GEMV = 0, 1, 2
+VARIANTS = {"auto": 0, "tensor": 1, "gemv": 2}
 UW_FORM_HUFFMAN, UW_FORM_PALETTE = 1, 2
 SECTIONS = ["sm", "vbits", "vpre", "vexp", "vcol", "idx", "stream", "chunk_off", "seg_rel", "lut"]
 
@@ -35,7 +37,8 @@ EXPORTS = ["uw_status_str", "uw_version", "uw_last_device_status", "uw_compress_
            "uw_blob_serialized_bytes", "uw_blob_serialize", "uw_blob_device_bytes",
            "uw_blob_deserialize", "uw_blob_free", "uw_decode_full", "uw_decode_exponent",
            "uw_transcode_palette", "uw_gemm_workspace", "uw_gemm", "uw_dense_gemm_workspace",
-           "uw_dense_gemm", "uw_autotune", "uw_gemm_direct_palette_noalloc"]
+           "uw_dense_gemm", "uw_autotune", "uw_gemm_direct_palette_noalloc", "uw_plan_resolve",
+           "uw_plan_load_json"]
 
 
 class UnweightError(RuntimeError):
@@ -56,15 +59,18 @@ class BlobInfo(ctypes.Structure):
                 ("section_bytes", ctypes.c_uint64 * 10)]
 
 
-class GemmOpts(ctypes.Structure):
-    _fields_ = [("pipeline", ctypes.c_int32), ("sm_dec", ctypes.c_int32), ("grid", ctypes.c_int32),
-                ("out_f32", ctypes.c_int32), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
-
-
 class PlanEntry(ctypes.Structure):
     _fields_ = [("blob_index", ctypes.c_int32), ("M", ctypes.c_int64), ("pipeline", ctypes.c_int32),
-                ("sm_dec", ctypes.c_int32), ("grid", ctypes.c_int32), ("us", ctypes.c_double)]
+                ("variant", ctypes.c_int32), ("sm_dec", ctypes.c_int32), ("grid", ctypes.c_int32),
+                ("split_k", ctypes.c_int32), ("us", ctypes.c_double), ("layer_us", ctypes.c_double)]
+
+
+class GemmOpts(ctypes.Structure):
+    _fields_ = [("pipeline", ctypes.c_int32), ("sm_dec", ctypes.c_int32), ("grid", ctypes.c_int32),
+                ("out_f32", ctypes.c_int32), ("variant", ctypes.c_int32), ("split_k", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("projection", ctypes.c_int32),
+                ("plan", ctypes.POINTER(PlanEntry)), ("plan_entries", ctypes.c_int32),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -98,11 +104,13 @@ def lib():
             "uw_transcode_palette": ([P, P, P], I32),
             "uw_gemm_workspace": ([P, I64, ctypes.POINTER(GemmOpts), ctypes.POINTER(SZ)], I32),
             "uw_gemm": ([P, I64, P, P, ctypes.POINTER(GemmOpts), P], I32),
-            "uw_dense_gemm_workspace": ([I64, I64, I64, I32, ctypes.POINTER(SZ)], I32),
-            "uw_dense_gemm": ([P, I64, P, I64, I64, P, I32, I32, P, SZ, P], I32),
+            "uw_plan_resolve": ([ctypes.POINTER(GemmOpts), I64, ctypes.POINTER(GemmOpts)], I32),
+            "uw_dense_gemm_workspace": ([I64, I64, I64, I32, I32, I32, ctypes.POINTER(SZ)], I32),
+            "uw_dense_gemm": ([P, I64, P, I64, I64, P, I32, I32, I32, I32, P, SZ, P], I32),
             "uw_gemm_direct_palette_noalloc": ([P, I64, P, P, I32, P], I32),
-            "uw_autotune": ([ctypes.POINTER(P), I32, ctypes.POINTER(I64), I32, ctypes.POINTER(P),
+            "uw_autotune": ([ctypes.POINTER(P), I32, I32, ctypes.POINTER(I64), I32, ctypes.POINTER(P),
                              ctypes.POINTER(P), P, SZ, I32, ctypes.POINTER(PlanEntry), ctypes.c_char_p, P], I32),
+            "uw_plan_load_json": ([ctypes.c_char_p, ctypes.POINTER(PlanEntry), I32, ctypes.POINTER(I32)], I32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -233,22 +241,66 @@ def uw_transcode_palette(blob: Blob, out: Optional[torch.Tensor] = None, stream=
     return out
 
 
-def _opts(pipeline, sm_dec=0, grid=0, out_f32=False, ws: Optional[torch.Tensor] = None) -> GemmOpts:
+def _variant(v) -> int:
+    return VARIANTS[v] if isinstance(v, str) else int(v)
+
+
+class Plan:
+    """Autotuner entries held in host memory (the array uw_gemm reads under
+    UW_PIPE_AUTO)."""
+
+    def __init__(self, entries: Sequence[dict]):
+        self.entries = list(entries)
+        self._arr = (PlanEntry * max(1, len(self.entries)))()
+        for i, e in enumerate(self.entries):
+            a = self._arr[i]
+            a.blob_index, a.M = int(e["projection"]), int(e["M"])
+            p = e["pipeline"]
+            a.pipeline = PIPELINES[p] if isinstance(p, str) else int(p)
+            a.variant, a.sm_dec = int(e.get("variant", 0)), int(e.get("sm_dec", 0))
+            a.grid, a.split_k = int(e.get("grid", 0)), int(e.get("split_k", 0))
+            a.us, a.layer_us = float(e.get("us", 0.0)), float(e.get("layer_us", 0.0))
+
+    def __len__(self):
+        return len(self.entries)
+
+
+def _opts(pipeline, sm_dec=0, grid=0, out_f32=False, ws: Optional[torch.Tensor] = None, variant=0,
+          split_k=0, stages=0, plan: Optional[Plan] = None, projection: int = 0) -> GemmOpts:
     o = GemmOpts()
+    if pipeline == "auto":
+        pipeline = UW_PIPE_AUTO
     o.pipeline = PIPELINES[pipeline] if isinstance(pipeline, str) else int(pipeline)
     o.sm_dec = int(sm_dec)
     o.grid = int(grid)
     o.out_f32 = 1 if out_f32 else 0
+    o.variant = _variant(variant)
+    o.split_k = int(split_k)
+    o.stages = int(stages)
+    o.projection = int(projection)
+    if plan is not None:
+        o.plan = ctypes.cast(plan._arr, ctypes.POINTER(PlanEntry))
+        o.plan_entries = len(plan)
     o.workspace = ws.data_ptr() if ws is not None else None
     o.workspace_bytes = ws.numel() if ws is not None else 0
     return o
 
 
-def uw_gemm_workspace(blob: Blob, M: int, pipeline="direct_palette", sm_dec=0, grid=0) -> int:
-    o = _opts(pipeline, sm_dec, grid)
+def uw_gemm_workspace(blob: Blob, M: int, pipeline="direct_palette", sm_dec=0, grid=0, variant=0, split_k=0,
+                      plan: Optional[Plan] = None, projection: int = 0) -> int:
+    o = _opts(pipeline, sm_dec, grid, variant=variant, split_k=split_k, plan=plan, projection=projection)
     n = ctypes.c_size_t()
     _check(lib().uw_gemm_workspace(blob.handle, int(M), ctypes.byref(o), ctypes.byref(n)), "uw_gemm_workspace")
     return n.value
+
+
+def uw_plan_resolve(plan: Plan, projection: int, M: int) -> dict:
+    """The options UW_PIPE_AUTO takes for (projection, M) under `plan`."""
+    o = _opts("auto", plan=plan, projection=projection)
+    r = GemmOpts()
+    _check(lib().uw_plan_resolve(ctypes.byref(o), int(M), ctypes.byref(r)), "uw_plan_resolve")
+    names = {v: k for k, v in PIPELINES.items()}
+    return dict(pipeline=names[r.pipeline], variant=r.variant, sm_dec=r.sm_dec, grid=r.grid, split_k=r.split_k)
 
 
 _ws_cache = {}
@@ -266,16 +318,20 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 def uw_gemm(X: torch.Tensor, blob: Blob, pipeline="direct_palette", out: Optional[torch.Tensor] = None,
             out_f32: bool = False, ws: Optional[torch.Tensor] = None, sm_dec: int = 0, grid: int = 0,
+            variant=0, split_k: int = 0, stages: int = 0, plan: Optional[Plan] = None, projection: int = 0,
             stream=None) -> torch.Tensor:
-    """Y[M, N] = X[M, K] . W^T with W compressed in `blob` (tensor cores; batch 1
-    on a projection with few 128-row tiles runs the library's CUDA-core GEMV)."""
+    """Y[M, N] = X[M, K] . W^T with W compressed in `blob`.  pipeline "auto"
+    takes the plan's choice for (projection, M).  Tensor cores, except batch 1
+    on a projection with few 128-row tiles (or variant "gemv"): the library's
+    CUDA-core GEMV."""
     X = _bits16(X)
     M = X.shape[0]
     if out is None:
         out = torch.empty(M, blob.N, dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
     if ws is None:
-        ws = workspace(uw_gemm_workspace(blob, M, pipeline, sm_dec, grid), X.device)
-    o = _opts(pipeline, sm_dec, grid, out_f32, ws)
+        ws = workspace(uw_gemm_workspace(blob, M, pipeline, sm_dec, grid, variant, split_k, plan, projection),
+                       X.device)
+    o = _opts(pipeline, sm_dec, grid, out_f32, ws, variant, split_k, stages, plan, projection)
     _check(lib().uw_gemm(_ptr(X), M, blob.handle, _ptr(out), ctypes.byref(o), _stream(stream)), "uw_gemm")
     return out
 
@@ -294,15 +350,16 @@ def uw_gemm_direct_palette_noalloc(X: torch.Tensor, blob: Blob, out: Optional[to
     return out
 
 
-def uw_dense_gemm_workspace(M: int, N: int, K: int, grid: int = 0) -> int:
+def uw_dense_gemm_workspace(M: int, N: int, K: int, grid: int = 0, variant=0, split_k: int = 0) -> int:
     n = ctypes.c_size_t()
-    _check(lib().uw_dense_gemm_workspace(int(M), int(N), int(K), int(grid), ctypes.byref(n)),
-           "uw_dense_gemm_workspace")
+    _check(lib().uw_dense_gemm_workspace(int(M), int(N), int(K), _variant(variant), int(grid), int(split_k),
+                                         ctypes.byref(n)), "uw_dense_gemm_workspace")
     return n.value
 
 
 def uw_dense_gemm(X: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = None, out_f32: bool = False,
-                  ws: Optional[torch.Tensor] = None, grid: int = 0, stream=None) -> torch.Tensor:
+                  ws: Optional[torch.Tensor] = None, grid: int = 0, variant=0, split_k: int = 0,
+                  stream=None) -> torch.Tensor:
     """The uncompressed baseline: the same GEMM (tensor cores, or the GEMV where
     uw_gemm would use it) on plain BF16 W[N, K]."""
     X = _bits16(X)
@@ -312,9 +369,9 @@ def uw_dense_gemm(X: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] 
     if out is None:
         out = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
     if ws is None:
-        ws = workspace(uw_dense_gemm_workspace(M, N, K, grid), X.device)
-    _check(lib().uw_dense_gemm(_ptr(X), M, _ptr(W), N, K, _ptr(out), 1 if out_f32 else 0, int(grid), _ptr(ws),
-                               ws.numel(), _stream(stream)), "uw_dense_gemm")
+        ws = workspace(uw_dense_gemm_workspace(M, N, K, grid, variant, split_k), X.device)
+    _check(lib().uw_dense_gemm(_ptr(X), M, _ptr(W), N, K, _ptr(out), 1 if out_f32 else 0, _variant(variant),
+                               int(grid), int(split_k), _ptr(ws), ws.numel(), _stream(stream)), "uw_dense_gemm")
     return out
 
 
@@ -344,15 +401,34 @@ def uw_blob_deserialize(data: bytes, device="cuda", stream=None) -> Blob:
 
 
 def uw_autotune(blobs: Sequence[Blob], Ms: Sequence[int], X: Sequence[torch.Tensor], Y: Sequence[torch.Tensor],
-                ws: torch.Tensor, reps: int = 5, plan_json_path: Optional[str] = None, stream=None) -> list:
-    """Coordinate-descent choice of pipeline per projection and batch size."""
-    nb, nm = len(blobs), len(Ms)
+                ws: torch.Tensor, reps: int = 5, plan_json_path: Optional[str] = None, copies: int = 1,
+                stream=None) -> list:
+    """Coordinate-descent choice of pipeline, variant, grid and decoder split
+    per projection and batch size.  `blobs` holds `copies` copies of every
+    projection, copy-major ([copy0: p0, p1, ...], [copy1: ...]); X and Y one
+    buffer per projection."""
+    nb = len(blobs)
+    assert nb % copies == 0
+    nproj, nm = nb // copies, len(Ms)
     H = (ctypes.c_void_p * nb)(*[b.handle.value if hasattr(b.handle, "value") else b.handle for b in blobs])
     Ms_c = (ctypes.c_int64 * nm)(*[int(m) for m in Ms])
-    Xp = (ctypes.c_void_p * nb)(*[x.data_ptr() for x in X])
-    Yp = (ctypes.c_void_p * nb)(*[y.data_ptr() for y in Y])
-    plan = (PlanEntry * (nb * nm))()
-    _check(lib().uw_autotune(H, nb, Ms_c, nm, Xp, Yp, _ptr(ws), ws.numel(), int(reps), plan,
+    Xp = (ctypes.c_void_p * nproj)(*[x.data_ptr() for x in X])
+    Yp = (ctypes.c_void_p * nproj)(*[y.data_ptr() for y in Y])
+    plan = (PlanEntry * (nproj * nm))()
+    _check(lib().uw_autotune(H, nproj, copies, Ms_c, nm, Xp, Yp, _ptr(ws), ws.numel(), int(reps), plan,
                              plan_json_path.encode() if plan_json_path else None, _stream(stream)), "uw_autotune")
+    return [_entry_dict(p) for p in plan]
+
+
+def _entry_dict(p: PlanEntry) -> dict:
     names = {v: k for k, v in PIPELINES.items()}
-    return [dict(projection=p.blob_index, M=p.M, pipeline=names[p.pipeline], sm_dec=p.sm_dec, us=p.us) for p in plan]
+    return dict(projection=p.blob_index, M=p.M, pipeline=names[p.pipeline], variant=p.variant, sm_dec=p.sm_dec,
+                grid=p.grid, split_k=p.split_k, us=p.us, layer_us=p.layer_us)
+
+
+def uw_plan_load_json(path: str, cap: int = 4096) -> list:
+    """The plan entries of a JSON file written by uw_autotune."""
+    arr = (PlanEntry * cap)()
+    n = ctypes.c_int32()
+    _check(lib().uw_plan_load_json(path.encode(), arr, cap, ctypes.byref(n)), "uw_plan_load_json")
+    return [_entry_dict(arr[i]) for i in range(min(n.value, cap))]

@@ -756,11 +756,14 @@ uint64_t timeout_ns() {
 int gemm_default_grid() { return num_sms(); }
 
 // Batch 1 on a projection with fewer than half as many 128-row tiles as
-// GEMM CTAs (every tile would be cut several ways along k) runs the GEMV;
-// the choice depends only on the shape, never on the weight source, so the
-// pipelines and the dense baseline keep identical summation orders.
+// GEMM CTAs (every tile would be cut several ways along k) runs the GEMV
+// under UW_VARIANT_AUTO; the choice depends only on the shape and options,
+// never on the weight source, so the pipelines and the dense baseline keep
+// identical summation orders.
 bool gemv_serves(const GemmArgs& a) {
-    if (a.M != 1 || a.band_ready) return false;
+    if (a.band_ready) return false;
+    if (a.variant == UW_VARIANT_GEMV) return true;
+    if (a.variant == UW_VARIANT_TENSOR || a.M != 1) return false;
     const int64_t n_tiles = (a.N + kBlockN - 1) / kBlockN;
     const int64_t P = a.grid > 0 ? a.grid : gemm_default_grid();
     return 2 * n_tiles < P;
@@ -770,46 +773,70 @@ unsigned long long gemm_next_epoch() { return next_epoch(); }
 
 int gemm_status_take() { return unit_status_take(); }
 
-size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid) {
-    (void)N;
-    (void)K;
-    int P = grid > 0 ? grid : gemm_default_grid();
-    int MG = pick_mg(M);
-    size_t part = (size_t)2 * P * MG * kBlockN * 4;
-    size_t flags = (size_t)2 * P * kBlockN * 8;
+GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k) {
+    GemmSplit g;
+    g.MG = pick_mg(M);
+    // stage k: 128 for small batch tiles (halves the per-stage TMA, barrier
+    // and MMA-issue overhead per weight byte), 64 where a stage is already
+    // large (batch tiles above 64 rows)
+    g.KB = (g.MG <= 64 && K % 128 == 0) ? 128 : 64;
+    g.m_tiles = (int)((M + g.MG - 1) / g.MG);
+    g.n_tiles = (int)((N + kBlockN - 1) / kBlockN);
+    g.kt = (int)(K / g.KB);
+    g.tiles = (int64_t)g.m_tiles * g.n_tiles;
+    g.total = g.tiles * g.kt;
+    const int sms = gemm_default_grid();
+    int64_t P;
+    if (split_k > 0) {
+        // every tile cut into the same number of k ranges, one CTA each
+        const int64_t c = split_k < g.kt ? split_k : g.kt;
+        P = g.tiles * c;
+        if (c >= 2 && P > sms) g.ok = false;   // finishers would wait on CTAs of a later wave
+    } else {
+        P = grid > 0 ? grid : sms;
+        // Default grid: with batch tiles of 64+ rows and no more output tiles
+        // than SMs, every tile is cut into the same whole number of k ranges,
+        // one CTA each (one CTA per tile when the tiles number half the SMs
+        // or more): each CTA then holds a single segment, instead of a tail
+        // and a head whose fix-ups move 32-128 KB of fp32 partials per cut
+        // and stall the MMA while they are written.
+        if (grid == 0 && g.MG >= 64 && g.tiles <= P) P = g.tiles * (P / g.tiles);
+    }
+    if (P > g.total) P = g.total;
+    if (P < 1) P = 1;
+    if (P > 0x7FFFFFFF || g.total * P >= (int64_t(1) << 32)) g.ok = false;
+    g.P = (int)P;
+    g.fixup = P != g.tiles;
+    return g;
+}
+
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k) {
+    const GemmSplit g = gemm_split(M, N, K, grid, split_k);
+    if (!g.fixup) return 256;
+    size_t part = (size_t)2 * g.P * g.MG * kBlockN * 4;
+    size_t flags = (size_t)2 * g.P * kBlockN * 8;
     return ((part + 255) & ~size_t(255)) + ((flags + 255) & ~size_t(255));
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     *st = UW_OK;
     if (a.M == 0) return cudaSuccess;
+    if (a.variant < UW_VARIANT_AUTO || a.variant > UW_VARIANT_GEMV) { *st = UW_ERR_INVALID_ARG; return cudaSuccess; }
     if (gemv_serves(a)) return launch_gemv(a, s, st);
+    const GemmSplit sp = gemm_split(a.M, a.N, a.K, a.grid, a.split_k);
+    if (!sp.ok) { *st = a.split_k > 0 ? UW_ERR_INVALID_ARG : UW_ERR_SHAPE; return cudaSuccess; }
     GemmParams p{};
     p.M = a.M;
     p.N = a.N;
     p.K = a.K;
     p.KG = a.K / kGroup;
-    p.MG = pick_mg(a.M);
-    // stage k: 128 for small batch tiles (halves the per-stage TMA, barrier
-    // and MMA-issue overhead per weight byte), 64 where a stage is already
-    // large (batch tiles above 64 rows)
-    const int KB = (p.MG <= 64 && a.K % 128 == 0) ? 128 : 64;
-    p.m_tiles = (int)((a.M + p.MG - 1) / p.MG);
-    p.n_tiles = (int)((a.N + kBlockN - 1) / kBlockN);
-    p.kt_count = (int)(a.K / KB);
-    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
-    const int64_t total = tiles * p.kt_count;
-    int P = a.grid > 0 ? a.grid : gemm_default_grid();
-    // Default grid: with batch tiles of 64+ rows and no more output tiles
-    // than SMs, every tile is cut into the same whole number of k ranges,
-    // one CTA each (one CTA per tile when the tiles number half the SMs or
-    // more): each CTA then holds a single segment, instead of a tail and a
-    // head whose fix-ups move 32-128 KB of fp32 partials per cut and stall
-    // the MMA while they are written.
-    if (a.grid == 0 && p.MG >= 64 && tiles <= P) P = (int)(tiles * (P / tiles));
-    if (P > total) P = (int)total;
-    if (total * (int64_t)P >= (int64_t(1) << 32)) { *st = UW_ERR_SHAPE; return cudaSuccess; }
-    p.total_iters = (uint32_t)total;
+    p.MG = sp.MG;
+    const int KB = sp.KB;
+    p.m_tiles = sp.m_tiles;
+    p.n_tiles = sp.n_tiles;
+    p.kt_count = sp.kt;
+    const int P = sp.P;
+    p.total_iters = (uint32_t)sp.total;
     p.P = P;
     p.vbits = a.vbits;
     p.vpre = a.vpre;
@@ -820,9 +847,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
                        ((uint32_t)a.palette[4 * i + 2] << 16) | ((uint32_t)a.palette[4 * i + 3] << 24);
     p.Y = a.Y;
     p.out_f32 = a.out_f32;
-    size_t need = gemm_ws_bytes(a.M, a.N, a.K, P);
+    size_t need = gemm_ws_bytes(a.M, a.N, a.K, a.grid, a.split_k);
     if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
-    size_t part = (size_t)2 * P * p.MG * kBlockN * 4;
+    size_t part = sp.fixup ? (size_t)2 * P * p.MG * kBlockN * 4 : 0;
     p.partial = (float*)a.ws;
     p.flags = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
     p.epoch = a.epoch ? a.epoch : next_epoch();
@@ -864,6 +891,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (a.smem_cap > 0 && (size_t)a.smem_cap < budget + 2048) budget = (size_t)a.smem_cap - 2048;
     int S = (int)(budget / p.stage_bytes);
     if (S > kMaxStages) S = kMaxStages;
+    if (a.stages >= 2 && S > a.stages) S = a.stages;
     // TMEM: accumulator columns [0, MG); rebuilt-A stages of 32 columns after it
     uint32_t acc_cols = 32;
     while (acc_cols < (uint32_t)p.MG) acc_cols <<= 1;
@@ -1000,7 +1028,7 @@ extern "C" uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M
     if (!(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
     if (M == 0) return UW_OK;
     if (!X || !Y || ((uintptr_t)X & 15) || ((uintptr_t)Y & 15)) return UW_ERR_INVALID_ARG;
-    if (gemm_ws_bytes(M, b->geo.N, b->geo.K, 0) > kNoAllocScratchBytes) return UW_ERR_WORKSPACE;
+    if (gemm_ws_bytes(M, b->geo.N, b->geo.K, 0, 0) > kNoAllocScratchBytes) return UW_ERR_WORKSPACE;
     uw_status st = UW_OK;
     void* scratch = noalloc_scratch(&st);
     if (!scratch) return st;

@@ -239,7 +239,7 @@ static const void* gemv_kernel(int mb, bool xs) {
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     *st = UW_OK;
     if (a.M == 0) return cudaSuccess;
-    if (a.M > kGemvMaxM) { *st = UW_ERR_SHAPE; return cudaSuccess; }
+    if (a.M > kGemvMaxM) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     GemvParams p{};
     p.X = a.X;
     p.M = a.M;

@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -184,7 +185,7 @@ extern "C" const char* uw_status_str(int s) {
     }
 }
 
-extern "C" int uw_version(void) { return 10000; }
+extern "C" int uw_version(void) { return 10100; }
 
 extern "C" uw_status uw_last_device_status(void* stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
@@ -645,13 +646,51 @@ static bool runs_beside(const uw_gemm_opts* o) { return o->sm_dec > 0 && o->pipe
 
 static size_t band_counter_bytes(const uw_blob* b) { return al256((uint64_t)((b->geo.N + 127) / 128) * 8); }
 
-extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gemm_opts* o, size_t* bytes) {
+extern "C" uw_status uw_plan_resolve(const uw_gemm_opts* o, int64_t M, uw_gemm_opts* out) {
+    if (!o || !out || M < 0) return UW_ERR_INVALID_ARG;
+    *out = *o;
+    if (o->pipeline != UW_PIPE_AUTO) return UW_OK;
+    if (!o->plan || o->plan_entries <= 0) return UW_ERR_INVALID_ARG;
+    // exact M, else the largest tuned M below it, else the smallest tuned M
+    const uw_plan_entry* exact = nullptr, *below = nullptr, *lowest = nullptr;
+    for (int i = 0; i < o->plan_entries; i++) {
+        const uw_plan_entry& e = o->plan[i];
+        if (e.blob_index != o->projection) continue;
+        if (e.M == M && !exact) exact = &e;
+        if (e.M <= M && (!below || e.M > below->M)) below = &e;
+        if (!lowest || e.M < lowest->M) lowest = &e;
+    }
+    const uw_plan_entry* e = exact ? exact : below ? below : lowest;
+    if (!e || e->pipeline < UW_PIPE_FULL || e->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    out->pipeline = e->pipeline;
+    out->variant = e->variant;
+    out->sm_dec = e->sm_dec;
+    out->grid = e->grid;
+    out->split_k = e->split_k;
+    out->plan = nullptr;
+    out->plan_entries = 0;
+    return UW_OK;
+}
+
+static uw_status check_opts(const uw_gemm_opts* o) {
+    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (o->sm_dec < 0 || o->grid < 0 || o->split_k < 0 || o->stages < 0) return UW_ERR_INVALID_ARG;
+    if (o->variant < UW_VARIANT_AUTO || o->variant > UW_VARIANT_GEMV) return UW_ERR_INVALID_ARG;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gemm_opts* oin, size_t* bytes) {
     uw_status st = check_committed(b);
     if (st) return st;
-    if (!o || !bytes || M < 0) return UW_ERR_INVALID_ARG;
-    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (!oin || !bytes || M < 0) return UW_ERR_INVALID_ARG;
+    uw_gemm_opts ov;
+    st = uw_plan_resolve(oin, M, &ov);
+    if (st) return st;
+    const uw_gemm_opts* o = &ov;
+    st = check_opts(o);
+    if (st) return st;
     if (M == 0) { *bytes = 0; return UW_OK; }
-    *bytes = decode_buffer_bytes(b, o->pipeline) + al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid)) +
+    *bytes = decode_buffer_bytes(b, o->pipeline) + al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid, o->split_k)) +
              (runs_beside(o) ? band_counter_bytes(b) : 0);
     return UW_OK;
 }
@@ -686,18 +725,34 @@ static SideStream* side_stream(uw_status* st) {
     return &ss;
 }
 
-extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, void* Y, const uw_gemm_opts* o,
+// Test hook (UW_DEBUG_SKIP_DECODER=1): a decoder-beside-GEMM call launches
+// only its GEMM, whose bounded waits for decoded bands then run out.
+static bool debug_skip_decoder() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("UW_DEBUG_SKIP_DECODER");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, void* Y, const uw_gemm_opts* oin,
                              void* stream) {
     uw_status st = check_committed(b);
     if (st) return st;
-    if (!o || M < 0) return UW_ERR_INVALID_ARG;
-    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
-    if (o->sm_dec < 0 || o->grid < 0) return UW_ERR_INVALID_ARG;
+    if (!oin || M < 0) return UW_ERR_INVALID_ARG;
+    uw_gemm_opts ov;
+    st = uw_plan_resolve(oin, M, &ov);
+    if (st) return st;
+    const uw_gemm_opts* o = &ov;
+    st = check_opts(o);
+    if (st) return st;
     if (M == 0) return UW_OK;
     if (!X || !Y || !aligned(X, 16) || !aligned(Y, 16)) return UW_ERR_INVALID_ARG;
     const bool needs_huff = o->pipeline != UW_PIPE_DIRECT_PALETTE;
     if (needs_huff && !(b->forms & UW_FORM_HUFFMAN)) return UW_ERR_UNSUPPORTED;
     if (!needs_huff && !(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
+    if (runs_beside(o) && o->variant == UW_VARIANT_GEMV) return UW_ERR_UNSUPPORTED;
     size_t need = 0;
     uw_gemm_workspace(b, M, o, &need);
     if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
@@ -712,7 +767,10 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     a.K = b->geo.K;
     a.Y = Y;
     a.out_f32 = o->out_f32 ? 1 : 0;
+    a.variant = o->variant;
     a.grid = o->grid;
+    a.split_k = o->split_k;
+    a.stages = o->stages;
     a.ws = ws + dbuf;
     a.ws_bytes = o->workspace_bytes - dbuf;
     a.sm = b->sec(UW_SEC_SM);
@@ -751,7 +809,7 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     // The GEMM keeps room for one decoder CTA on every SM.
     SideStream* ss = side_stream(&st);
     if (!ss) return st;
-    a.ws_bytes = al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid));
+    a.ws_bytes = al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid, o->split_k));
     unsigned long long* band = (unsigned long long*)(ws + dbuf + a.ws_bytes);
     a.epoch = gemm_next_epoch();
     a.band_ready = band;
@@ -759,7 +817,8 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     a.ntasks = (b->geo.n + 8191) / 8192;
     a.smem_cap = 228 * 1024 - kDecodeBesideSmem - 2048;
     if (cuda_ok(cudaEventRecord(ss->fork, s)) || cuda_ok(cudaStreamWaitEvent(ss->s, ss->fork, 0))) return UW_ERR_CUDA;
-    if (cuda_ok(launch_decode_beside(b, mode, ws, o->sm_dec, band, a.epoch, s))) return UW_ERR_CUDA;
+    if (!debug_skip_decoder() && cuda_ok(launch_decode_beside(b, mode, ws, o->sm_dec, band, a.epoch, s)))
+        return UW_ERR_CUDA;
     cudaError_t e = launch_gemm(a, ss->s, &st);
     if (!st && e == cudaSuccess) e = cudaEventRecord(ss->join, ss->s);
     if (!st && e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
@@ -767,22 +826,27 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     return cuda_ok(e);
 }
 
-extern "C" uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int grid, size_t* bytes) {
-    if (!bytes || M < 0 || grid < 0) return UW_ERR_INVALID_ARG;
+extern "C" uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int variant, int grid, int split_k,
+                                             size_t* bytes) {
+    if (!bytes || M < 0 || grid < 0 || split_k < 0) return UW_ERR_INVALID_ARG;
+    if (variant < UW_VARIANT_AUTO || variant > UW_VARIANT_GEMV) return UW_ERR_INVALID_ARG;
     uw_status st = check_shape(N, K);
     if (st) return st;
-    *bytes = M ? gemm_ws_bytes(M, N, K, grid) : 0;
+    *bytes = M ? gemm_ws_bytes(M, N, K, grid, split_k) : 0;
     return UW_OK;
 }
 
 extern "C" uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K, void* Y,
-                                   int out_f32, int grid, void* workspace, size_t workspace_bytes, void* stream) {
-    if (M < 0 || grid < 0) return UW_ERR_INVALID_ARG;
+                                   int out_f32, int variant, int grid, int split_k, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    if (M < 0 || grid < 0 || split_k < 0) return UW_ERR_INVALID_ARG;
+    if (variant < UW_VARIANT_AUTO || variant > UW_VARIANT_GEMV) return UW_ERR_INVALID_ARG;
     uw_status st = check_shape(N, K);
     if (st) return st;
     if (M == 0) return UW_OK;
     if (!X || !W || !Y || !aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16)) return UW_ERR_INVALID_ARG;
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < gemm_ws_bytes(M, N, K, grid)) return UW_ERR_WORKSPACE;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < gemm_ws_bytes(M, N, K, grid, split_k))
+        return UW_ERR_WORKSPACE;
     GemmArgs a;
     a.src = kSrcDense;
     a.X = X;
@@ -792,7 +856,9 @@ extern "C" uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t*
     a.W = W;
     a.Y = Y;
     a.out_f32 = out_f32 ? 1 : 0;
+    a.variant = variant;
     a.grid = grid;
+    a.split_k = split_k;
     a.ws = workspace;
     a.ws_bytes = workspace_bytes;
     cudaError_t e = launch_gemm(a, (cudaStream_t)stream, &st);
@@ -803,95 +869,190 @@ extern "C" uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t*
 // ===========================================================================
 // autotune (§自動調優機制)
 // ===========================================================================
-extern "C" uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const int64_t* Ms, int nM,
+namespace {
+
+const char* kPipeNames[] = {"full", "exponent", "transcode", "direct_palette"};
+
+struct Cand {
+    int pipe, variant, grid, split_k, sm_dec;
+    bool operator==(const Cand& o) const {
+        return pipe == o.pipe && variant == o.variant && grid == o.grid && split_k == o.split_k && sm_dec == o.sm_dec;
+    }
+};
+
+uw_gemm_opts cand_opts(const Cand& c, void* ws, size_t wsb) {
+    uw_gemm_opts o{};
+    o.pipeline = c.pipe;
+    o.variant = c.variant;
+    o.grid = c.grid;
+    o.split_k = c.split_k;
+    o.sm_dec = c.sm_dec;
+    o.workspace = ws;
+    o.workspace_bytes = wsb;
+    return o;
+}
+
+// The kernel path and work split a candidate leads to, so that candidates
+// that run the same thing are measured once.
+struct PathKey {
+    int pipe, gemv, P, sm_dec;
+    bool operator==(const PathKey& o) const { return pipe == o.pipe && gemv == o.gemv && P == o.P && sm_dec == o.sm_dec; }
+};
+
+PathKey path_of(const Cand& c, const uw_blob* b, int64_t M) {
+    GemmArgs a;
+    a.M = M;
+    a.N = b->geo.N;
+    a.K = b->geo.K;
+    a.variant = c.variant;
+    a.grid = c.grid;
+    a.split_k = c.split_k;
+    const bool beside = c.sm_dec > 0 && c.pipe != UW_PIPE_DIRECT_PALETTE;
+    const bool gemv = !beside && gemv_serves(a);
+    PathKey k{c.pipe, gemv ? 1 : 0, gemv ? 0 : gemm_split(M, a.N, a.K, c.grid, c.split_k).P, beside ? c.sm_dec : 0};
+    return k;
+}
+
+// Feasible candidates of one projection at batch M, one per distinct path.
+std::vector<Cand> candidates(const uw_blob* b, int64_t M, size_t wsb) {
+    const int sms = num_sms();
+    std::vector<Cand> raw;
+    for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_DIRECT_PALETTE; pp++) {
+        raw.push_back({pp, UW_VARIANT_AUTO, 0, 0, 0});
+        if (M == 1) {
+            raw.push_back({pp, UW_VARIANT_TENSOR, 0, 0, 0});
+            raw.push_back({pp, UW_VARIANT_GEMV, 0, 0, 0});
+        }
+        raw.push_back({pp, UW_VARIANT_TENSOR, sms, 0, 0});       // stream-K over one CTA per SM
+        raw.push_back({pp, UW_VARIANT_TENSOR, 0, 1, 0});         // one CTA per output tile
+        if (pp != UW_PIPE_DIRECT_PALETTE)
+            for (int f : {1, 2, 4}) raw.push_back({pp, UW_VARIANT_AUTO, 0, 0, f * sms / 2});
+    }
+    std::vector<Cand> out;
+    std::vector<PathKey> seen;
+    for (const Cand& c : raw) {
+        const bool has = c.pipe == UW_PIPE_DIRECT_PALETTE ? (b->forms & UW_FORM_PALETTE) : (b->forms & UW_FORM_HUFFMAN);
+        if (!has) continue;
+        if (c.split_k > 0 && !gemm_split(M, b->geo.N, b->geo.K, c.grid, c.split_k).ok) continue;
+        uw_gemm_opts o = cand_opts(c, nullptr, 0);
+        size_t need = 0;
+        if (uw_gemm_workspace(b, M, &o, &need) != UW_OK || need > wsb) continue;
+        const PathKey k = path_of(c, b, M);
+        bool dup = false;
+        for (const PathKey& s : seen) dup = dup || s == k;
+        if (dup) continue;
+        seen.push_back(k);
+        out.push_back(c);
+    }
+    return out;
+}
+
+struct Trial {
+    int64_t M;
+    int round, proj;
+    Cand c;
+    double layer_us;
+};
+
+}  // namespace
+
+extern "C" uw_status uw_autotune(const uw_blob* const* blobs, int nproj, int ncopies, const int64_t* Ms, int nM,
                                  const uint16_t* const* X, void* const* Y, void* workspace, size_t workspace_bytes,
                                  int reps, uw_plan_entry* plan, const char* plan_json_path, void* stream) {
-    if (!blobs || nblobs < 1 || !Ms || nM < 1 || !X || !Y || !plan || reps < 1) return UW_ERR_INVALID_ARG;
-    for (int i = 0; i < nblobs; i++) {
-        uw_status st = check_committed(blobs[i]);
-        if (st) return st;
+    if (!blobs || nproj < 1 || ncopies < 1 || !Ms || nM < 1 || !X || !Y || !plan || reps < 1) return UW_ERR_INVALID_ARG;
+    for (int c = 0; c < ncopies; c++)
+        for (int i = 0; i < nproj; i++) {
+            const uw_blob* b = blobs[c * nproj + i];
+            uw_status st = check_committed(b);
+            if (st) return st;
+            if (b->geo.N != blobs[i]->geo.N || b->geo.K != blobs[i]->geo.K) return UW_ERR_SHAPE;
+        }
+    for (int i = 0; i < nproj; i++)
         if (!X[i] || !Y[i]) return UW_ERR_INVALID_ARG;
-    }
+    for (int m = 0; m < nM; m++)
+        if (Ms[m] < 1) return UW_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     cudaEvent_t e0, e1;
-    if (cuda_ok(cudaEventCreate(&e0)) || cuda_ok(cudaEventCreate(&e1))) return UW_ERR_CUDA;
-    struct Cand { int pipe, sm_dec; };
-    std::vector<Cand> cands;
-    for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_DIRECT_PALETTE; pp++) cands.push_back({pp, 0});
-    // decoder beside the GEMM, with a few decoder CTA counts
-    const int sms = num_sms();
-    for (int pp = UW_PIPE_FULL; pp <= UW_PIPE_TRANSCODE; pp++)
-        for (int f : {1, 2, 4}) cands.push_back({pp, f * sms / 2});
+    if (cuda_ok(cudaEventCreate(&e0))) return UW_ERR_CUDA;
+    if (cuda_ok(cudaEventCreate(&e1))) { cudaEventDestroy(e0); return UW_ERR_CUDA; }
+    // a call refused, a launch that failed, or a device status raised (a
+    // bounded wait that expired) makes the candidate infeasible
+    auto run_calls = [&](int64_t M, const std::vector<Cand>& ch, int only, int passes, int first_pass) -> bool {
+        bool ok = true;
+        for (int r = 0; r < passes; r++) {
+            const int c = (first_pass + r) % ncopies;
+            for (int i = 0; i < nproj; i++) {
+                if (only >= 0 && i != only) continue;
+                uw_gemm_opts o = cand_opts(ch[i], workspace, workspace_bytes);
+                if (uw_gemm(X[i], M, blobs[c * nproj + i], Y[i], &o, stream) != UW_OK) ok = false;
+            }
+        }
+        return ok;
+    };
+    // device time per pass (microseconds), or -1 if the candidate failed
+    auto measure = [&](int64_t M, const std::vector<Cand>& ch, int only) -> double {
+        bool ok = run_calls(M, ch, only, ncopies, 0);   // warm-up: every copy once
+        if (uw_last_device_status(stream) != UW_OK) ok = false;
+        if (!ok) return -1.0;
+        cudaEventRecord(e0, s);
+        ok = run_calls(M, ch, only, reps, 0);
+        cudaEventRecord(e1, s);
+        if (cudaEventSynchronize(e1) != cudaSuccess) { cudaGetLastError(); return -1.0; }
+        if (uw_last_device_status(stream) != UW_OK || !ok) return -1.0;
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, e0, e1);
+        return 1000.0 * ms / reps;
+    };
+    std::vector<Trial> trials;
     uw_status result = UW_OK;
     for (int mi = 0; mi < nM && result == UW_OK; mi++) {
         const int64_t M = Ms[mi];
-        // feasible candidates per projection
-        std::vector<std::vector<int>> feas(nblobs);
-        for (int i = 0; i < nblobs; i++)
-            for (int c = 0; c < (int)cands.size(); c++) {
-                uw_gemm_opts o{};
-                o.pipeline = cands[c].pipe;
-                o.sm_dec = cands[c].sm_dec;
-                size_t need = 0;
-                bool has = cands[c].pipe == UW_PIPE_DIRECT_PALETTE ? (blobs[i]->forms & UW_FORM_PALETTE)
-                                                                   : (blobs[i]->forms & UW_FORM_HUFFMAN);
-                if (has && uw_gemm_workspace(blobs[i], M, &o, &need) == UW_OK && need <= workspace_bytes)
-                    feas[i].push_back(c);
-            }
-        for (int i = 0; i < nblobs; i++)
-            if (feas[i].empty()) result = UW_ERR_WORKSPACE;
+        std::vector<std::vector<Cand>> cands(nproj);
+        for (int i = 0; i < nproj; i++) {
+            cands[i] = candidates(blobs[i], M, workspace_bytes);
+            if (cands[i].empty()) result = UW_ERR_WORKSPACE;
+        }
         if (result) break;
-        std::vector<int> choice(nblobs);
-        for (int i = 0; i < nblobs; i++) choice[i] = feas[i][0];
-        std::vector<double> per(nblobs, 0.0);
-        auto run_layer = [&](const std::vector<int>& ch, std::vector<double>* per_out) -> double {
-            double total = 0.0;
-            for (int i = 0; i < nblobs; i++) {
-                uw_gemm_opts o{};
-                o.pipeline = cands[ch[i]].pipe;
-                o.sm_dec = cands[ch[i]].sm_dec;
-                o.workspace = workspace;
-                o.workspace_bytes = workspace_bytes;
-                // warm-up
-                if (uw_gemm(X[i], M, blobs[i], Y[i], &o, stream) != UW_OK) return -1.0;
-                cudaEventRecord(e0, s);
-                for (int r = 0; r < reps; r++) uw_gemm(X[i], M, blobs[i], Y[i], &o, stream);
-                cudaEventRecord(e1, s);
-                if (cudaEventSynchronize(e1) != cudaSuccess) return -1.0;
-                float ms = 0.f;
-                cudaEventElapsedTime(&ms, e0, e1);
-                double us = 1000.0 * ms / reps;
-                if (per_out) (*per_out)[i] = us;
-                total += us;
+        // start: the first candidate that runs (pipeline 1 first, as listed)
+        std::vector<Cand> choice(nproj);
+        for (int i = 0; i < nproj; i++) choice[i] = cands[i][0];
+        double best = measure(M, choice, -1);
+        for (int i = 0; i < nproj && best < 0; i++) {
+            // the first candidates failed: take, per projection, the first that runs alone
+            for (const Cand& c : cands[i]) {
+                std::vector<Cand> t = choice;
+                t[i] = c;
+                if (measure(M, t, i) >= 0) { choice[i] = c; break; }
             }
-            return total;
-        };
-        double best = run_layer(choice, &per);
-        if (best < 0) { result = UW_ERR_CUDA; break; }
+            best = measure(M, choice, -1);
+        }
+        if (best < 0) { result = UW_ERR_DEVICE; break; }
+        for (int i = 0; i < nproj; i++) trials.push_back({M, 0, i, choice[i], best});
         for (int round = 0; round < 8; round++) {
             bool improved = false;
-            for (int i = 0; i < nblobs; i++) {
-                for (int c : feas[i]) {
+            for (int i = 0; i < nproj; i++) {
+                for (const Cand& c : cands[i]) {
                     if (c == choice[i]) continue;
-                    std::vector<int> trial = choice;
+                    std::vector<Cand> trial = choice;
                     trial[i] = c;
-                    std::vector<double> tp(nblobs, 0.0);
-                    double t = run_layer(trial, &tp);
-                    if (t < 0) { result = UW_ERR_CUDA; break; }
-                    if (t < best * 0.99) { best = t; choice = trial; per = tp; improved = true; }
+                    const double t = measure(M, trial, -1);
+                    trials.push_back({M, round, i, c, t});
+                    if (t >= 0 && t < best * 0.99) { best = t; choice = trial; improved = true; }
                 }
-                if (result) break;
             }
-            if (!improved || result) break;
+            if (!improved) break;
         }
-        for (int i = 0; i < nblobs; i++) {
-            uw_plan_entry& pe = plan[mi * nblobs + i];
+        for (int i = 0; i < nproj; i++) {
+            uw_plan_entry& pe = plan[mi * nproj + i];
             pe.blob_index = i;
             pe.M = M;
-            pe.pipeline = cands[choice[i]].pipe;
-            pe.sm_dec = cands[choice[i]].sm_dec;
-            pe.grid = 0;
-            pe.us = per[i];
+            pe.pipeline = choice[i].pipe;
+            pe.variant = choice[i].variant;
+            pe.sm_dec = choice[i].sm_dec;
+            pe.grid = choice[i].grid;
+            pe.split_k = choice[i].split_k;
+            pe.us = measure(M, choice, i);
+            pe.layer_us = best;
         }
     }
     cudaEventDestroy(e0);
@@ -899,14 +1060,106 @@ extern "C" uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const 
     if (result == UW_OK && plan_json_path) {
         FILE* f = fopen(plan_json_path, "w");
         if (!f) return UW_ERR_INVALID_ARG;
-        static const char* names[] = {"full", "exponent", "transcode", "direct_palette"};
         fprintf(f, "{\"plan\": [\n");
-        for (int k = 0; k < nM * nblobs; k++)
-            fprintf(f, "  {\"projection\": %d, \"M\": %lld, \"pipeline\": \"%s\", \"sm_dec\": %d, \"us\": %.3f}%s\n",
-                    plan[k].blob_index, (long long)plan[k].M, names[plan[k].pipeline], plan[k].sm_dec, plan[k].us,
-                    k + 1 < nM * nblobs ? "," : "");
+        for (int k = 0; k < nM * nproj; k++)
+            fprintf(f,
+                    "  {\"projection\": %d, \"M\": %lld, \"pipeline\": \"%s\", \"variant\": %d, \"sm_dec\": %d, "
+                    "\"grid\": %d, \"split_k\": %d, \"us\": %.3f, \"layer_us\": %.3f}%s\n",
+                    plan[k].blob_index, (long long)plan[k].M, kPipeNames[plan[k].pipeline], plan[k].variant,
+                    plan[k].sm_dec, plan[k].grid, plan[k].split_k, plan[k].us, plan[k].layer_us,
+                    k + 1 < nM * nproj ? "," : "");
+        fprintf(f, "],\n\"trials\": [\n");
+        for (size_t k = 0; k < trials.size(); k++) {
+            const Trial& t = trials[k];
+            fprintf(f,
+                    "  {\"M\": %lld, \"round\": %d, \"projection\": %d, \"pipeline\": \"%s\", \"variant\": %d, "
+                    "\"sm_dec\": %d, \"grid\": %d, \"split_k\": %d, \"layer_us\": %.3f}%s\n",
+                    (long long)t.M, t.round, t.proj, kPipeNames[t.c.pipe], t.c.variant, t.c.sm_dec, t.c.grid,
+                    t.c.split_k, t.layer_us, k + 1 < trials.size() ? "," : "");
+        }
         fprintf(f, "]}\n");
         fclose(f);
     }
     return result;
+}
+
+// ---------------------------------------------------------------------------
+// Reads back the "plan" array written above: objects of "key": value pairs
+// (numbers, or the pipeline's name as a string).
+// ---------------------------------------------------------------------------
+static bool json_field(const std::string& obj, const char* key, std::string* val) {
+    const std::string k = std::string("\"") + key + "\"";
+    size_t p = obj.find(k);
+    if (p == std::string::npos) return false;
+    p = obj.find(':', p + k.size());
+    if (p == std::string::npos) return false;
+    p++;
+    while (p < obj.size() && (obj[p] == ' ' || obj[p] == '\t' || obj[p] == '\n' || obj[p] == '\r')) p++;
+    if (p >= obj.size()) return false;
+    if (obj[p] == '"') {
+        size_t q = obj.find('"', p + 1);
+        if (q == std::string::npos) return false;
+        *val = obj.substr(p + 1, q - p - 1);
+        return true;
+    }
+    size_t q = p;
+    while (q < obj.size() && obj[q] != ',' && obj[q] != '}') q++;
+    *val = obj.substr(p, q - p);
+    return !val->empty();
+}
+
+extern "C" uw_status uw_plan_load_json(const char* path, uw_plan_entry* entries, int cap, int* n) {
+    if (!path || !n || cap < 0 || (cap > 0 && !entries)) return UW_ERR_INVALID_ARG;
+    FILE* f = fopen(path, "rb");
+    if (!f) return UW_ERR_INVALID_ARG;
+    std::string text;
+    char buf[4096];
+    size_t got;
+    while ((got = fread(buf, 1, sizeof buf, f)) > 0) text.append(buf, got);
+    fclose(f);
+    size_t p = text.find("\"plan\"");
+    if (p == std::string::npos) return UW_ERR_CORRUPT;
+    p = text.find('[', p);
+    if (p == std::string::npos) return UW_ERR_CORRUPT;
+    const size_t end = text.find(']', p);
+    if (end == std::string::npos) return UW_ERR_CORRUPT;
+    int count = 0;
+    for (;;) {
+        const size_t a = text.find('{', p);
+        if (a == std::string::npos || a > end) break;
+        const size_t b = text.find('}', a);
+        if (b == std::string::npos || b > end) return UW_ERR_CORRUPT;
+        const std::string obj = text.substr(a, b - a + 1);
+        uw_plan_entry e{};
+        std::string v;
+        if (!json_field(obj, "projection", &v)) return UW_ERR_CORRUPT;
+        e.blob_index = atoi(v.c_str());
+        if (!json_field(obj, "M", &v)) return UW_ERR_CORRUPT;
+        e.M = atoll(v.c_str());
+        if (!json_field(obj, "pipeline", &v)) return UW_ERR_CORRUPT;
+        e.pipeline = -1;
+        for (int k = 0; k < 4; k++)
+            if (v == kPipeNames[k]) e.pipeline = k;
+        if (e.pipeline < 0) {
+            char* q = nullptr;
+            long pv = strtol(v.c_str(), &q, 10);
+            if (q == v.c_str() || pv < UW_PIPE_FULL || pv > UW_PIPE_DIRECT_PALETTE) return UW_ERR_CORRUPT;
+            e.pipeline = (int32_t)pv;
+        }
+        if (json_field(obj, "variant", &v)) e.variant = atoi(v.c_str());
+        if (json_field(obj, "sm_dec", &v)) e.sm_dec = atoi(v.c_str());
+        if (json_field(obj, "grid", &v)) e.grid = atoi(v.c_str());
+        if (json_field(obj, "split_k", &v)) e.split_k = atoi(v.c_str());
+        if (json_field(obj, "us", &v)) e.us = atof(v.c_str());
+        if (json_field(obj, "layer_us", &v)) e.layer_us = atof(v.c_str());
+        if (e.M < 1 || e.blob_index < 0 || e.variant < UW_VARIANT_AUTO || e.variant > UW_VARIANT_GEMV || e.sm_dec < 0 ||
+            e.grid < 0 || e.split_k < 0)
+            return UW_ERR_CORRUPT;
+        if (count < cap) entries[count] = e;
+        count++;
+        p = b + 1;
+    }
+    if (count == 0) return UW_ERR_CORRUPT;
+    *n = count;
+    return UW_OK;
 }

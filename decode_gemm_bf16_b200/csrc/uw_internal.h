@@ -132,7 +132,10 @@ struct GemmArgs {
     const uint8_t* palette = nullptr; // host array of 16
     void* Y = nullptr;
     int out_f32 = 0;
+    int variant = UW_VARIANT_AUTO;
     int grid = 0;
+    int split_k = 0;                  // >0: k ranges per output tile (grid ignored)
+    int stages = 0;                   // >0: cap on the stage ring depth
     void* ws = nullptr;               // partial sums + tile counters
     size_t ws_bytes = 0;
     int smem_cap = 0;                 // >0: dynamic shared memory limit (room for a decoder CTA)
@@ -142,10 +145,20 @@ struct GemmArgs {
     int static_sm = 0;                // sm plane and verbatim flags read from the committed blob (no kernel writes it)
     int static_s2 = 0;                // second plane too (the stored index plane)
 };
-size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid);
-// Tensor-core GEMM; the shapes gemv_serves() accepts (batch 1 on a
-// projection with few 128-row tiles, no decoder beside) go to the CUDA-core
-// GEMV instead.
+// Work split of the tensor-core kernel: batch tile MG, stage k KB, tiles,
+// (tile, k step) iterations and CTA count P.  fixup: some tile is cut
+// between CTAs (partial sums and tags in the workspace).  ok = false when the
+// options are inconsistent (split_k >= 2 with more CTAs than SMs).
+struct GemmSplit {
+    int MG = 16, KB = 64, m_tiles = 0, n_tiles = 0, kt = 0, P = 0;
+    int64_t tiles = 0, total = 0;
+    bool fixup = false, ok = true;
+};
+GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k);
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k);
+// Tensor-core GEMM; the calls gemv_serves() accepts (by the variant, or with
+// UW_VARIANT_AUTO batch 1 on a projection with few 128-row tiles and no
+// decoder beside) go to the CUDA-core GEMV instead.
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st);
 bool gemv_serves(const GemmArgs& a);
 constexpr int kGemvMaxM = 1;   // batches the GEMV kernel supports

@@ -56,13 +56,24 @@ typedef enum {
     UW_ERR_DEVICE = 8        /* a device-side check failed (bad stream data)  */
 } uw_status;
 
-/* The four pipelines of §四種執行管道. */
+/* The four pipelines of §四種執行管道, and the autotuned choice of
+ * §自動調優機制 (UW_PIPE_AUTO: the plan given in the options picks the
+ * pipeline and matmul settings for this projection and batch size). */
 typedef enum {
+    UW_PIPE_AUTO = -1,           /* resolved through uw_gemm_opts.plan (see uw_plan_resolve)  */
     UW_PIPE_FULL = 0,            /* Huffman full decode -> BF16 W in workspace -> dense GEMM  */
     UW_PIPE_EXPONENT = 1,        /* Huffman exponent decode -> E in workspace -> reconstructive GEMM */
     UW_PIPE_TRANSCODE = 2,       /* Huffman -> 4-bit index plane in workspace -> reconstructive GEMM */
     UW_PIPE_DIRECT_PALETTE = 3   /* reconstructive GEMM straight from the stored index plane */
 } uw_pipeline;
+
+/* Matmul variant: which kernel family computes the product. */
+typedef enum {
+    UW_VARIANT_AUTO = 0,     /* batch 1 on a projection with fewer than grid/2 tiles of 128 rows
+                                runs the CUDA-core GEMV, everything else the tensor cores      */
+    UW_VARIANT_TENSOR = 1,   /* tcgen05 tensor-core kernel at every batch size                 */
+    UW_VARIANT_GEMV = 2      /* CUDA-core GEMV (batch 1 only; other batches: UW_ERR_UNSUPPORTED) */
+} uw_variant;
 
 /* Forms a compressed matrix may hold (bit mask). */
 enum { UW_FORM_HUFFMAN = 1, UW_FORM_PALETTE = 2 };
@@ -105,6 +116,20 @@ typedef struct {
     uint64_t section_bytes[UW_NSECT];   /* byte length (0 = absent)                    */
 } uw_blob_info;
 
+/* One autotuner decision (§自動調優機制): the configuration chosen for one
+ * projection and one batch size. */
+typedef struct {
+    int32_t blob_index;      /* which projection (its index in the autotuner's blobs)     */
+    int64_t M;               /* batch size                                                */
+    int32_t pipeline;        /* chosen uw_pipeline (never UW_PIPE_AUTO)                   */
+    int32_t variant;         /* chosen uw_variant                                         */
+    int32_t sm_dec;          /* chosen decoder SM count (0: decode, then GEMM)            */
+    int32_t grid;            /* chosen tensor-core CTA count (0: default rule)            */
+    int32_t split_k;         /* chosen k ranges per output tile (0: default rule)         */
+    double us;               /* measured time of this projection alone, microseconds      */
+    double layer_us;         /* measured time of the whole sequence of projections        */
+} uw_plan_entry;
+
 typedef struct {
     int32_t pipeline;        /* uw_pipeline                                               */
     int32_t sm_dec;          /* >0: the Huffman decoder runs on sm_dec SMs beside the GEMM
@@ -112,23 +137,22 @@ typedef struct {
     int32_t grid;            /* tensor-core GEMM CTAs; 0 = one per SM, or, when batch
                                 tiles have 64+ rows and there are no more output tiles than
                                 SMs, the largest whole multiple of the tile count that
-                                fits.  It also decides whether batch 1 runs the CUDA-core
-                                GEMV (see uw_gemm)                                         */
+                                fits.  With UW_VARIANT_AUTO it also decides whether batch 1
+                                runs the CUDA-core GEMV (see uw_gemm)                      */
     int32_t out_f32;         /* 0: Y is BF16 (round to nearest even); 1: Y is float32      */
+    int32_t variant;         /* uw_variant                                                 */
+    int32_t split_k;         /* 0: grid decides; >0: every output tile is cut into split_k
+                                k ranges (at most its k steps), one CTA each, grid ignored.
+                                split_k >= 2 needs tiles * split_k <= SMs (else
+                                UW_ERR_INVALID_ARG)                                        */
+    int32_t stages;          /* 0: the deepest stage ring that fits; >= 2: at most this many */
+    int32_t projection;      /* UW_PIPE_AUTO: the projection index looked up in `plan`     */
+    const uw_plan_entry* plan;   /* UW_PIPE_AUTO: the autotuner's entries (host memory)    */
+    int32_t plan_entries;
     void* workspace;         /* device, 256-byte aligned, any contents; a call owns it
                                 until it completes (one workspace per stream)              */
     size_t workspace_bytes;
 } uw_gemm_opts;
-
-/* One autotuner decision: best configuration for one projection and batch. */
-typedef struct {
-    int32_t blob_index;      /* which projection (index into the blobs array)  */
-    int64_t M;               /* batch size                                     */
-    int32_t pipeline;        /* chosen uw_pipeline                             */
-    int32_t sm_dec;          /* chosen decoder SM count                        */
-    int32_t grid;            /* chosen GEMM CTA count                          */
-    double us;               /* measured time of this projection, microseconds */
-} uw_plan_entry;
 
 /* ---------------------------------------------------------------- misc */
 
@@ -211,12 +235,18 @@ uw_status uw_transcode_palette(const uw_blob* blob, uint8_t* idx_out, void* stre
  * Y[M,N] = X[M,K] . W^T with W given compressed (§重建矩陣乘法核心運作).
  * X: device BF16 [M,K], 16-byte aligned; Y: device [M,N] BF16 or float32.
  * M = 0 is a no-op.  Accumulation is float32 on the tensor cores, except
- * for M = 1 on a projection with fewer than grid/2 tiles of 128 rows (grid:
- * the GEMM CTA count, one per SM by default) and sm_dec = 0: that runs on
- * the CUDA cores (a GEMV that rebuilds the weights in registers).  The
- * choice depends on the shape only, so all pipelines and uw_dense_gemm take
- * the same summation order for a given M, N, K and grid and agree bit for
- * bit.
+ * with UW_VARIANT_GEMV, or with UW_VARIANT_AUTO for M = 1 on a projection
+ * with fewer than grid/2 tiles of 128 rows (grid: the GEMM CTA count, one
+ * per SM by default) and sm_dec = 0: those run on the CUDA cores (a GEMV that
+ * rebuilds the weights in registers).  The choice depends on the shape and
+ * options only, so all pipelines and uw_dense_gemm take the same summation
+ * order for a given M, N, K, variant, grid and split_k and agree bit for bit.
+ * Every device-side wait is bounded: UW_TIMEOUT_MS (environment, read once,
+ * default 2000, at least 10) milliseconds, after which the kernel raises
+ * UW_ERR_TIMEOUT in the device status word and returns.  For tests of that
+ * path, UW_DEBUG_SKIP_DECODER=1 (environment, read once) makes a
+ * decoder-beside-GEMM call (sm_dec > 0) launch its GEMM without the decoder,
+ * so the GEMM's waits for decoded bands run out.
  * Kernels are launched with programmatic dependent launch.  The direct-palette
  * pipeline requests its first weight tiles from the blob's device image
  * before waiting for the preceding kernel on the stream to finish, so that
@@ -224,19 +254,29 @@ uw_status uw_transcode_palette(const uw_blob* blob, uint8_t* idx_out, void* stre
  * the call is enqueued (the library never writes a committed blob; ordinary
  * kernels and copies finish before a dependent kernel starts). */
 
-/* Workspace bytes for uw_gemm with these options and M. */
+/* Workspace bytes for uw_gemm with these options and M (UW_PIPE_AUTO: for the
+ * plan's choice). */
 uw_status uw_gemm_workspace(const uw_blob* blob, int64_t M, const uw_gemm_opts* opts, size_t* bytes);
+
+/* UW_PIPE_AUTO lookup: copies into *out the options the plan gives for
+ * (opts->projection, M) -- the entry of that projection with exactly M, else
+ * the largest tuned M below it, else the smallest tuned M -- keeping out_f32,
+ * workspace and stages from opts.  A concrete pipeline is copied unchanged.
+ * UW_ERR_INVALID_ARG when the plan has no entry for the projection. */
+uw_status uw_plan_resolve(const uw_gemm_opts* opts, int64_t M, uw_gemm_opts* out);
 
 uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* blob, void* Y,
                   const uw_gemm_opts* opts, void* stream);
 
 /* The uncompressed baseline: the same GEMM (tensor cores, or the GEMV where
- * uw_gemm would use it) on a plain BF16 W. */
-uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int grid, size_t* bytes);
+ * uw_gemm would use it) on a plain BF16 W.  variant, grid and split_k as in
+ * uw_gemm_opts. */
+uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int variant, int grid, int split_k,
+                                  size_t* bytes);
 
 uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K,
-                        void* Y, int out_f32, int grid, void* workspace, size_t workspace_bytes,
-                        void* stream);
+                        void* Y, int out_f32, int variant, int grid, int split_k, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------- allocation-free GEMM
  * An addition of this library; the pages have no counterpart.
@@ -261,20 +301,41 @@ uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M, const uw_
                                          int out_f32, void* stream);
 
 /* ---------------------------------------------------------------- autotune
- * §自動調優機制: coordinate descent over (pipeline, sm_dec) for each
- * projection, timing the whole sequence of projections with CUDA events:
- * sweep projection 0 with the others fixed, then 1, then 2, ..., and repeat
- * until a full round brings no improvement.  Done once per batch size in Ms.
- *   blobs[i], X[i], Y[i]: projection i and device buffers for its input
- *     (at least max(Ms) x K_i) and output (max(Ms) x N_i, BF16);
- *   workspace: at least the largest uw_gemm_workspace over the candidates;
- *   plan_out: nblobs * nM entries, written in (M, projection) order;
- *   plan_json_path: if not NULL, the plan is also written there as JSON.
+ * §自動調優機制: a measured coordinate descent.  For each batch size in Ms:
+ * start every projection at the first feasible candidate, then sweep the
+ * candidates of projection 0 with the others fixed, then 1, then 2, ..., and
+ * repeat until a full round brings no improvement of more than 1%.  The cost
+ * of a configuration is the device time (CUDA events) of the whole sequence
+ * of projections, run `reps` times; pass r uses copy r % ncopies of every
+ * projection, so with enough copies no weight is still in L2 from the pass
+ * before.  Candidates: the four pipelines (those the blob's forms allow), the
+ * matmul variants (batch 1: GEMV or tensor cores), an alternative grid (one
+ * CTA per SM instead of the default rule) and, for the decoding pipelines,
+ * decoder CTAs beside the GEMM (sm_dec = SMs/2, SMs, 2 SMs).  A candidate
+ * whose call fails or whose kernels raise the device status (a bounded wait
+ * that expired) counts as infeasible.
+ *   blobs[c * nproj + i]: copy c of projection i (copies of one projection
+ *     have the same shape); X[i], Y[i]: device buffers for the input (at
+ *     least max(Ms) x K_i, BF16) and output (max(Ms) x N_i, BF16);
+ *   workspace: at least the largest uw_gemm_workspace over the candidates
+ *     (candidates that need more are skipped);
+ *   plan_out: nproj * nM entries, written in (M, projection) order, each with
+ *     the projection's own time (measured alone over the copies) and the
+ *     whole sequence's time;
+ *   plan_json_path: if not NULL, the plan is written there as JSON, with
+ *     every measured trial ("trials": M, round, projection, candidate, time),
+ *     and can be read back with uw_plan_load_json.
  * Synchronizes `stream`. */
-uw_status uw_autotune(const uw_blob* const* blobs, int nblobs, const int64_t* Ms, int nM,
+uw_status uw_autotune(const uw_blob* const* blobs, int nproj, int ncopies, const int64_t* Ms, int nM,
                       const uint16_t* const* X, void* const* Y, void* workspace,
                       size_t workspace_bytes, int reps, uw_plan_entry* plan_out,
                       const char* plan_json_path, void* stream);
+
+/* Reads the "plan" entries of a JSON file written by uw_autotune (the
+ * per-model configuration file of §自動調優機制).  *n = entries found; at
+ * most `cap` are stored.  UW_ERR_CORRUPT if the file holds no plan or an entry
+ * lacks a field; UW_ERR_INVALID_ARG if it cannot be opened. */
+uw_status uw_plan_load_json(const char* path, uw_plan_entry* entries, int cap, int* n);
 
 #ifdef __cplusplus
 }

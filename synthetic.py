@@ -1,10 +1,12 @@
 """Seeded synthetic inputs shared by the tests, the smoke check and the bench.
 
 This module holds random-number recipes only -- none of the compression or
-product arithmetic.  Everything is drawn on the host with a CPU
-``torch.Generator`` so that the CPU oracle and the GPU library see identical
-BF16 bit patterns; arrays come back as numpy ``uint16`` bit patterns
-(row-major) so that neither side depends on the other's tensor types.
+product arithmetic.  The inputs of tests and the smoke check are drawn on the
+host with a CPU ``torch.Generator`` so that the CPU oracle and the GPU
+library see identical BF16 bit patterns; arrays come back as numpy
+``uint16`` bit patterns (row-major) so that neither side depends on the
+other's tensor types.  The benchmark's 32-layer stack is drawn on the device
+(same distributions, a CUDA generator; see the end of the file).
 
 The shapes stand in for the Llama-3.1-8B MLP projections that the Unweight
 pages measure on (gate/up ``[14336, 4096]``, down ``[4096, 14336]``); those
@@ -124,3 +126,46 @@ def stack_layer(layer: int):
     return (weight_with_tail(14336, 4096, base, sd),
             weight_with_tail(14336, 4096, base + 1, sd),
             weight_with_tail(4096, 14336, base + 2, sd))
+
+
+# --------------------------------------------------------------------------
+# Device-side draws for the benchmark's 32-layer stack (5.6 G weights): the
+# same distributions as weight_with_tail, drawn with a CUDA torch.Generator
+# so that generating the stack takes seconds instead of minutes.  The bits
+# differ from the host recipe; anything that compares against the oracle
+# copies the device bits back to the host first.
+# --------------------------------------------------------------------------
+def _gen_cuda(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def weight_with_tail_device(N: int, K: int, seed: int, device, std: float = 0.02, frac: float = 0.001) -> torch.Tensor:
+    """Device BF16 W[N, K] ~ N(0, std) with a fraction `frac` of the elements
+    (seeded distinct positions) replaced by std * t_3."""
+    g = _gen_cuda(seed, device)
+    w = torch.randn(N * K, generator=g, dtype=torch.float32, device=device) * std
+    cnt = int(round(frac * N * K))
+    if cnt:
+        pos = torch.randperm(N * K, generator=g, device=device)[:cnt]
+        z = torch.randn(cnt, generator=g, dtype=torch.float64, device=device)
+        c = torch.randn(3, cnt, generator=g, dtype=torch.float64, device=device).pow(2).sum(0)
+        w[pos] = std * (z / torch.sqrt(c / 3.0)).to(torch.float32)
+    return w.view(N, K).to(torch.bfloat16)
+
+
+def stack_layer_device(layer: int, device):
+    """Layer `layer` of the 32-layer stack drawn on the device: (gate, up,
+    down) BF16 tensors with that layer's std, seeds 1000 + 3*layer (+0, +1, +2)."""
+    sd = float(layer_stds()[layer])
+    base = 1000 + 3 * layer
+    return (weight_with_tail_device(14336, 4096, base, device, sd),
+            weight_with_tail_device(14336, 4096, base + 1, device, sd),
+            weight_with_tail_device(4096, 14336, base + 2, device, sd))
+
+
+def activations_device(M: int, K: int, seed: int, device) -> torch.Tensor:
+    """Device BF16 X[M, K] ~ N(0, 1)."""
+    g = _gen_cuda(seed, device)
+    return torch.randn(M, K, generator=g, dtype=torch.float32, device=device).to(torch.bfloat16)

@@ -58,9 +58,13 @@ def test_shape_validation_on_host(L):
     assert L.uw_compress_scratch_bytes(0, 64, ctypes.byref(n)) == 2         # empty N
     assert L.uw_compress_scratch_bytes(1 << 20, 1 << 12, ctypes.byref(n)) == 2   # > 2^31 elements
     assert L.uw_compress_scratch_bytes((1 << 31) // 4096 - 1, 4096, ctypes.byref(n)) == 0
-    assert L.uw_dense_gemm_workspace(4, 512, 2048, 0, ctypes.byref(n)) == 0
-    assert L.uw_dense_gemm_workspace(0, 512, 2048, 0, ctypes.byref(n)) == 0 and n.value == 0
-    assert L.uw_dense_gemm_workspace(4, 512, 96, 0, ctypes.byref(n)) == 2
+    assert L.uw_dense_gemm_workspace(4, 512, 2048, 0, 0, 0, ctypes.byref(n)) == 0
+    assert L.uw_dense_gemm_workspace(0, 512, 2048, 0, 0, 0, ctypes.byref(n)) == 0 and n.value == 0
+    assert L.uw_dense_gemm_workspace(4, 512, 96, 0, 0, 0, ctypes.byref(n)) == 2
+    assert L.uw_dense_gemm_workspace(4, 512, 2048, 3, 0, 0, ctypes.byref(n)) == 1       # no such variant
+    assert L.uw_dense_gemm_workspace(4, 512, 2048, 0, 0, -1, ctypes.byref(n)) == 1      # negative split
+    # one CTA per output tile: no fix-up scratch beyond the minimum
+    assert L.uw_dense_gemm_workspace(1024, 14336, 4096, 0, 0, 1, ctypes.byref(n)) == 0 and n.value == 256
     # null pointers are rejected before any device work
     h = ctypes.c_void_p()
     db = ctypes.c_size_t()
@@ -147,3 +151,71 @@ def test_code_hash_ignores_comments_only():
     assert len(B.code_hash()) == 64
     assert B.kernel_code_hash("k_decode<full>") == B.code_hash("uw_decode.cu")
     assert B.kernel_code_hash("k_gemm_recon<palette>") != B.kernel_code_hash("k_decode<full>")
+
+
+# -------- autotuned plans (§自動調優機制): file format and UW_PIPE_AUTO lookup
+def _write_plan(path, entries):
+    import json
+    with open(path, "w") as f:
+        json.dump({"plan": entries, "trials": []}, f)
+
+
+def test_plan_json_round_trip_and_resolve(L, tmp_path):
+    entries = [dict(projection=0, M=1, pipeline="direct_palette", variant=2, sm_dec=0, grid=0, split_k=0, us=25.0,
+                    layer_us=80.0),
+               dict(projection=0, M=64, pipeline="exponent", variant=0, sm_dec=74, grid=0, split_k=0, us=30.0,
+                    layer_us=90.0),
+               dict(projection=1, M=8, pipeline="transcode", variant=1, sm_dec=0, grid=148, split_k=0, us=40.0,
+                    layer_us=90.0),
+               dict(projection=1, M=256, pipeline="full", variant=0, sm_dec=0, grid=0, split_k=1, us=50.0,
+                    layer_us=100.0)]
+    path = str(tmp_path / "plan.json")
+    _write_plan(path, entries)
+    got = uw.uw_plan_load_json(path)
+    assert [(e["projection"], e["M"], e["pipeline"], e["variant"], e["sm_dec"], e["grid"], e["split_k"])
+            for e in got] == [(e["projection"], e["M"], e["pipeline"], e["variant"], e["sm_dec"], e["grid"],
+                               e["split_k"]) for e in entries]
+    plan = uw.Plan(got)
+    # exact M; the largest tuned M below; the smallest tuned M when none is below
+    assert uw.uw_plan_resolve(plan, 0, 1)["pipeline"] == "direct_palette"
+    assert uw.uw_plan_resolve(plan, 0, 1)["variant"] == 2
+    r = uw.uw_plan_resolve(plan, 0, 1000)
+    assert r["pipeline"] == "exponent" and r["sm_dec"] == 74
+    assert uw.uw_plan_resolve(plan, 0, 63)["pipeline"] == "direct_palette"
+    assert uw.uw_plan_resolve(plan, 1, 1)["pipeline"] == "transcode"
+    assert uw.uw_plan_resolve(plan, 1, 1)["grid"] == 148
+    r = uw.uw_plan_resolve(plan, 1, 4096)
+    assert r["pipeline"] == "full" and r["split_k"] == 1
+    # a projection the plan does not cover
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_plan_resolve(plan, 2, 1)
+    assert ei.value.status == 1
+
+
+def test_plan_resolve_passes_concrete_pipelines_through(L):
+    o = uw._opts("transcode", sm_dec=5, grid=7, out_f32=True, variant="tensor", split_k=3, stages=4)
+    r = uw.GemmOpts()
+    assert L.uw_plan_resolve(ctypes.byref(o), 16, ctypes.byref(r)) == 0
+    assert (r.pipeline, r.sm_dec, r.grid, r.out_f32, r.variant, r.split_k, r.stages) == (2, 5, 7, 1, 1, 3, 4)
+    # AUTO without a plan
+    o = uw._opts("auto")
+    assert L.uw_plan_resolve(ctypes.byref(o), 16, ctypes.byref(r)) == 1
+
+
+def test_plan_json_rejects_bad_files(L, tmp_path):
+    bad = tmp_path / "bad.json"
+    bad.write_text('{"nothing": []}')
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_plan_load_json(str(bad))
+    assert ei.value.status == 3
+    bad.write_text('{"plan": [{"projection": 0, "pipeline": "full"}]}')       # no M
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_plan_load_json(str(bad))
+    assert ei.value.status == 3
+    bad.write_text('{"plan": [{"projection": 0, "M": 4, "pipeline": "huffman"}]}')   # unknown pipeline
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_plan_load_json(str(bad))
+    assert ei.value.status == 3
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_plan_load_json(str(tmp_path / "missing.json"))
+    assert ei.value.status == 1

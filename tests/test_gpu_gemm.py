@@ -13,7 +13,7 @@ import torch
 import decode_gemm_bf16_b200 as uw
 import synthetic as S
 from oracle import oracle as O
-from tests.gpu_util import check_gemm, dev16, host16
+from tests.gpu_util import check_gemm, dev16, host16, oracle_gemm
 
 pytestmark = pytest.mark.gpu
 
@@ -122,22 +122,10 @@ def _sampled(X, W, Y, n_samples, seed, bf16_out):
     check_gemm(Y[ms, ns], ref, bf16_out=bf16_out)
 
 
-@pytest.mark.parametrize("M", [1, 64])
-def test_full_size_gate_sampled(M):
+@pytest.fixture(scope="module")
+def gate_case():
     W = S.gate_projection()
-    blob = uw.uw_compress(dev16(W))
-    X = S.activations(M, 4096, seed=1 + S.X_SEED_OFFSET)
-    Xd = dev16(X)
-    ref = None
-    for pipe in PIPES:
-        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
-        _sampled(X, W, Y, 256, seed=M, bf16_out=True)
-        if ref is None:
-            ref = Y
-        assert np.array_equal(Y, ref), pipe
-    Yd = _f32(uw.uw_dense_gemm(Xd, dev16(W)))
-    assert np.array_equal(Yd, ref)
-    assert uw.uw_last_device_status() == 0
+    return W, uw.uw_compress(dev16(W))
 
 
 @pytest.fixture(scope="module")
@@ -146,34 +134,51 @@ def down_case():
     return W, uw.uw_compress(dev16(W))
 
 
-def test_full_size_down_sampled(down_case):
-    W, blob = down_case
-    X = S.activations(256, 14336, seed=4 + S.X_SEED_OFFSET)
+def _full_size_all_paths(W, blob, M, seed):
+    """Every output of the four pipelines and the dense baseline, BF16 and
+    float32 outputs, against the oracle's fp32-accumulated product."""
+    X = S.activations(M, W.shape[1], seed=seed)
+    R = oracle_gemm(X, W, "f32")
     Xd = dev16(X)
-    for pipe in ["exponent", "direct_palette"]:
-        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
-        _sampled(X, W, Y, 128, seed=3, bf16_out=True)
+    ref = None
+    for pipe in PIPES:
+        Yb = _f32(uw.uw_gemm(Xd, blob, pipe))
+        check_gemm(Yb, R, bf16_out=True)
+        if ref is None:
+            ref = Yb
+        assert np.array_equal(Yb, ref), pipe
+    check_gemm(_f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True)), R, bf16_out=False)
+    Wd = dev16(W)
+    Yd = _f32(uw.uw_dense_gemm(Xd, Wd))
+    check_gemm(Yd, R, bf16_out=True)
+    assert np.array_equal(Yd, ref)
+    check_gemm(_f32(uw.uw_dense_gemm(Xd, Wd, out_f32=True)), R, bf16_out=False)
     assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 64, 1024])
+def test_full_size_gate_every_output(gate_case, M):
+    """Gate projection W[14336,4096] at batch 1 (tensor cores, stream-K over
+    the 112 row tiles), 64 (one CTA per tile) and 1024 (stream-K over 448
+    tiles): every output element of every path against the oracle."""
+    W, blob = gate_case
+    _full_size_all_paths(W, blob, M, seed=1 + S.X_SEED_OFFSET + M)
+
+
+@pytest.mark.parametrize("M", [256, 1024])
+def test_full_size_down_every_output(down_case, M):
+    """Down projection W[4096,14336] (32 row tiles, K = 14336) at batch 256
+    (four CTAs per tile) and 1024 (one CTA per tile, 128 tiles)."""
+    W, blob = down_case
+    _full_size_all_paths(W, blob, M, seed=4 + S.X_SEED_OFFSET + M)
 
 
 @pytest.mark.parametrize("M", [1, 16])
 def test_full_size_down_small_batch(down_case, M):
-    """Down projection (32 row tiles, K = 14336) at batch 1 (the CUDA-core
-    GEMV serves it) and 16 (tensor cores, 128-k stages, each tile cut ~4-5
-    ways): every pipeline and the dense baseline agree bit for bit and match
-    sampled oracle outputs."""
+    """Down projection at batch 1 (the CUDA-core GEMV serves it) and 16
+    (tensor cores, 128-k stages, each tile cut ~4-5 ways): every output."""
     W, blob = down_case
-    X = S.activations(M, 14336, seed=40 + M)
-    Xd = dev16(X)
-    ref = None
-    for pipe in PIPES:
-        Y = _f32(uw.uw_gemm(Xd, blob, pipe))
-        if ref is None:
-            ref = Y
-            _sampled(X, W, Y, 128, seed=M, bf16_out=True)
-        assert np.array_equal(Y, ref), pipe
-    assert np.array_equal(_f32(uw.uw_dense_gemm(Xd, dev16(W))), ref)
-    assert uw.uw_last_device_status() == 0
+    _full_size_all_paths(W, blob, M, seed=40 + M)
 
 
 @pytest.mark.parametrize("fill", [0x00, 0xFF, "random"])
@@ -216,9 +221,8 @@ def test_decoder_beside_gemm(pipe, sm_dec):
     assert uw.uw_last_device_status() == 0
 
 
-def test_decoder_beside_gemm_full_size():
-    W = S.gate_projection()
-    blob = uw.uw_compress(dev16(W))
+def test_decoder_beside_gemm_full_size(gate_case):
+    W, blob = gate_case
     X = S.activations(16, 4096, seed=12)
     Xd = dev16(X)
     for pipe in ["exponent", "transcode"]:
@@ -230,25 +234,155 @@ def test_decoder_beside_gemm_full_size():
 
 
 def test_autotune_plan(tmp_path):
-    """The autotuner returns one feasible, measured choice per projection
-    and batch size and writes the plan as JSON."""
+    """The autotuner (§自動調優機制) over two copies of a three-projection
+    layer: one entry per projection and batch, each the measured minimum of
+    its candidates in the last round of the descent (within the 1% it
+    requires before it moves), the plan file reads back, and UW_PIPE_AUTO
+    under the plan matches the oracle."""
     import json
     shapes = [(384, 512), (384, 512), (512, 384 + 128)]
     Ws = [S.gaussian_weight(n, k, seed=60 + i) for i, (n, k) in enumerate(shapes)]
-    blobs = [uw.uw_compress(dev16(w)) for w in Ws]
+    copies = 2
+    blobs = [uw.uw_compress(dev16(w)) for _ in range(copies) for w in Ws]
     Ms = [1, 64]
-    Xs = [dev16(S.activations(max(Ms), k, seed=70 + i)) for i, (n, k) in enumerate(shapes)]
+    Xh = [S.activations(max(Ms), k, seed=70 + i) for i, (n, k) in enumerate(shapes)]
+    Xs = [dev16(x) for x in Xh]
     Ys = [torch.empty(max(Ms), n, dtype=torch.bfloat16, device="cuda") for (n, k) in shapes]
-    need = max(uw.uw_gemm_workspace(b, max(Ms), p, sm_dec=sd) for b in blobs
+    need = max(uw.uw_gemm_workspace(b, max(Ms), p, sm_dec=sd) for b in blobs[:3]
                for p in PIPES for sd in (0, 300))
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     path = str(tmp_path / "plan.json")
-    plan = uw.uw_autotune(blobs, Ms, Xs, Ys, ws, reps=3, plan_json_path=path)
-    assert len(plan) == len(Ms) * len(blobs)
+    plan = uw.uw_autotune(blobs, Ms, Xs, Ys, ws, reps=3, plan_json_path=path, copies=copies)
+    assert len(plan) == len(Ms) * len(shapes)
     for i, e in enumerate(plan):
         assert e["M"] == Ms[i // 3] and e["projection"] == i % 3
-        assert e["pipeline"] in PIPES and e["us"] > 0
-    saved = json.load(open(path))["plan"]
-    assert [(d["projection"], d["M"], d["pipeline"]) for d in saved] == \
+        assert e["pipeline"] in PIPES and e["us"] > 0 and e["layer_us"] > 0
+    saved = json.load(open(path))
+    assert [(d["projection"], d["M"], d["pipeline"], d["variant"], d["sm_dec"], d["grid"], d["split_k"])
+            for d in saved["plan"]] == [(e["projection"], e["M"], e["pipeline"], e["variant"], e["sm_dec"],
+                                         e["grid"], e["split_k"]) for e in plan]
+    trials = saved["trials"]
+    for M in Ms:
+        last = max(t["round"] for t in trials if t["M"] == M)
+        chosen = {e["projection"]: e for e in plan if e["M"] == M}
+        for proj in range(3):
+            ts = [t for t in trials if t["M"] == M and t["round"] == last and t["projection"] == proj
+                  and t["layer_us"] > 0]
+            # no candidate of the last round beat the chosen configuration by 1%
+            assert all(t["layer_us"] >= 0.99 * chosen[proj]["layer_us"] for t in ts), (M, proj)
+            assert len(ts) >= 1
+    # the plan file is the per-model configuration: read it back and run AUTO
+    loaded = uw.uw_plan_load_json(path)
+    assert [(e["projection"], e["M"], e["pipeline"]) for e in loaded] == \
         [(e["projection"], e["M"], e["pipeline"]) for e in plan]
+    P = uw.Plan(loaded)
+    for M in [1, 5, 64, 100]:
+        for proj, (n, k) in enumerate(shapes):
+            X = Xh[proj][:M]
+            Y = uw.uw_gemm(dev16(X), blobs[proj], "auto", plan=P, projection=proj)
+            check_gemm(_f32(Y), O.gemm(X, Ws[proj], "f32"), bf16_out=True)
     assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("variant", ["tensor", "gemv"])
+def test_variant_forced_at_batch_one(variant):
+    """Batch 1 forced onto the tensor cores or onto the CUDA-core GEMV: each
+    matches the oracle, and all pipelines agree bit for bit within a variant."""
+    W, blob = _case("384x512")
+    X = S.activations(1, 512, seed=91)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    ref = None
+    for pipe in PIPES:
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True, variant=variant))
+        check_gemm(Y, R, bf16_out=False)
+        if ref is None:
+            ref = Y
+        assert np.array_equal(Y, ref), pipe
+    assert np.array_equal(_f32(uw.uw_dense_gemm(Xd, dev16(W), out_f32=True, variant=variant)), ref)
+    # the GEMV serves batch 1 only
+    if variant == "gemv":
+        with pytest.raises(uw.UnweightError) as ei:
+            uw.uw_gemm(dev16(S.activations(2, 512, seed=92)), blob, "direct_palette", variant="gemv")
+        assert ei.value.status == 4
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("split_k", [1, 2, 3, 8])
+@pytest.mark.parametrize("M", [5, 64, 200])
+def test_split_k_and_stages(split_k, M):
+    """Every output tile cut into split_k k ranges (one CTA each), with the
+    ring held to two stages: matches the oracle, pipelines agree."""
+    W, blob = _case("200x1408")
+    X = S.activations(M, 1408, seed=93 + M)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    ref = None
+    for pipe in PIPES:
+        for stages in (0, 2):
+            Y = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True, split_k=split_k, stages=stages))
+            check_gemm(Y, R, bf16_out=False)
+            if ref is None:
+                ref = Y
+            assert np.array_equal(Y, ref), (pipe, stages)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_default_grid_uneven_k_ranges():
+    """The default grid with 64-row batch tiles and fewer tiles than SMs cuts
+    every tile into floor(SMs / tiles) k ranges: N = 1024 gives 8 tiles, so
+    18 ranges over 32 k steps of 128 (uneven).  Every output against the
+    oracle, and bit for bit against the dense baseline."""
+    W = S.weight_with_verbatim_rows(1024, 4096, seed=94, frac_groups=0.01)
+    blob = uw.uw_compress(dev16(W))
+    X = S.activations(64, 4096, seed=95)
+    R = oracle_gemm(X, W, "f32")
+    Xd = dev16(X)
+    Yd = _f32(uw.uw_dense_gemm(Xd, dev16(W), out_f32=True))
+    check_gemm(Yd, R, bf16_out=False)
+    for pipe in PIPES:
+        Y = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True))
+        check_gemm(Y, R, bf16_out=False)
+        assert np.array_equal(Y, Yd), pipe
+    assert uw.uw_last_device_status() == 0
+
+
+_TIMEOUT_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import decode_gemm_bf16_b200 as uw, synthetic as S
+from tests.gpu_util import dev16
+from oracle import oracle as O
+W = S.weight_with_verbatim_rows(200, 1408, seed=32, frac_groups=0.01)
+blob = uw.uw_compress(dev16(W))
+X = S.activations(24, 1408, seed=11)
+Xd = dev16(X)
+# decoder beside the GEMM, but no decoder launched: the GEMM's bounded waits
+# for its bands run out and report UW_ERR_TIMEOUT
+uw.uw_gemm(Xd, blob, "transcode", sm_dec=37)
+print("status", uw.uw_last_device_status())
+# the context stays usable: a normal call afterwards is correct
+Y = uw.uw_gemm(Xd, blob, "transcode", out_f32=True).double().cpu().numpy()
+R = O.gemm(X, W, "f32")
+print("after", uw.uw_last_device_status(), float(np.abs(Y - R).max() / np.abs(R).max()))
+"""
+
+
+def test_bounded_wait_expires_with_timeout_status():
+    """A device-side wait that nothing satisfies (a decoder band never
+    published, via the UW_DEBUG_SKIP_DECODER hook) ends after UW_TIMEOUT_MS
+    with UW_ERR_TIMEOUT in the device status word; the process keeps using
+    the GPU normally afterwards.  Runs in a child process so the short
+    timeout and the hook stay out of the other tests."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, UW_TIMEOUT_MS="20", UW_DEBUG_SKIP_DECODER="1")
+    r = subprocess.run([sys.executable, "-c", _TIMEOUT_CHILD, root], env=env, capture_output=True, text=True,
+                       timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = dict(l.split(" ", 1) for l in r.stdout.strip().splitlines() if " " in l)
+    assert int(lines["status"]) == 7          # UW_ERR_TIMEOUT
+    after = lines["after"].split()
+    assert int(after[0]) == 0 and float(after[1]) < 1e-2
