@@ -16,7 +16,8 @@ method:
   -> encode (stream + chunk offsets)
 
 and back (decode -> exponents -> BF16), plus the reference product
-R = X . W^T accumulated in float64 (or float32 in ascending k).
+R = X . W^T accumulated in float64 (or float32 in ascending k), and the
+SwiGLU that joins the gate and up products, H = silu(G) * U.
 """
 from __future__ import annotations
 
@@ -78,6 +79,7 @@ def lib():
         L.or_gemm.argtypes = [P, P, I64, I64, I64, ctypes.c_int, P]
         L.or_gemm_one.argtypes = [P, P, I64, I64, I64, ctypes.c_int]
         L.or_gemm_one.restype = ctypes.c_double
+        L.or_swiglu.argtypes = [P, P, I64, P]
     return _lib
 
 
@@ -267,3 +269,13 @@ def gemm_one(X: np.ndarray, W: np.ndarray, m: int, n: int, acc: str = "f64") -> 
     X = np.ascontiguousarray(X, np.uint16)
     W = np.ascontiguousarray(W, np.uint16)
     return float(lib().or_gemm_one(_p(X), _p(W), X.shape[1], int(m), int(n), 1 if acc == "f64" else 0))
+
+
+def swiglu(G: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """H = silu(G) * U elementwise (float64), silu(z) = z / (1 + e^-z)."""
+    G = np.ascontiguousarray(G, np.float64)
+    U = np.ascontiguousarray(U, np.float64)
+    assert G.shape == U.shape
+    H = np.empty_like(G)
+    lib().or_swiglu(_p(G), _p(U), G.size, _p(H))
+    return H

@@ -409,3 +409,15 @@ double or_gemm_one(const uint16_t *X, const uint16_t *W, int64_t K, int64_t m, i
     }
     return acc_f64 ? accd : (double)accf;
 }
+
+/* Step 16 -- SwiGLU, the activation the MLP applies between its projections
+ * (named in the "future directions" section of the page): the down
+ * projection reads H = silu(G) * U, elementwise over the gate product G and
+ * the up product U, with silu(z) = z / (1 + e^-z).  Double precision. */
+void or_swiglu(const double *G, const double *U, int64_t n, double *H)
+{
+    for (int64_t i = 0; i < n; i++) {
+        double z = G[i];
+        H[i] = z / (1.0 + exp(-z)) * U[i];
+    }
+}

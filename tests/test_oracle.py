@@ -500,3 +500,26 @@ def test_gemm_matches_library_matmul_and_f32_bound():
     absdot = np.abs(S.bits_to_float(X).astype(np.float64)) @ np.abs(S.bits_to_float(W).astype(np.float64)).T
     assert np.all(np.abs(R32 - R) <= 256 * 2.0 ** -24 * absdot + 1e-30)
     assert O.gemm_one(X, W, 3, 5) == R[3, 5]
+
+
+# --------------------------------------------------------------------------
+# SwiGLU (the MLP's activation between gate/up and down)
+# --------------------------------------------------------------------------
+def test_swiglu_identities():
+    z = np.array([0.0, 0.25, -0.25, 1.0, -1.0, 3.5, -3.5, 12.0, -12.0, 40.0, -40.0])
+    ones = np.ones_like(z)
+    h = O.swiglu(z, ones)
+    # silu(0) = 0; silu(z) - silu(-z) = z (z s(z) + z s(-z) = z)
+    assert h[0] == 0.0
+    hn = O.swiglu(-z, ones)
+    assert np.allclose(h - hn, z, rtol=1e-14, atol=1e-14)
+    # an independent form: silu(z) = z/2 * (1 + tanh(z/2))
+    for zi, hi in zip(z, h):
+        assert abs(hi - zi / 2 * (1 + math.tanh(zi / 2))) <= 1e-14 * max(1.0, abs(zi))
+    # far tails: silu(40) = 40 to double precision, silu(-40) = -40 e^-40 (1 + O(e^-40))
+    assert h[-2] == 40.0
+    assert abs(h[-1] / (-40.0 * math.exp(-40.0)) - 1) < 1e-12
+    # the up product scales the result linearly (the gate does not)
+    u = np.array([2.0, -3.0, 0.5, 8.0, -0.125, 1.0, 1.0, 4.0, 4.0, 1.0, 1.0])
+    assert np.array_equal(O.swiglu(z, u), h * u)
+    assert O.swiglu(np.array([1.0]), np.array([2.0]))[0] == pytest.approx(2.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
