@@ -18,8 +18,10 @@ The line also carries, outside the timed step: per (projection, M) the time
 of one call (the plan's choice, rotated over the layers) with its compressed
 GB/s, TFLOP/s, roofline fraction and slowdown against the library's own
 dense BF16 GEMM; the compressed footprint of the stack per form; the
-decoders and the four pipelines at batch 1 on the gate projection; and the
-decoder/matmul SM split swept on the down projection at M = 256 and 1024.
+decoders and the five pipelines at batch 1 on the gate projection; the
+decoder/matmul SM split swept on the down projection at M = 256 and 1024;
+one MLP layer with gate+up in one launch (SwiGLU epilogue) feeding down; and
+the stack run as a sequence of hard (Huffman) and easy (palette) layers.
 
 --impl reference times the CPU oracle (plain C) on a bounded row sample of the
 same step and prints the same metric.
@@ -274,10 +276,14 @@ def _alg_bytes(info, pipeline, M, gemv):
         return (stream_b + n // 2) + (n + n // 2 + vstore + vcol + xy)
     if pipeline == "exponent":
         return (stream_b + vstore + n) + (2 * n + xy)
+    if pipeline == "fused_huffman":
+        return stream_b + n + vstore + xy
     return (stream_b + vstore + n + 2 * n) + (2 * n + xy)   # full
 
 
 def _kernel_name(pipeline, gemv):
+    if pipeline == "fused_huffman":
+        return "k_fused_huffman"
     if pipeline == "full":
         return "k_gemv<dense, M=1>" if gemv else "k_gemm_dense"
     src = "exponent" if pipeline == "exponent" else "palette"
@@ -483,7 +489,7 @@ def run_gpu(args):
         del g
         ops[name] = {"us": us, "alg_bytes": dec_alg[name], "alg_gbs": dec_alg[name] / (us * 1e-6) / 1e9,
                      "hbm_frac": dec_alg[name] / (us * 1e-6) / 1e9 / hbm_peak}
-    for pipe in ["full", "exponent", "transcode", "direct_palette"]:
+    for pipe in ["full", "exponent", "transcode", "direct_palette", "fused_huffman"]:
         g = capture(lambda pipe=pipe: [uw.uw_gemm(Xg[1], gate_blobs[i % n_copies], pipe, out=Y[("gate", 1)], ws=ws)
                                        for i in range(OP_BURST)])
         us = time_graph(g, OP_BURST)
@@ -506,6 +512,53 @@ def run_gpu(args):
                 del g
                 row[f"{pipe}/sm_dec={sd}"] = {"us": us, "tflops": 2.0 * M * 4096 * 14336 / (us * 1e-6) / 1e12}
         sm_split[f"M={M}"] = row
+    # ---- one MLP layer with the real data flow: gate+up in one launch with
+    # the SwiGLU epilogue, its output H feeding the down projection, against
+    # the plan's separate gate, up and down calls (layers rotated)
+    mlp = {}
+    Hs = {M: torch.empty(M, 14336, dtype=torch.bfloat16, device=dev) for M in MS}
+    sw_ws = torch.zeros(max(uw.uw_gemm_swiglu_workspace(blobs[0][0], blobs[0][1], M) for M in MS),
+                        dtype=torch.uint8, device=dev)
+    for M in MS:
+        g = capture(lambda M=M: [(uw.uw_gemm_swiglu(Xg[M], blobs[l][0], blobs[l][1], out=Hs[M], ws=sw_ws),
+                                  call("down", M, l, xin=Hs[M])) for l in range(L)])
+        us_fused = time_graph(g, L)
+        del g
+        g = capture(lambda M=M: [uw.uw_gemm_swiglu(Xg[M], blobs[l][0], blobs[l][1], out=Hs[M], ws=sw_ws)
+                                 for l in range(L)])
+        us_sw = time_graph(g, L)
+        del g
+        sep = per[f"gate/M={M}"]["us"] + per[f"up/M={M}"]["us"] + per[f"down/M={M}"]["us"]
+        mlp[f"M={M}"] = {"fused_layer_us": us_fused, "swiglu_gate_up_us": us_sw,
+                         "separate_gate_up_us": per[f"gate/M={M}"]["us"] + per[f"up/M={M}"]["us"],
+                         "separate_layer_us": sep, "speedup": sep / us_fused,
+                         "swiglu_tflops": 2 * 2.0 * M * 14336 * 4096 / (us_sw * 1e-6) / 1e12}
+
+    # ---- cross-layer hard/easy pipelining (§跨層管道化): the stack's
+    # projections as one sequence, every layer easy (palette form), every
+    # even layer hard (Huffman form, transcoded ahead on a side stream), or
+    # every layer hard
+    hard_easy = {}
+    seq_ws = None
+    for M in (1, 64, 256):
+        row = {}
+        for name, hard_of in (("all_easy", lambda l: False), ("alternate", lambda l: l % 2 == 0),
+                              ("all_hard", lambda l: True)):
+            items = [(blobs[l][j], Xof[p][M], Y[(p, M)], hard_of(l)) for l in range(L) for j, p in enumerate(PROJ)]
+            need = uw.uw_sequence_workspace(items, M)
+            if seq_ws is None or seq_ws.numel() < need:
+                seq_ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+            for dec in ((0, sms) if name != "all_easy" else (0,)):
+                g = capture(lambda items=items, dec=dec: uw.uw_gemm_sequence(items, M, dec_ctas=dec, ws=seq_ws))
+                us = time_graph(g, L, reps=3)
+                del g
+                row[f"{name}/dec_ctas={dec}"] = {"us_per_layer": us}
+        hard_easy[f"M={M}"] = row
+    pal_b = foot["palette_form"] / L
+    huf_b = foot["huffman_form"] / L
+    hard_easy["footprint_ratio"] = {"all_easy": foot["palette_form"] / foot["bf16"],
+                                    "alternate": (pal_b * (L // 2) + huf_b * (L - L // 2)) / foot["bf16"],
+                                    "all_hard": foot["huffman_form"] / foot["bf16"]}
     if uw.uw_last_device_status() != 0:
         raise RuntimeError("device status set during the breakdowns")
 
@@ -588,6 +641,8 @@ def run_gpu(args):
                                           for p, r in per_proj_ratio.items()}),
         "ops_gate_M1": ops,
         "sm_split_down": sm_split,
+        "mlp_layer_swiglu": mlp,
+        "hard_easy_layers": hard_easy,
         "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "path": "eager uw_gemm calls (ctypes C ABI), UW_PIPE_AUTO"},
         "gpu_launches": launches_per_step * args.steps,

@@ -25,7 +25,8 @@ STATUS = {0: "UW_OK", 1: "UW_ERR_INVALID_ARG", 2: "UW_ERR_SHAPE", 3: "UW_ERR_COR
           4: "UW_ERR_UNSUPPORTED", 5: "UW_ERR_WORKSPACE", 6: "UW_ERR_CUDA", 7: "UW_ERR_TIMEOUT",
           8: "UW_ERR_DEVICE"}
 UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXPONENT, UW_PIPE_TRANSCODE, UW_PIPE_DIRECT_PALETTE = -1, 0, 1, 2, 3
-PIPELINES = {"full": 0, "exponent": 1, "transcode": 2, "direct_palette": 3}
+UW_PIPE_FUSED_HUFFMAN = 4
+PIPELINES = {"full": 0, "exponent": 1, "transcode": 2, "direct_palette": 3, "fused_huffman": 4}
 UW_VARIANT_AUTO, UW_VARIANT_TENSOR, UW_VARIANT_GEMV = 0, 1, 2
 VARIANTS = {"auto": 0, "tensor": 1, "gemv": 2}
 UW_FORM_HUFFMAN, UW_FORM_PALETTE = 1, 2
@@ -38,7 +39,8 @@ EXPORTS = ["uw_status_str", "uw_version", "uw_last_device_status", "uw_compress_
            "uw_blob_deserialize", "uw_blob_free", "uw_decode_full", "uw_decode_exponent",
            "uw_transcode_palette", "uw_gemm_workspace", "uw_gemm", "uw_dense_gemm_workspace",
            "uw_dense_gemm", "uw_autotune", "uw_gemm_direct_palette_noalloc", "uw_plan_resolve",
-           "uw_plan_load_json"]
+           "uw_plan_load_json", "uw_gemm_swiglu_workspace", "uw_gemm_swiglu",
+           "uw_sequence_workspace", "uw_gemm_sequence"]
 
 
 class UnweightError(RuntimeError):
@@ -57,6 +59,10 @@ class BlobInfo(ctypes.Structure):
                 ("mean_code_len", ctypes.c_double), ("exponent_entropy", ctypes.c_double),
                 ("palette_coverage", ctypes.c_double), ("section_offset", ctypes.c_uint64 * 10),
                 ("section_bytes", ctypes.c_uint64 * 10)]
+
+
+class SeqItem(ctypes.Structure):
+    _fields_ = [("blob", ctypes.c_void_p), ("X", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("hard", ctypes.c_int32)]
 
 
 class PlanEntry(ctypes.Structure):
@@ -105,6 +111,10 @@ def lib():
             "uw_gemm_workspace": ([P, I64, ctypes.POINTER(GemmOpts), ctypes.POINTER(SZ)], I32),
             "uw_gemm": ([P, I64, P, P, ctypes.POINTER(GemmOpts), P], I32),
             "uw_plan_resolve": ([ctypes.POINTER(GemmOpts), I64, ctypes.POINTER(GemmOpts)], I32),
+            "uw_gemm_swiglu_workspace": ([P, P, I64, ctypes.POINTER(GemmOpts), ctypes.POINTER(SZ)], I32),
+            "uw_gemm_swiglu": ([P, I64, P, P, P, ctypes.POINTER(GemmOpts), P], I32),
+            "uw_sequence_workspace": ([ctypes.POINTER(SeqItem), I32, I64, ctypes.POINTER(SZ)], I32),
+            "uw_gemm_sequence": ([ctypes.POINTER(SeqItem), I32, I64, I32, I32, P, SZ, P], I32),
             "uw_dense_gemm_workspace": ([I64, I64, I64, I32, I32, I32, ctypes.POINTER(SZ)], I32),
             "uw_dense_gemm": ([P, I64, P, I64, I64, P, I32, I32, I32, I32, P, SZ, P], I32),
             "uw_gemm_direct_palette_noalloc": ([P, I64, P, P, I32, P], I32),
@@ -334,6 +344,61 @@ def uw_gemm(X: torch.Tensor, blob: Blob, pipeline="direct_palette", out: Optiona
     o = _opts(pipeline, sm_dec, grid, out_f32, ws, variant, split_k, stages, plan, projection)
     _check(lib().uw_gemm(_ptr(X), M, blob.handle, _ptr(out), ctypes.byref(o), _stream(stream)), "uw_gemm")
     return out
+
+
+def uw_gemm_swiglu_workspace(gate: Blob, up: Blob, M: int, grid: int = 0, split_k: int = 0, variant=0) -> int:
+    o = _opts("direct_palette", 0, grid, variant=variant, split_k=split_k)
+    n = ctypes.c_size_t()
+    _check(lib().uw_gemm_swiglu_workspace(gate.handle, up.handle, int(M), ctypes.byref(o), ctypes.byref(n)),
+           "uw_gemm_swiglu_workspace")
+    return n.value
+
+
+def uw_gemm_swiglu(X: torch.Tensor, gate: Blob, up: Blob, out: Optional[torch.Tensor] = None, out_f32: bool = False,
+                   ws: Optional[torch.Tensor] = None, grid: int = 0, split_k: int = 0, stages: int = 0, variant=0,
+                   pipeline="direct_palette", stream=None) -> torch.Tensor:
+    """H[M, N] = silu(X . Wg^T) * (X . Wu^T) in one launch from the palette
+    forms of the gate and up projections."""
+    X = _bits16(X)
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, gate.N, dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = workspace(uw_gemm_swiglu_workspace(gate, up, M, grid, split_k, variant), X.device)
+    o = _opts(pipeline, 0, grid, out_f32, ws, variant, split_k, stages)
+    _check(lib().uw_gemm_swiglu(_ptr(X), M, gate.handle, up.handle, _ptr(out), ctypes.byref(o), _stream(stream)),
+           "uw_gemm_swiglu")
+    return out
+
+
+def _seq_items(items):
+    arr = (SeqItem * len(items))()
+    for i, (blob, X, Y, hard) in enumerate(items):
+        h = blob.handle
+        arr[i].blob = h.value if hasattr(h, "value") else h
+        arr[i].X = X.data_ptr()
+        arr[i].Y = Y.data_ptr()
+        arr[i].hard = 1 if hard else 0
+    return arr
+
+
+def uw_sequence_workspace(items, M: int) -> int:
+    """items: sequence of (blob, X, Y, hard)."""
+    arr = _seq_items(items)
+    n = ctypes.c_size_t()
+    _check(lib().uw_sequence_workspace(arr, len(items), int(M), ctypes.byref(n)), "uw_sequence_workspace")
+    return n.value
+
+
+def uw_gemm_sequence(items, M: int, out_f32: bool = False, dec_ctas: int = 0, ws: Optional[torch.Tensor] = None,
+                     stream=None):
+    """Runs (blob, X, Y, hard) items in order; hard items' transcodes run ahead
+    on a side stream (§跨層管道化)."""
+    arr = _seq_items(items)
+    if ws is None:
+        ws = workspace(uw_sequence_workspace(items, M), items[0][1].device)
+    _check(lib().uw_gemm_sequence(arr, len(items), int(M), 1 if out_f32 else 0, int(dec_ctas), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "uw_gemm_sequence")
 
 
 def uw_gemm_direct_palette_noalloc(X: torch.Tensor, blob: Blob, out: Optional[torch.Tensor] = None,

@@ -309,7 +309,313 @@ __global__ void __launch_bounds__(WARPS * 32, kStaged<MODE, WARPS> ? 3 : 4) k_de
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fused Huffman-decode GEMV / small-batch product: Y[M,N] = X[M,K] . W^T read
+// straight from the Huffman form (sign+mantissa plane + stream + verbatim
+// store, ~1.34 bytes per weight), with no decoded plane written to HBM.  The
+// pages' Hopper design could not keep the 16 KB decode table beside the
+// matmul's buffers (§解壓與運算資源共享); here the decode table, the decoded
+// nibbles and the activations share one CTA's shared memory with the
+// multiply.
+//
+// Work split: a warp owns 32 consecutive rows (lane = row) and a range of
+// kseg consecutive 256-weight segments of each.  Per segment, each lane
+// decodes its row's 256 symbols from the segment's start bit (the decoder
+// core above) into its shared-memory words, then walks them 16 weights at a
+// time: sign+mantissa bytes from the plane (16-byte loads), exponents from the
+// palette (or the verbatim store), BF16 rebuilt in registers and widened,
+// fused multiply-adds in k order into per-batch-row sums (even and odd
+// weights apart).  All lanes read the same activations at the same time
+// (shared-memory broadcast).  With several k ranges per row, each warp
+// publishes its 32 x M partial sums and the last warp of the row group to
+// arrive (a tagged counter) adds them in k-range order: the result does not
+// depend on the launch, only on the shape.
+// ---------------------------------------------------------------------------
+constexpr int kFusedWarps = 8;
+constexpr size_t kFusedXsMax = 64 * 1024;   // fp32 activations in shared memory up to this size
+
+struct FusedParams {
+    DecodeParams d;
+    const uint16_t* X;
+    int M;
+    int64_t N, K, KG;
+    int S;                     // 256-weight segments per row
+    int kseg;                  // segments per k range
+    int nkr;                   // k ranges per row
+    int64_t ngroups;           // groups of 32 rows
+    int64_t items;             // ngroups * nkr warp tasks
+    float* part;               // [nkr][N][M] partial sums
+    unsigned long long* cnt;   // [ngroups] tagged arrival counters
+    unsigned long long epoch;
+    void* Y;
+    int out_f32;
+};
+
+__device__ __forceinline__ void fma_bf16x2(float2& acc, uint32_t w, float x0, float x1) {
+    acc.x = fmaf(__uint_as_float(w << 16), x0, acc.x);
+    acc.y = fmaf(__uint_as_float(w & 0xFFFF0000u), x1, acc.y);
+}
+
+template <int MB, bool XS>
+__global__ void __launch_bounds__(kFusedWarps * 32, 2) k_fused_huffman(const FusedParams p) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    uint32_t* stage = smem + kLutSize;
+    float* xs = reinterpret_cast<float*>(stage + kFusedWarps * 32 * 32);
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(p.d.lut);
+        uint4* dst = reinterpret_cast<uint4*>(lut);
+        for (int i = threadIdx.x; i < kLutSize / 4; i += kFusedWarps * 32) dst[i] = __ldg(&src[i]);
+    }
+    // programmatic stream serialization: the table comes from the committed
+    // blob; activations, partial sums and outputs after the previous kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (XS) {
+        const int64_t n4 = (int64_t)p.M * p.K / 4;
+        for (int64_t c = threadIdx.x; c < n4; c += kFusedWarps * 32) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.X) + c);
+            reinterpret_cast<float4*>(xs)[c] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                                                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+        }
+    }
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* st = stage + warp * (32 * 32) + lane * 32;
+    const uint32_t P0 = p.d.pal[0], P1 = p.d.pal[1], P2 = p.d.pal[2], P3 = p.d.pal[3];
+    const int M = p.M;
+    for (int64_t item = (int64_t)blockIdx.x * kFusedWarps + warp; item < p.items;
+         item += (int64_t)gridDim.x * kFusedWarps) {
+        const int64_t rg = item / p.nkr;
+        const int kr = (int)(item - rg * p.nkr);
+        const int64_t r = rg * 32 + lane;
+        const bool valid = r < p.N;
+        const int j0 = kr * p.kseg, j1 = min(p.S, j0 + p.kseg);
+        float2 acc[MB];
+#pragma unroll
+        for (int m = 0; m < MB; m++) acc[m] = make_float2(0.f, 0.f);
+        if (valid) {
+            for (int j = j0; j < j1; j++) {
+                const int64_t seg = r * p.S + j;
+                const uint64_t bitpos = __ldg(&p.d.chunk_off[seg >> 4]) + __ldg(&p.d.seg_rel[seg]);
+                decode_bits<false>(p.d, lut, p.d.stream, p.d.nwords - 1, bitpos, kSeg, st, lane);
+                const int64_t kbase = (int64_t)j * kSeg;
+                const uint8_t* smr = p.d.sm + r * p.K + kbase;
+#pragma unroll 1
+                for (int q = 0; q < kSeg / kGroup; q++) {
+                    const int64_t g = r * p.KG + (kbase >> 6) + q;
+                    const uint32_t vw = __ldg(&p.d.vbits[g >> 5]);
+                    const bool verb = (vw >> (g & 31)) & 1u;
+                    const uint8_t* vsrc = nullptr;
+                    if (verb) {
+                        const int64_t rank = __ldg(&p.d.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
+                        vsrc = p.d.vexp + rank * kGroup;
+                    }
+#pragma unroll 2
+                    for (int i = 0; i < kGroup / 16; i++) {
+                        const int c = q * 4 + i;   // 16-weight chunk of the segment
+                        const uint4 sv = __ldcs(reinterpret_cast<const uint4*>(smr + c * 16));
+                        uint32_t E[4];
+                        if (verb) {
+                            const uint4 e = __ldg(reinterpret_cast<const uint4*>(vsrc + i * 16));
+                            E[0] = e.x; E[1] = e.y; E[2] = e.z; E[3] = e.w;
+                        } else {
+                            const uint32_t w0 = st[(2 * c + lane) & 31], w1 = st[(2 * c + 1 + lane) & 31];
+                            if (p.d.pal_small) {
+                                const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
+                                E[0] = palette4_small(w0, x0, P0, P1, P2, P3);
+                                E[1] = palette4_small(w0 >> 16, x0 >> 16, P0, P1, P2, P3);
+                                E[2] = palette4_small(w1, x1, P0, P1, P2, P3);
+                                E[3] = palette4_small(w1 >> 16, x1 >> 16, P0, P1, P2, P3);
+                            } else {
+                                E[0] = palette4(w0, P0, P1, P2, P3);
+                                E[1] = palette4(w0 >> 16, P0, P1, P2, P3);
+                                E[2] = palette4(w1, P0, P1, P2, P3);
+                                E[3] = palette4(w1 >> 16, P0, P1, P2, P3);
+                            }
+                        }
+                        const uint32_t S4[4] = {sv.x, sv.y, sv.z, sv.w};
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int t = 0; t < 4; t++) {
+                            const uint2 mm = merge4(E[t], S4[t]);
+                            wv[2 * t] = mm.x;
+                            wv[2 * t + 1] = mm.y;
+                        }
+                        const int64_t k = kbase + c * 16;
+#pragma unroll
+                        for (int m = 0; m < MB; m++) {
+                            if (m < M) {
+                                if (XS) {
+                                    const float4* x4 = reinterpret_cast<const float4*>(xs + (int64_t)m * p.K + k);
+#pragma unroll
+                                    for (int t = 0; t < 4; t++) {
+                                        const float4 xv = x4[t];
+                                        fma_bf16x2(acc[m], wv[2 * t], xv.x, xv.y);
+                                        fma_bf16x2(acc[m], wv[2 * t + 1], xv.z, xv.w);
+                                    }
+                                } else {
+                                    const uint4* xp = reinterpret_cast<const uint4*>(p.X + (int64_t)m * p.K + k);
+#pragma unroll
+                                    for (int t = 0; t < 2; t++) {
+                                        const uint4 xv = __ldg(xp + t);
+                                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                                        for (int u = 0; u < 4; u++)
+                                            fma_bf16x2(acc[m], wv[4 * t + u], __uint_as_float(xw[u] << 16),
+                                                       __uint_as_float(xw[u] & 0xFFFF0000u));
+                                    }
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        if (p.nkr == 1) {
+            if (valid) {
+#pragma unroll
+                for (int m = 0; m < MB; m++) {
+                    if (m >= M) break;
+                    const float v = acc[m].x + acc[m].y;
+                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[(int64_t)m * p.N + r] = v;
+                    else {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                        reinterpret_cast<uint16_t*>(p.Y)[(int64_t)m * p.N + r] = *reinterpret_cast<const uint16_t*>(&h);
+                    }
+                }
+            }
+            continue;
+        }
+        // several k ranges: publish, and the last warp of the row group sums
+        if (valid) {
+#pragma unroll
+            for (int m = 0; m < MB; m++)
+                if (m < M) p.part[((int64_t)kr * p.N + r) * M + m] = acc[m].x + acc[m].y;
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned c = 0;
+        if (lane == 0) c = arrive_counter(p.cnt + rg, p.epoch);
+        c = __shfl_sync(0xFFFFFFFFu, c, 0);
+        if (c == (unsigned)p.nkr) {
+            __threadfence();
+            if (valid) {
+                for (int m = 0; m < M; m++) {
+                    float v = 0.f;
+                    for (int kk = 0; kk < p.nkr; kk++) v += __ldcg(p.part + ((int64_t)kk * p.N + r) * M + m);
+                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[(int64_t)m * p.N + r] = v;
+                    else {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                        reinterpret_cast<uint16_t*>(p.Y)[(int64_t)m * p.N + r] = *reinterpret_cast<const uint16_t*>(&h);
+                    }
+                }
+            }
+            // a replay of the same captured call reuses its tag: start again from zero
+            if (lane == 0) p.cnt[rg] = 0ull;
+        }
+    }
+}
+
+// Split of one fused call: k ranges per row and segments per range, so that
+// about 24 warp tasks per SM exist.
+struct FusedSplit {
+    int S, kseg, nkr;
+    int64_t ngroups, items;
+};
+
+FusedSplit fused_split(int64_t N, int64_t K) {
+    FusedSplit f;
+    f.S = (int)(K / kSeg);
+    f.ngroups = (N + 31) / 32;
+    const int64_t target = (int64_t)num_sms() * 24;
+    int64_t kseg = (f.S * f.ngroups + target / 2) / target;
+    if (kseg < 1) kseg = 1;
+    if (kseg > f.S) kseg = f.S;
+    f.kseg = (int)kseg;
+    f.nkr = (f.S + f.kseg - 1) / f.kseg;
+    f.items = f.ngroups * f.nkr;
+    return f;
+}
+
 }  // namespace
+
+static DecodeParams decode_params(const uw_blob* b, void* out);
+
+size_t fused_ws_bytes(int64_t M, int64_t N, int64_t K) {
+    if (K % kSeg) return 0;
+    const FusedSplit f = fused_split(N, K);
+    const int64_t mc = M < kFusedMaxM ? M : kFusedMaxM;
+    const size_t part = (size_t)f.nkr * N * mc * 4;
+    return ((part + 255) & ~size_t(255)) + (((size_t)f.ngroups * 8 + 255) & ~size_t(255));
+}
+
+cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M, void* Y, int out_f32, void* ws,
+                                 size_t ws_bytes, cudaStream_t s, uw_status* st) {
+    *st = UW_OK;
+    if (M == 0) return cudaSuccess;
+    if (M > kFusedMaxM || b->geo.K % kSeg) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
+    const size_t need = fused_ws_bytes(M, b->geo.N, b->geo.K);
+    if (!ws || ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
+    FusedParams p;
+    p.d = decode_params(b, nullptr);
+    p.X = X;
+    p.M = (int)M;
+    p.N = b->geo.N;
+    p.K = b->geo.K;
+    p.KG = b->geo.KG;
+    const FusedSplit f = fused_split(p.N, p.K);
+    p.S = f.S;
+    p.kseg = f.kseg;
+    p.nkr = f.nkr;
+    p.ngroups = f.ngroups;
+    p.items = f.items;
+    const size_t part = (size_t)f.nkr * p.N * M * 4;
+    p.part = (float*)ws;
+    p.cnt = (unsigned long long*)((uint8_t*)ws + ((part + 255) & ~size_t(255)));
+    p.epoch = gemm_next_epoch();
+    p.Y = Y;
+    p.out_f32 = out_f32;
+    const size_t xbytes = (size_t)M * p.K * 4;
+    const bool xs = xbytes <= kFusedXsMax;
+    const size_t smem = (size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4 + (xs ? xbytes : 0);
+    const int mb = M == 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+    typedef void (*Kern)(const FusedParams);
+    Kern kern = nullptr;
+#define UW_FUSED_CASE(B)                                                  \
+    if (mb == B) kern = xs ? k_fused_huffman<B, true> : k_fused_huffman<B, false>;
+    UW_FUSED_CASE(1)
+    UW_FUSED_CASE(2)
+    UW_FUSED_CASE(4)
+    UW_FUSED_CASE(8)
+    UW_FUSED_CASE(16)
+#undef UW_FUSED_CASE
+    static bool attr_set[5][2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int mi = mb == 1 ? 0 : mb == 2 ? 1 : mb == 4 ? 2 : mb == 8 ? 3 : 4;
+    bool& done = attr_set[mi][xs ? 1 : 0][dev & 63];
+    if (!done) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)((size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4 + kFusedXsMax));
+        if (e != cudaSuccess) return e;
+        done = true;
+    }
+    const int64_t grid = (p.items + kFusedWarps - 1) / kFusedWarps;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kFusedWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
 
 int decode_ctas_per_sm() { return 4; }
 

@@ -72,18 +72,28 @@ constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
 constexpr uint32_t kTileA64 = kBlockN * kBoxK * 2;       // 16 KB: one 64-k box of BF16 weights
 constexpr int kFinBufs = 4;                              // finisher staging rows in flight per warp
 
-struct GemmParams {
-    int64_t M, N, K, KG;
-    int MG, m_tiles, n_tiles, kt_count, P, stages;
-    uint32_t total_iters;
-    uint32_t stage_bytes, off_a, off_b, off_sm, off_s2, off_v, tx_bytes;
-    uint32_t tmem_cols;   // TMEM columns allocated (power of two)
-    uint32_t a_col0;      // first TMEM column of the rebuilt-A stages (32 columns each)
-    int pal_small;        // all palette exponents < 128: cheaper lookup
+// One weight matrix's planes as a stage sees them: where its TMA tiles sit
+// in the stage, its verbatim store and its palette.  A paired call (gate and
+// up projections, SwiGLU epilogue) carries two.
+struct PlaneSet {
+    uint32_t off_sm, off_s2, off_v;   // stage offsets: sign+mantissa, exponent/index, verbatim flags
+    int pal_small;                    // all palette exponents < 128: cheaper lookup
     const uint32_t* vbits;
     const uint32_t* vpre;
     const uint8_t* vexp;
     uint32_t pal[4];
+};
+
+struct GemmParams {
+    int64_t M, N, K, KG;
+    int MG, m_tiles, n_tiles, kt_count, P, stages;
+    int nh;               // weight matrices per tile: 1, or 2 (gate, up) with the SwiGLU epilogue
+    int acc_w;            // accumulator columns per tile: nh * MG (gate in [0, MG), up in [MG, 2 MG))
+    uint32_t total_iters;
+    uint32_t stage_bytes, off_a, off_b, tx_bytes;
+    uint32_t tmem_cols;   // TMEM columns allocated (power of two)
+    uint32_t a_col0;      // first TMEM column of the rebuilt-A stages (nh * KB/2 columns each)
+    PlaneSet ps[2];
     void* Y;
     int out_f32;
     float* partial;                // [2P][MG/4][128][4]: float4 j of row r at (slot*MG/4 + j)*128 + r
@@ -169,38 +179,38 @@ __device__ __forceinline__ uint32_t sw32_off(int r, int c) { return r * 32 + ((c
 // taddr .. +15 (one BF16 pair per column).  Sign+mantissa and exponent
 // tiles have rows of KB bytes (swizzle KB), index tiles rows of KB/2 bytes.
 template <int SRC, int KB>
-__device__ __forceinline__ void rebuild_row(const GemmParams& p, const uint8_t* stage, int64_t n0, int kt,
-                                            int q, int j, int lane, uint32_t taddr) {
+__device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet& ps, const uint8_t* stage, int64_t n0,
+                                            int kt, int q, int j, int lane, uint32_t taddr) {
     const int r = 32 * q + lane;
     auto row_off = [&](int c) { return KB == 128 ? sw128_off(r, c) : sw64_off(r, c); };
-    const uint8_t* SM = stage + p.off_sm;
+    const uint8_t* SM = stage + ps.off_sm;
     const uint4 s0 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j));
     const uint4 s1 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j + 1));
     uint32_t E[8];
     if (SRC == kSrcExponent) {
-        const uint8_t* EX = stage + p.off_s2;
+        const uint8_t* EX = stage + ps.off_s2;
         const uint4 e0 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j));
         const uint4 e1 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j + 1));
         E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
         E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
     } else {
         const int grp = j >> 1;   // 64-weight group within the stage
-        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + p.off_v + 16 * grp + 4 * q);
+        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + ps.off_v + 16 * grp + 4 * q);
         if ((vw >> lane) & 1u) {
             // verbatim group: raw exponents from the verbatim store
             const int64_t g = (n0 + r) * p.KG + (int64_t)kt * (KB / kGroup) + grp;
-            const uint32_t w = __ldg(&p.vbits[g >> 5]);
-            const int64_t rank = __ldg(&p.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
-            const uint4* src = reinterpret_cast<const uint4*>(p.vexp + rank * kGroup + 32 * (j & 1));
+            const uint32_t w = __ldg(&ps.vbits[g >> 5]);
+            const int64_t rank = __ldg(&ps.vpre[g >> 5]) + __popc(w & ((1u << (g & 31)) - 1u));
+            const uint4* src = reinterpret_cast<const uint4*>(ps.vexp + rank * kGroup + 32 * (j & 1));
             const uint4 e0 = __ldg(src), e1 = __ldg(src + 1);
             E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
             E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
         } else {
             const uint4 ix = *reinterpret_cast<const uint4*>(
-                stage + p.off_s2 + (KB == 128 ? sw64_off(r, j) : sw32_off(r, j)));
+                stage + ps.off_s2 + (KB == 128 ? sw64_off(r, j) : sw32_off(r, j)));
             const uint32_t w[4] = {ix.x, ix.y, ix.z, ix.w};
-            const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
-            if (p.pal_small) {
+            const uint32_t P0 = ps.pal[0], P1 = ps.pal[1], P2 = ps.pal[2], P3 = ps.pal[3];
+            if (ps.pal_small) {
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const uint32_t xs = w[i] ^ 0x88888888u;
@@ -250,28 +260,60 @@ __device__ __forceinline__ void store_y(void* Y, int64_t M, int64_t N, int out_f
     }
 }
 
+// SwiGLU of 16 outputs: h = silu(g) * u, silu(g) = g / (1 + e^-g), in fp32
+// from the two accumulators (bit patterns in, bit patterns out).
+__device__ __forceinline__ void swiglu16(const uint32_t (&g)[16], const uint32_t (&u)[16], uint32_t (&h)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const float gv = __uint_as_float(g[i]);
+        h[i] = __float_as_uint(gv / (1.0f + __expf(-gv)) * __uint_as_float(u[i]));
+    }
+}
+
+// Output of a finished accumulator in TMEM: Y directly, or (paired gate and
+// up accumulators) SwiGLU of the two halves.
+__device__ __forceinline__ void write_out(void* Y, int64_t M, int64_t N, int out_f32, int MG, int nh, uint32_t trow,
+                                          int64_t n, int64_t m0) {
+    for (int c0 = 0; c0 < MG; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(trow + (uint32_t)c0, v);
+        if (nh == 2) {
+            uint32_t u[16], h[16];
+            tmem_ld16(trow + (uint32_t)(MG + c0), u);
+            tmem_wait_ld();
+            swiglu16(v, u, h);
+            store_y(Y, M, N, out_f32, h, n, m0 + c0);
+        } else {
+            tmem_wait_ld();
+            store_y(Y, M, N, out_f32, v, n, m0 + c0);
+        }
+    }
+}
+
 // Finisher of a split tile: own accumulator (TMEM) + the partial rows of
 // CTAs blockIdx.x + 1 .. b_last in that order, then Y.  Columns go in blocks
 // of CB; this warp's accumulator rows (32 x CB) and kFinBufs staging rows
 // live in `fin` (rows of CB + 4 floats: a 16-byte bank shift per lane), and
 // the (block, contributor) items stream in with asynchronous copies,
-// kFinBufs - 1 ahead.  Kept out of line: it runs once per CTA and would
-// otherwise set the register budget of the whole kernel.
+// kFinBufs - 1 ahead.  A paired accumulator (gate and up halves) is summed
+// back into TMEM and written through the SwiGLU afterwards.  Kept out of
+// line: it runs once per CTA and would otherwise set the register budget of
+// the whole kernel.
 struct FinArgs {
     const float* partial;
     void* Y;
     int64_t M, N;
-    int MG, CB, out_f32;
+    int AW, MG, nh, CB, out_f32;   // accumulator columns (nh * MG), output columns, halves
     uint32_t total, P, kt;
 };
 
 __device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_t b_last, int64_t n, int64_t m0,
                                          uint32_t trow, float* fin, int lane) {
     const int CB = f.CB, RS = CB + 4;
-    const int MG4 = f.MG / 4;
+    const int AW4 = f.AW / 4;
     const int r = (int)(threadIdx.x & 127);
     const uint32_t nb = b_last - blockIdx.x;   // contributors, in k order after this CTA
-    const uint32_t nblk = (uint32_t)((f.MG + CB - 1) / CB);
+    const uint32_t nblk = (uint32_t)((f.AW + CB - 1) / CB);
     const uint32_t items = nb * nblk;
     float* facc = fin + lane * RS;
     const uint32_t fbuf = smem_u32(fin + 32 * RS + lane * RS);   // staging rows, 32*RS floats apart
@@ -282,9 +324,9 @@ __device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_
         if (t < items) {
             const uint32_t blk = t / nb, i = t - blk * nb;
             const int cb0 = (int)blk * CB;
-            const int cw = f.MG - cb0 < CB ? f.MG - cb0 : CB;
+            const int cw = f.AW - cb0 < CB ? f.AW - cb0 : CB;
             const uint32_t sl = slot_of(blockIdx.x + 1 + i, tile, f.total, f.P, f.kt);
-            const float4* src = part4 + ((size_t)sl * MG4 + cb0 / 4) * kBlockN + r;
+            const float4* src = part4 + ((size_t)sl * AW4 + cb0 / 4) * kBlockN + r;
             const uint32_t dst = fbuf + (t % kFinBufs) * (uint32_t)(32 * RS * 4);
             for (int q = 0; q < cw / 4; q++) cp_async16(dst + 16u * q, src + (size_t)q * kBlockN);
         }
@@ -294,7 +336,7 @@ __device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_
     uint32_t t = 0;
     for (uint32_t blk = 0; blk < nblk; blk++) {
         const int cb0 = (int)blk * CB;
-        const int cw = f.MG - cb0 < CB ? f.MG - cb0 : CB;
+        const int cw = f.AW - cb0 < CB ? f.AW - cb0 : CB;
         for (int c = 0; c < cw; c += 16) {
             uint32_t v[16];
             tmem_ld16(trow + (uint32_t)(cb0 + c), v);
@@ -331,16 +373,23 @@ __device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_
                 v[4 * i + 2] = x.z;
                 v[4 * i + 3] = x.w;
             }
-            store_y(f.Y, f.M, f.N, f.out_f32, v, n, m0 + cb0 + c);
+            if (f.nh == 2) tmem_st16(trow + (uint32_t)(cb0 + c), v);   // the sum, back into the accumulator
+            else store_y(f.Y, f.M, f.N, f.out_f32, v, n, m0 + cb0 + c);
         }
     }
     cp_async_wait<0>();
+    if (f.nh == 2) {
+        tmem_wait_st();
+        write_out(f.Y, f.M, f.N, f.out_f32, f.MG, 2, trow, n, m0);
+    }
 }
 
-template <int SRC, int KB>
+template <int SRC, int KB, int NH>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_a, const CUtensorMap& tm_s2,
-                                          const CUtensorMap& tm_v, const GemmParams& p) {
+                                          const CUtensorMap& tm_v, const CUtensorMap& tm_a2, const CUtensorMap& tm_s22,
+                                          const CUtensorMap& tm_v2, const GemmParams& p) {
     static_assert(KB == 64 || KB == 128, "stage k");
+    static_assert(NH == 1 || (NH == 2 && SRC == kSrcPalette), "paired tiles: palette source");
     constexpr int kHalves = KB / kBoxK;   // 64-k boxes of X (and of dense W) per stage
     constexpr bool kRecon = SRC != kSrcDense;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -358,6 +407,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = p.tmem_cols;
+    const CUtensorMap* maps_a[2] = {&tm_a, &tm_a2};
+    const CUtensorMap* maps_s2[2] = {&tm_s2, &tm_s22};
+    const CUtensorMap* maps_v[2] = {&tm_v, &tm_v2};
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
@@ -377,10 +429,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     }
     if (warp == kProdWarp && lane == 0) {
         tma_prefetch_desc(&tm_x);
-        tma_prefetch_desc(&tm_a);
-        if (kRecon) {
-            tma_prefetch_desc(&tm_s2);
-            if (SRC == kSrcPalette) tma_prefetch_desc(&tm_v);
+#pragma unroll
+        for (int h = 0; h < NH; h++) {
+            tma_prefetch_desc(maps_a[h]);
+            if (kRecon) {
+                tma_prefetch_desc(maps_s2[h]);
+                if (SRC == kSrcPalette) tma_prefetch_desc(maps_v[h]);
+            }
         }
     }
     tc_fence_before();
@@ -417,10 +472,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                         const uint32_t st = smem_base + npre * p.stage_bytes;
                         const uint32_t fb = smem_u32(&full_bar[npre]);
                         mbar_arrive_expect_tx(fb, p.tx_bytes);
-                        tma_load_2d(st + p.off_sm, &tm_a, kt * KB, n_tile * kBlockN, fb);
-                        if (SRC == kSrcPalette) {
-                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
-                            if (p.static_s2) tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
+#pragma unroll
+                        for (int h = 0; h < NH; h++) {
+                            const PlaneSet& ps = p.ps[h];
+                            tma_load_2d(st + ps.off_sm, maps_a[h], kt * KB, n_tile * kBlockN, fb);
+                            if (SRC == kSrcPalette) {
+                                tma_load_2d(st + ps.off_v, maps_v[h], n_tile * (kBlockN / 32), kt * kHalves, fb);
+                                if (p.static_s2)
+                                    tma_load_2d(st + ps.off_s2, maps_s2[h], kt * (KB / 2), n_tile * kBlockN, fb);
+                            }
                         }
                     }
                 }
@@ -455,9 +515,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                             for (int hb = 0; hb < kHalves; hb++)
                                 tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, fb);
                             if (SRC == kSrcExponent)
-                                tma_load_2d(st + p.off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
+                                tma_load_2d(st + p.ps[0].off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
                             else if (!p.static_s2)
-                                tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
+                                tma_load_2d(st + p.ps[0].off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
                         }
                         continue;
                     }
@@ -474,12 +534,16 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                         for (int hb = 0; hb < kHalves; hb++)
                             tma_load_2d(st + p.off_a + hb * kTileA64, &tm_a, kt * KB + hb * kBoxK, n_tile * kBlockN, fb);
                     } else {
-                        tma_load_2d(st + p.off_sm, &tm_a, kt * KB, n_tile * kBlockN, fb);
-                        if (SRC == kSrcExponent)
-                            tma_load_2d(st + p.off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
-                        else {
-                            tma_load_2d(st + p.off_s2, &tm_s2, kt * (KB / 2), n_tile * kBlockN, fb);
-                            tma_load_2d(st + p.off_v, &tm_v, n_tile * (kBlockN / 32), kt * kHalves, fb);
+#pragma unroll
+                        for (int h = 0; h < NH; h++) {
+                            const PlaneSet& ps = p.ps[h];
+                            tma_load_2d(st + ps.off_sm, maps_a[h], kt * KB, n_tile * kBlockN, fb);
+                            if (SRC == kSrcExponent)
+                                tma_load_2d(st + ps.off_s2, maps_s2[h], kt * KB, n_tile * kBlockN, fb);
+                            else {
+                                tma_load_2d(st + ps.off_s2, maps_s2[h], kt * (KB / 2), n_tile * kBlockN, fb);
+                                tma_load_2d(st + ps.off_v, maps_v[h], n_tile * (kBlockN / 32), kt * kHalves, fb);
+                            }
                         }
                     }
                 }
@@ -493,7 +557,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp walks the loop; one elected lane issues the MMAs
-        // and commits.
+        // and commits.  Paired tiles: the gate rows accumulate into columns
+        // [0, MG), the up rows into [MG, 2 MG).
         {
             const bool leader = elect_one();
             const uint32_t idesc = mma_idesc_bf16(kBlockN, p.MG);
@@ -511,22 +576,26 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     if (!mbar_wait(wb, rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_base + s * p.stage_bytes;
-                    // 16 k = 32 bytes further along a swizzled row: +2 in the
-                    // descriptor's start-address field (16-byte units)
-                    const uint32_t ta0 = tacc + p.a_col0 + (uint32_t)(KB / 2) * (uint32_t)s;
                     if (!leader) continue;
 #pragma unroll
-                    for (int hb = 0; hb < kHalves; hb++) {
-                        const uint64_t bd0 = sw128_desc(st + p.off_b + hb * p.MG * 128);
-                        const uint64_t ad0 = sw128_desc(st + p.off_a + hb * kTileA64);
+                    for (int h = 0; h < NH; h++) {
+                        // 16 k = 32 bytes further along a swizzled row: +2 in the
+                        // descriptor's start-address field (16-byte units)
+                        const uint32_t ta0 = tacc + p.a_col0 + (uint32_t)(KB / 2) * (uint32_t)(NH * s + h);
+                        const uint32_t dacc = tacc + (uint32_t)(h * p.MG);
 #pragma unroll
-                        for (int kk = 0; kk < kBoxK / 16; kk++) {
-                            const uint32_t acc = (kt > sg.kt0 || hb > 0 || kk > 0) ? 1u : 0u;
-                            if (kRecon) {
-                                // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
-                                tc_mma_tmem_a(tacc, ta0 + 8u * (uint32_t)(hb * 4 + kk), bd0 + 2u * kk, idesc, acc);
-                            } else {
-                                tc_mma(tacc, ad0 + 2u * kk, bd0 + 2u * kk, idesc, acc);
+                        for (int hb = 0; hb < kHalves; hb++) {
+                            const uint64_t bd0 = sw128_desc(st + p.off_b + hb * p.MG * 128);
+                            const uint64_t ad0 = sw128_desc(st + p.off_a + hb * kTileA64);
+#pragma unroll
+                            for (int kk = 0; kk < kBoxK / 16; kk++) {
+                                const uint32_t acc = (kt > sg.kt0 || hb > 0 || kk > 0) ? 1u : 0u;
+                                if (kRecon) {
+                                    // A: 8 TMEM columns (16 k) of this stage's rebuilt rows
+                                    tc_mma_tmem_a(dacc, ta0 + 8u * (uint32_t)(hb * 4 + kk), bd0 + 2u * kk, idesc, acc);
+                                } else {
+                                    tc_mma(dacc, ad0 + 2u * kk, bd0 + 2u * kk, idesc, acc);
+                                }
                             }
                         }
                     }
@@ -546,11 +615,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // warp w may only touch TMEM lanes 32(w%4)..+31.  Two groups of 8
         // warps take alternate stages (two stages rebuilt at once); inside a
         // group, two warps per lane quarter, one per half of the stage's k
-        // (one or two 32-k pieces each).
+        // (one or two 32-k pieces each), for each weight matrix of the tile.
         constexpr int kPieces = KB / 64;   // 32-k pieces per warp and stage
         const int rw = warp - kReconWarp0;
         const int group = rw / kReconGroupWarps;
-        const int quarter = warp & 3, h = (rw % kReconGroupWarps) >> 2;
+        const int quarter = warp & 3, hh = (rw % kReconGroupWarps) >> 2;
         const uint32_t tlane = tacc + ((uint32_t)(32 * quarter) << 16) + p.a_col0;
         SegWalker wk(blockIdx.x, p);
         Segment sg;
@@ -564,10 +633,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 const int s = rp.s;
                 if (!mbar_wait(smem_u32(&full_bar[s]), rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
 #pragma unroll
-                for (int pc = 0; pc < kPieces; pc++) {
-                    const int j = h * kPieces + pc;
-                    rebuild_row<SRC, KB>(p, smem + (size_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
-                                         tlane + (uint32_t)(KB / 2) * (uint32_t)s + 16u * (uint32_t)j);
+                for (int h = 0; h < NH; h++) {
+#pragma unroll
+                    for (int pc = 0; pc < kPieces; pc++) {
+                        const int j = hh * kPieces + pc;
+                        rebuild_row<SRC, KB>(p, p.ps[h], smem + (size_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
+                                             tlane + (uint32_t)(KB / 2) * (uint32_t)(NH * s + h) + 16u * (uint32_t)j);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -594,7 +666,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         const uint32_t trow = tacc + ((uint32_t)(warp * 32) << 16);
         // finisher staging: this warp's 1 + kFinBufs rows-of-32 of fin_cb + 4 floats
         float* fin = reinterpret_cast<float*>(smem) + (size_t)warp * (1 + kFinBufs) * 32 * (p.fin_cb + 4);
-        const int MG4 = p.MG / 4;
+        const int AW4 = p.acc_w / 4;
         bool ok = true;
         while (ok && wk.next(sg)) {
             const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
@@ -615,16 +687,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             tc_fence_after();
             const uint32_t slot = 2u * blockIdx.x + (sg.first ? 0u : 1u);
             if (whole) {
-                for (int c0 = 0; c0 < p.MG; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(trow + (uint32_t)c0, v);
-                    tmem_wait_ld();
-                    store_y(p.Y, p.M, p.N, p.out_f32, v, n, m0 + c0);
-                }
+                write_out(p.Y, p.M, p.N, p.out_f32, p.MG, NH, trow, n, m0);
             } else if (!finisher) {
-                // publish the partial rows
-                float4* dst = reinterpret_cast<float4*>(p.partial) + (size_t)slot * MG4 * kBlockN + r;
-                for (int c0 = 0; c0 < p.MG; c0 += 16) {
+                // publish the partial rows (every accumulator column)
+                float4* dst = reinterpret_cast<float4*>(p.partial) + (size_t)slot * AW4 * kBlockN + r;
+                for (int c0 = 0; c0 < p.acc_w; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(trow + (uint32_t)c0, v);
                     tmem_wait_ld();
@@ -634,7 +701,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                                                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
                 }
             } else {
-                const FinArgs fa = {p.partial, p.Y, p.M, p.N, p.MG, p.fin_cb, p.out_f32, p.total_iters, (uint32_t)p.P, kt};
+                const FinArgs fa = {p.partial, p.Y, p.M, p.N, p.acc_w, p.MG, NH, p.fin_cb, p.out_f32,
+                                    p.total_iters, (uint32_t)p.P, kt};
                 finish_tile(fa, sg.tile, b_last, n, m0, trow, fin, lane);
             }
             tc_fence_before();
@@ -662,8 +730,9 @@ template <int KB>
 __global__ void __launch_bounds__(kThreadsDense, 1)
     k_gemm_dense(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
-                 const GemmParams p) {
-    gemm_body<kSrcDense, KB>(tm_x, tm_a, tm_s2, tm_v, p);
+                 const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
+                 const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
+    gemm_body<kSrcDense, KB, 1>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
 }
 
 // Rebuilding sources: 22 warps held to 72 registers, which leaves one warp's
@@ -672,8 +741,21 @@ template <int SRC, int KB>
 __global__ void __maxnreg__(72)
     k_gemm_recon(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
-                 const GemmParams p) {
-    gemm_body<SRC, KB>(tm_x, tm_a, tm_s2, tm_v, p);
+                 const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
+                 const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
+    gemm_body<SRC, KB, 1>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
+}
+
+// Gate and up projections in one launch (direct palette, SwiGLU epilogue):
+// each stage carries both matrices' tiles for the same rows and k, each
+// tile accumulates into two halves of TMEM.
+template <int KB>
+__global__ void __maxnreg__(72)
+    k_gemm_swiglu(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
+                  const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
+    gemm_body<kSrcPalette, KB, 2>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -773,9 +855,10 @@ unsigned long long gemm_next_epoch() { return next_epoch(); }
 
 int gemm_status_take() { return unit_status_take(); }
 
-GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k) {
+GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k, int nh) {
     GemmSplit g;
     g.MG = pick_mg(M);
+    if (nh == 2 && g.MG > 128) g.MG = 128;   // two accumulators must fit TMEM beside the rebuilt-A ring
     // stage k: 128 for small batch tiles (halves the per-stage TMA, barrier
     // and MMA-issue overhead per weight byte), 64 where a stage is already
     // large (batch tiles above 64 rows)
@@ -810,20 +893,41 @@ GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k) {
     return g;
 }
 
-size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k) {
-    const GemmSplit g = gemm_split(M, N, K, grid, split_k);
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k, int nh) {
+    const GemmSplit g = gemm_split(M, N, K, grid, split_k, nh);
     if (!g.fixup) return 256;
-    size_t part = (size_t)2 * g.P * g.MG * kBlockN * 4;
+    size_t part = (size_t)2 * g.P * nh * g.MG * kBlockN * 4;
     size_t flags = (size_t)2 * g.P * kBlockN * 8;
     return ((part + 255) & ~size_t(255)) + ((flags + 255) & ~size_t(255));
+}
+
+static void set_planes(PlaneSet& ps, const uint8_t* palette, const uint32_t* vbits, const uint32_t* vpre,
+                       const uint8_t* vexp) {
+    ps.vbits = vbits;
+    ps.vpre = vpre;
+    ps.vexp = vexp;
+    ps.pal_small = 1;
+    for (int i = 0; i < 4; i++) ps.pal[i] = 0;
+    if (palette) {
+        for (int i = 0; i < 4; i++)
+            ps.pal[i] = (uint32_t)palette[4 * i] | ((uint32_t)palette[4 * i + 1] << 8) |
+                        ((uint32_t)palette[4 * i + 2] << 16) | ((uint32_t)palette[4 * i + 3] << 24);
+        for (int i = 0; i < 16; i++)
+            if (palette[i] >= 128) ps.pal_small = 0;
+    }
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     *st = UW_OK;
     if (a.M == 0) return cudaSuccess;
     if (a.variant < UW_VARIANT_AUTO || a.variant > UW_VARIANT_GEMV) { *st = UW_ERR_INVALID_ARG; return cudaSuccess; }
-    if (gemv_serves(a)) return launch_gemv(a, s, st);
-    const GemmSplit sp = gemm_split(a.M, a.N, a.K, a.grid, a.split_k);
+    const int NH = a.pair ? 2 : 1;
+    if (a.pair && (a.src != kSrcPalette || a.variant == UW_VARIANT_GEMV || a.band_ready)) {
+        *st = UW_ERR_UNSUPPORTED;
+        return cudaSuccess;
+    }
+    if (!a.pair && gemv_serves(a)) return launch_gemv(a, s, st);
+    const GemmSplit sp = gemm_split(a.M, a.N, a.K, a.grid, a.split_k, NH);
     if (!sp.ok) { *st = a.split_k > 0 ? UW_ERR_INVALID_ARG : UW_ERR_SHAPE; return cudaSuccess; }
     GemmParams p{};
     p.M = a.M;
@@ -831,6 +935,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.K = a.K;
     p.KG = a.K / kGroup;
     p.MG = sp.MG;
+    p.nh = NH;
+    p.acc_w = NH * sp.MG;
     const int KB = sp.KB;
     p.m_tiles = sp.m_tiles;
     p.n_tiles = sp.n_tiles;
@@ -838,18 +944,13 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     const int P = sp.P;
     p.total_iters = (uint32_t)sp.total;
     p.P = P;
-    p.vbits = a.vbits;
-    p.vpre = a.vpre;
-    p.vexp = a.vexp;
-    if (a.palette)
-        for (int i = 0; i < 4; i++)
-            p.pal[i] = (uint32_t)a.palette[4 * i] | ((uint32_t)a.palette[4 * i + 1] << 8) |
-                       ((uint32_t)a.palette[4 * i + 2] << 16) | ((uint32_t)a.palette[4 * i + 3] << 24);
+    set_planes(p.ps[0], a.palette, a.vbits, a.vpre, a.vexp);
+    if (a.pair) set_planes(p.ps[1], a.palette2, a.vbits2, a.vpre2, a.vexp2);
     p.Y = a.Y;
     p.out_f32 = a.out_f32;
-    size_t need = gemm_ws_bytes(a.M, a.N, a.K, a.grid, a.split_k);
+    size_t need = gemm_ws_bytes(a.M, a.N, a.K, a.grid, a.split_k, NH);
     if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
-    size_t part = sp.fixup ? (size_t)2 * P * p.MG * kBlockN * 4 : 0;
+    size_t part = sp.fixup ? (size_t)2 * P * p.acc_w * kBlockN * 4 : 0;
     p.partial = (float*)a.ws;
     p.flags = (unsigned long long*)((uint8_t*)a.ws + ((part + 255) & ~size_t(255)));
     p.epoch = a.epoch ? a.epoch : next_epoch();
@@ -874,15 +975,19 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     } else {
         const uint32_t sm_bytes = kBlockN * KB, idx_bytes = kBlockN * KB / 2, v_bytes = 16 * halves;
         p.off_b = 0;
-        p.off_sm = al1k(b_bytes);
-        p.off_s2 = p.off_sm + sm_bytes;
-        if (a.src == kSrcExponent) {
-            off = p.off_s2 + sm_bytes;
-            p.tx_bytes += 2 * sm_bytes;
-        } else {
-            p.off_v = al1k(p.off_s2 + idx_bytes);
-            off = p.off_v + v_bytes;
-            p.tx_bytes += sm_bytes + idx_bytes + v_bytes;
+        off = al1k(b_bytes);
+        for (int h = 0; h < NH; h++) {
+            PlaneSet& ps = p.ps[h];
+            ps.off_sm = off;
+            ps.off_s2 = ps.off_sm + sm_bytes;
+            if (a.src == kSrcExponent) {
+                off = al1k(ps.off_s2 + sm_bytes);
+                p.tx_bytes += 2 * sm_bytes;
+            } else {
+                ps.off_v = al1k(ps.off_s2 + idx_bytes);
+                off = al1k(ps.off_v + v_bytes);
+                p.tx_bytes += sm_bytes + idx_bytes + v_bytes;
+            }
         }
     }
     p.stage_bytes = al1k(off);
@@ -892,11 +997,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     int S = (int)(budget / p.stage_bytes);
     if (S > kMaxStages) S = kMaxStages;
     if (a.stages >= 2 && S > a.stages) S = a.stages;
-    // TMEM: accumulator columns [0, MG); rebuilt-A stages of 32 columns after it
+    // TMEM: accumulator columns [0, acc_w); rebuilt-A stages of NH * KB/2
+    // columns after it
     uint32_t acc_cols = 32;
-    while (acc_cols < (uint32_t)p.MG) acc_cols <<= 1;
+    while (acc_cols < (uint32_t)p.acc_w) acc_cols <<= 1;
     if (a.src != kSrcDense) {
-        const int s_tmem = (int)((512u - acc_cols) / (uint32_t)(KB / 2));
+        const int s_tmem = (int)((512u - acc_cols) / (uint32_t)(NH * KB / 2));
         if (S > s_tmem) S = s_tmem;
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
@@ -904,23 +1010,19 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     // finisher staging in the idle ring: 4 warps x (1 + kFinBufs) rows-of-32 x (CB + 4) floats
     p.fin_cb = 0;
     for (int cb = 64; cb >= 16; cb >>= 1)
-        if (cb <= p.MG && (size_t)4 * (1 + kFinBufs) * 32 * (cb + 4) * 4 <= (size_t)S * p.stage_bytes) {
+        if (cb <= p.acc_w && (size_t)4 * (1 + kFinBufs) * 32 * (cb + 4) * 4 <= (size_t)S * p.stage_bytes) {
             p.fin_cb = cb;
             break;
         }
     if (p.fin_cb == 0) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.a_col0 = acc_cols;
-    uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + (uint32_t)(KB / 2) * (uint32_t)S;
+    uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + (uint32_t)(NH * KB / 2) * (uint32_t)S;
     p.tmem_cols = 32;
     while (p.tmem_cols < need_cols) p.tmem_cols <<= 1;
     if (p.tmem_cols > 512) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
-    p.pal_small = 1;
-    if (a.palette)
-        for (int i = 0; i < 16; i++)
-            if (a.palette[i] >= 128) p.pal_small = 0;
     size_t smem = (size_t)S * p.stage_bytes + ctrl + 1024;
 
-    CUtensorMap tx{}, ta{}, ts2{}, tv{};
+    CUtensorMap tx{}, ta{}, ts2{}, tv{}, ta2{}, ts22{}, tv2{};
     bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBoxK, p.MG,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (a.src == kSrcDense) {
@@ -932,24 +1034,37 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
         // byte planes: rows of KB bytes (swizzle KB), index rows of KB/2 bytes
         const CUtensorMapSwizzle swz = KB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
         const CUtensorMapSwizzle swz_i = KB == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-        ok = ok && make_map_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sm, a.K, a.N, a.K, KB, kBlockN, swz);
-        if (a.src == kSrcExponent) {
-            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, KB, kBlockN, swz);
-            tv = ts2;
-        } else {
-            int64_t NW = 4 * ((a.N + 127) / 128);
-            ok = ok && make_map_2d(&ts2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.idx, a.K / 2, a.N, a.K / 2, KB / 2,
-                                   kBlockN, swz_i);
-            ok = ok && make_map_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.vcol, NW, a.K / kGroup, NW * 4, 4,
-                                   KB / kGroup, CU_TENSOR_MAP_SWIZZLE_NONE);
+        const int64_t NW = 4 * ((a.N + 127) / 128);
+        for (int h = 0; h < NH; h++) {
+            CUtensorMap* m_a = h ? &ta2 : &ta;
+            CUtensorMap* m_s2 = h ? &ts22 : &ts2;
+            CUtensorMap* m_v = h ? &tv2 : &tv;
+            const uint8_t* sm = h ? a.sm2 : a.sm;
+            ok = ok && make_map_2d(m_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sm, a.K, a.N, a.K, KB, kBlockN, swz);
+            if (a.src == kSrcExponent) {
+                ok = ok && make_map_2d(m_s2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.ex, a.K, a.N, a.K, KB, kBlockN, swz);
+                *m_v = *m_s2;
+            } else {
+                ok = ok && make_map_2d(m_s2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h ? a.idx2 : a.idx, a.K / 2, a.N, a.K / 2,
+                                       KB / 2, kBlockN, swz_i);
+                ok = ok && make_map_2d(m_v, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, h ? a.vcol2 : a.vcol, NW, a.K / kGroup,
+                                       NW * 4, 4, KB / kGroup, CU_TENSOR_MAP_SWIZZLE_NONE);
+            }
         }
+    }
+    if (NH == 1) {
+        ta2 = ta;
+        ts22 = ts2;
+        tv2 = tv;
     }
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
 
     typedef void (*GemmKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                               const GemmParams);
+                               const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams);
     GemmKernel kern;
-    if (KB == 128)
+    if (a.pair)
+        kern = KB == 128 ? k_gemm_swiglu<128> : k_gemm_swiglu<64>;
+    else if (KB == 128)
         kern = a.src == kSrcDense      ? k_gemm_dense<128>
                : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent, 128>
                                        : k_gemm_recon<kSrcPalette, 128>;
@@ -969,7 +1084,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tx, ta, ts2, tv, p);
+    e = cudaLaunchKernelEx(&cfg, kern, tx, ta, ts2, tv, ta2, ts22, tv2, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1028,7 +1143,7 @@ extern "C" uw_status uw_gemm_direct_palette_noalloc(const uint16_t* X, int64_t M
     if (!(b->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
     if (M == 0) return UW_OK;
     if (!X || !Y || ((uintptr_t)X & 15) || ((uintptr_t)Y & 15)) return UW_ERR_INVALID_ARG;
-    if (gemm_ws_bytes(M, b->geo.N, b->geo.K, 0, 0) > kNoAllocScratchBytes) return UW_ERR_WORKSPACE;
+    if (gemm_ws_bytes(M, b->geo.N, b->geo.K, 0, 0, 1) > kNoAllocScratchBytes) return UW_ERR_WORKSPACE;
     uw_status st = UW_OK;
     void* scratch = noalloc_scratch(&st);
     if (!scratch) return st;

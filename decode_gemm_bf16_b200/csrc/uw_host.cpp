@@ -642,7 +642,9 @@ static size_t decode_buffer_bytes(const uw_blob* b, int pipeline) {
     }
 }
 
-static bool runs_beside(const uw_gemm_opts* o) { return o->sm_dec > 0 && o->pipeline != UW_PIPE_DIRECT_PALETTE; }
+static bool runs_beside(const uw_gemm_opts* o) {
+    return o->sm_dec > 0 && o->pipeline != UW_PIPE_DIRECT_PALETTE && o->pipeline != UW_PIPE_FUSED_HUFFMAN;
+}
 
 static size_t band_counter_bytes(const uw_blob* b) { return al256((uint64_t)((b->geo.N + 127) / 128) * 8); }
 
@@ -661,7 +663,7 @@ extern "C" uw_status uw_plan_resolve(const uw_gemm_opts* o, int64_t M, uw_gemm_o
         if (!lowest || e.M < lowest->M) lowest = &e;
     }
     const uw_plan_entry* e = exact ? exact : below ? below : lowest;
-    if (!e || e->pipeline < UW_PIPE_FULL || e->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (!e || e->pipeline < UW_PIPE_FULL || e->pipeline > UW_PIPE_FUSED_HUFFMAN) return UW_ERR_INVALID_ARG;
     out->pipeline = e->pipeline;
     out->variant = e->variant;
     out->sm_dec = e->sm_dec;
@@ -673,7 +675,7 @@ extern "C" uw_status uw_plan_resolve(const uw_gemm_opts* o, int64_t M, uw_gemm_o
 }
 
 static uw_status check_opts(const uw_gemm_opts* o) {
-    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_DIRECT_PALETTE) return UW_ERR_INVALID_ARG;
+    if (o->pipeline < UW_PIPE_FULL || o->pipeline > UW_PIPE_FUSED_HUFFMAN) return UW_ERR_INVALID_ARG;
     if (o->sm_dec < 0 || o->grid < 0 || o->split_k < 0 || o->stages < 0) return UW_ERR_INVALID_ARG;
     if (o->variant < UW_VARIANT_AUTO || o->variant > UW_VARIANT_GEMV) return UW_ERR_INVALID_ARG;
     return UW_OK;
@@ -690,6 +692,10 @@ extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gem
     st = check_opts(o);
     if (st) return st;
     if (M == 0) { *bytes = 0; return UW_OK; }
+    if (o->pipeline == UW_PIPE_FUSED_HUFFMAN) {
+        *bytes = al256(fused_ws_bytes(M, b->geo.N, b->geo.K));
+        return UW_OK;
+    }
     *bytes = decode_buffer_bytes(b, o->pipeline) + al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, o->grid, o->split_k)) +
              (runs_beside(o) ? band_counter_bytes(b) : 0);
     return UW_OK;
@@ -701,6 +707,8 @@ extern "C" uw_status uw_gemm_workspace(const uw_blob* b, int64_t M, const uw_gem
 struct SideStream {
     cudaStream_t s = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t done[2] = {nullptr, nullptr};    // layer sequences: decode buffer b filled
+    cudaEvent_t freed[2] = {nullptr, nullptr};   // layer sequences: decode buffer b read by its GEMM
 };
 static SideStream* side_stream(uw_status* st) {
     static std::mutex mu;
@@ -714,9 +722,13 @@ static SideStream* side_stream(uw_status* st) {
     std::lock_guard<std::mutex> lock(mu);
     SideStream& ss = per_dev[dev];
     if (!ss.s) {
-        if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+        bool ok = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) == cudaSuccess;
+        for (int b = 0; b < 2 && ok; b++)
+            ok = cudaEventCreateWithFlags(&ss.done[b], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&ss.freed[b], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
             cudaGetLastError();
             *st = UW_ERR_CUDA;
             return nullptr;
@@ -758,6 +770,19 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     uint8_t* ws = (uint8_t*)o->workspace;
+    if (o->pipeline == UW_PIPE_FUSED_HUFFMAN) {
+        // one pass per kFusedMaxM batch rows; each pass decodes the stream again
+        if (b->geo.K % kSeg) return UW_ERR_UNSUPPORTED;
+        const size_t ysz = o->out_f32 ? 4 : 2;
+        for (int64_t m0 = 0; m0 < M; m0 += kFusedMaxM) {
+            const int64_t mc = M - m0 < kFusedMaxM ? M - m0 : kFusedMaxM;
+            cudaError_t e = launch_fused_huffman(b, X + m0 * b->geo.K, mc, (uint8_t*)Y + (size_t)m0 * b->geo.N * ysz,
+                                                 o->out_f32 ? 1 : 0, ws, o->workspace_bytes, s, &st);
+            if (st) return st;
+            if (cuda_ok(e)) return UW_ERR_CUDA;
+        }
+        return UW_OK;
+    }
     const size_t dbuf = decode_buffer_bytes(b, o->pipeline);
 
     GemmArgs a;
@@ -826,6 +851,197 @@ extern "C" uw_status uw_gemm(const uint16_t* X, int64_t M, const uw_blob* b, voi
     return cuda_ok(e);
 }
 
+// ===========================================================================
+// layer sequences with "hard" and "easy" projections (§跨層管道化)
+// ===========================================================================
+// Workspace: two index-plane buffers (the largest hard item's plane each)
+// then the GEMM scratch (the largest item's), shared by the items in turn.
+static void sequence_layout(const uw_seq_item* items, int n, int64_t M, size_t* plane, size_t* gemm) {
+    *plane = 0;
+    *gemm = 0;
+    for (int i = 0; i < n; i++) {
+        const uw_blob* b = items[i].blob;
+        if (items[i].hard) *plane = std::max(*plane, (size_t)al256(b->geo.n / 2));
+        *gemm = std::max(*gemm, (size_t)al256(gemm_ws_bytes(M, b->geo.N, b->geo.K, 0, 0)));
+    }
+}
+
+static uw_status sequence_check(const uw_seq_item* items, int n, int64_t M, bool need_ptrs) {
+    if (!items || n < 1 || M < 0) return UW_ERR_INVALID_ARG;
+    for (int i = 0; i < n; i++) {
+        uw_status st = check_committed(items[i].blob);
+        if (st) return st;
+        const unsigned need = items[i].hard ? UW_FORM_HUFFMAN : UW_FORM_PALETTE;
+        if (!(items[i].blob->forms & need)) return UW_ERR_UNSUPPORTED;
+        if (need_ptrs && M > 0 &&
+            (!items[i].X || !items[i].Y || !aligned(items[i].X, 16) || !aligned(items[i].Y, 16)))
+            return UW_ERR_INVALID_ARG;
+    }
+    return UW_OK;
+}
+
+extern "C" uw_status uw_sequence_workspace(const uw_seq_item* items, int n, int64_t M, size_t* bytes) {
+    if (!bytes) return UW_ERR_INVALID_ARG;
+    uw_status st = sequence_check(items, n, M, false);
+    if (st) return st;
+    size_t plane = 0, gemm = 0;
+    sequence_layout(items, n, M, &plane, &gemm);
+    *bytes = M ? 2 * plane + gemm : 0;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_gemm_sequence(const uw_seq_item* items, int n, int64_t M, int out_f32, int dec_ctas,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+    uw_status st = sequence_check(items, n, M, true);
+    if (st) return st;
+    if (dec_ctas < 0) return UW_ERR_INVALID_ARG;
+    if (M == 0) return UW_OK;
+    size_t plane = 0, gemm = 0;
+    sequence_layout(items, n, M, &plane, &gemm);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < 2 * plane + gemm) return UW_ERR_WORKSPACE;
+    uint8_t* ws = (uint8_t*)workspace;
+    uint8_t* buf[2] = {ws, ws + plane};
+    uint8_t* gws = ws + 2 * plane;
+    cudaStream_t s = (cudaStream_t)stream;
+    bool any_hard = false;
+    for (int i = 0; i < n; i++) any_hard = any_hard || items[i].hard;
+    SideStream* ss = nullptr;
+    if (any_hard) {
+        ss = side_stream(&st);
+        if (!ss) return st;
+        // decodes write this call's buffers: after the work already on `stream`
+        if (cuda_ok(cudaEventRecord(ss->fork, s)) || cuda_ok(cudaStreamWaitEvent(ss->s, ss->fork, 0)))
+            return UW_ERR_CUDA;
+    }
+    // with decoder CTAs beside the GEMMs, every GEMM leaves room for one
+    const int smem_cap = dec_ctas > 0 ? 228 * 1024 - kDecodeBesideSmem - 2048 : 0;
+    int h = 0;                 // hard items so far
+    for (int i = 0; i < n; i++) {
+        const uw_seq_item& it = items[i];
+        const uw_blob* b = it.blob;
+        GemmArgs a;
+        a.src = kSrcPalette;
+        a.X = it.X;
+        a.M = M;
+        a.N = b->geo.N;
+        a.K = b->geo.K;
+        a.Y = it.Y;
+        a.out_f32 = out_f32 ? 1 : 0;
+        a.variant = UW_VARIANT_TENSOR;
+        a.ws = gws;
+        a.ws_bytes = gemm;
+        a.sm = b->sec(UW_SEC_SM);
+        a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
+        a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
+        a.vexp = b->sec(UW_SEC_VEXP);
+        a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
+        a.palette = b->palette;
+        a.static_sm = 1;
+        a.smem_cap = smem_cap;
+        if (it.hard) {
+            // the transcode of this item runs on the side stream as soon as its
+            // buffer's previous GEMM (two hard items back) has read it, i.e.
+            // ahead of the GEMMs in between
+            const int bi = h & 1;
+            if (h >= 2 && cuda_ok(cudaStreamWaitEvent(ss->s, ss->freed[bi], 0))) return UW_ERR_CUDA;
+            cudaError_t e = dec_ctas > 0 ? launch_decode_beside(b, kDecodeTranscode, buf[bi], dec_ctas, nullptr, 0, ss->s)
+                                         : launch_decode(b, kDecodeTranscode, buf[bi], 0, ss->s);
+            if (cuda_ok(e) || cuda_ok(cudaEventRecord(ss->done[bi], ss->s)) ||
+                cuda_ok(cudaStreamWaitEvent(s, ss->done[bi], 0)))
+                return UW_ERR_CUDA;
+            a.idx = buf[bi];
+            a.static_s2 = 0;
+            cudaError_t eg = launch_gemm(a, s, &st);
+            if (st) return st;
+            if (cuda_ok(eg) || cuda_ok(cudaEventRecord(ss->freed[bi], s))) return UW_ERR_CUDA;
+            h++;
+        } else {
+            a.idx = b->sec(UW_SEC_IDX);
+            a.static_s2 = 1;
+            cudaError_t eg = launch_gemm(a, s, &st);
+            if (st) return st;
+            if (cuda_ok(eg)) return UW_ERR_CUDA;
+        }
+    }
+    if (any_hard) {
+        // the side stream joins back (its last decode is already awaited by a GEMM)
+        if (cuda_ok(cudaEventRecord(ss->join, ss->s)) || cuda_ok(cudaStreamWaitEvent(s, ss->join, 0)))
+            return UW_ERR_CUDA;
+    }
+    return UW_OK;
+}
+
+// ===========================================================================
+// gate + up with the SwiGLU epilogue (§未來方向)
+// ===========================================================================
+static uw_status swiglu_check(const uw_blob* g, const uw_blob* u, int64_t M, const uw_gemm_opts* o) {
+    uw_status st = check_committed(g);
+    if (st) return st;
+    st = check_committed(u);
+    if (st) return st;
+    if (!o || M < 0) return UW_ERR_INVALID_ARG;
+    st = check_opts(o);
+    if (st) return st;
+    if (g->geo.N != u->geo.N || g->geo.K != u->geo.K) return UW_ERR_SHAPE;
+    if (o->pipeline != UW_PIPE_DIRECT_PALETTE || o->variant == UW_VARIANT_GEMV || o->sm_dec != 0)
+        return UW_ERR_UNSUPPORTED;
+    if (!(g->forms & UW_FORM_PALETTE) || !(u->forms & UW_FORM_PALETTE)) return UW_ERR_UNSUPPORTED;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_gemm_swiglu_workspace(const uw_blob* g, const uw_blob* u, int64_t M, const uw_gemm_opts* o,
+                                              size_t* bytes) {
+    if (!bytes) return UW_ERR_INVALID_ARG;
+    uw_status st = swiglu_check(g, u, M, o);
+    if (st) return st;
+    *bytes = M ? al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 2)) : 0;
+    return UW_OK;
+}
+
+extern "C" uw_status uw_gemm_swiglu(const uint16_t* X, int64_t M, const uw_blob* g, const uw_blob* u, void* H,
+                                    const uw_gemm_opts* o, void* stream) {
+    uw_status st = swiglu_check(g, u, M, o);
+    if (st) return st;
+    if (M == 0) return UW_OK;
+    if (!X || !H || !aligned(X, 16) || !aligned(H, 16)) return UW_ERR_INVALID_ARG;
+    const size_t need = al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 2));
+    if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
+    GemmArgs a;
+    a.src = kSrcPalette;
+    a.pair = 1;
+    a.X = X;
+    a.M = M;
+    a.N = g->geo.N;
+    a.K = g->geo.K;
+    a.Y = H;
+    a.out_f32 = o->out_f32 ? 1 : 0;
+    a.variant = o->variant;
+    a.grid = o->grid;
+    a.split_k = o->split_k;
+    a.stages = o->stages;
+    a.ws = o->workspace;
+    a.ws_bytes = o->workspace_bytes;
+    a.static_sm = 1;
+    a.static_s2 = 1;
+    a.sm = g->sec(UW_SEC_SM);
+    a.idx = g->sec(UW_SEC_IDX);
+    a.vbits = (const uint32_t*)g->sec(UW_SEC_VBITS);
+    a.vpre = (const uint32_t*)g->sec(UW_SEC_VPRE);
+    a.vexp = g->sec(UW_SEC_VEXP);
+    a.vcol = (const uint32_t*)g->sec(UW_SEC_VCOL);
+    a.palette = g->palette;
+    a.sm2 = u->sec(UW_SEC_SM);
+    a.idx2 = u->sec(UW_SEC_IDX);
+    a.vbits2 = (const uint32_t*)u->sec(UW_SEC_VBITS);
+    a.vpre2 = (const uint32_t*)u->sec(UW_SEC_VPRE);
+    a.vexp2 = u->sec(UW_SEC_VEXP);
+    a.vcol2 = (const uint32_t*)u->sec(UW_SEC_VCOL);
+    a.palette2 = u->palette;
+    cudaError_t e = launch_gemm(a, (cudaStream_t)stream, &st);
+    if (st) return st;
+    return cuda_ok(e);
+}
+
 extern "C" uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int variant, int grid, int split_k,
                                              size_t* bytes) {
     if (!bytes || M < 0 || grid < 0 || split_k < 0) return UW_ERR_INVALID_ARG;
@@ -871,7 +1087,7 @@ extern "C" uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t*
 // ===========================================================================
 namespace {
 
-const char* kPipeNames[] = {"full", "exponent", "transcode", "direct_palette"};
+const char* kPipeNames[] = {"full", "exponent", "transcode", "direct_palette", "fused_huffman"};
 
 struct Cand {
     int pipe, variant, grid, split_k, sm_dec;
@@ -900,6 +1116,7 @@ struct PathKey {
 };
 
 PathKey path_of(const Cand& c, const uw_blob* b, int64_t M) {
+    if (c.pipe == UW_PIPE_FUSED_HUFFMAN) return PathKey{c.pipe, 0, 0, 0};
     GemmArgs a;
     a.M = M;
     a.N = b->geo.N;
@@ -928,6 +1145,7 @@ std::vector<Cand> candidates(const uw_blob* b, int64_t M, size_t wsb) {
         if (pp != UW_PIPE_DIRECT_PALETTE)
             for (int f : {1, 2, 4}) raw.push_back({pp, UW_VARIANT_AUTO, 0, 0, f * sms / 2});
     }
+    if (M <= kFusedMaxM && b->geo.K % kSeg == 0) raw.push_back({UW_PIPE_FUSED_HUFFMAN, UW_VARIANT_AUTO, 0, 0, 0});
     std::vector<Cand> out;
     std::vector<PathKey> seen;
     for (const Cand& c : raw) {
@@ -1138,12 +1356,12 @@ extern "C" uw_status uw_plan_load_json(const char* path, uw_plan_entry* entries,
         e.M = atoll(v.c_str());
         if (!json_field(obj, "pipeline", &v)) return UW_ERR_CORRUPT;
         e.pipeline = -1;
-        for (int k = 0; k < 4; k++)
+        for (int k = 0; k <= UW_PIPE_FUSED_HUFFMAN; k++)
             if (v == kPipeNames[k]) e.pipeline = k;
         if (e.pipeline < 0) {
             char* q = nullptr;
             long pv = strtol(v.c_str(), &q, 10);
-            if (q == v.c_str() || pv < UW_PIPE_FULL || pv > UW_PIPE_DIRECT_PALETTE) return UW_ERR_CORRUPT;
+            if (q == v.c_str() || pv < UW_PIPE_FULL || pv > UW_PIPE_FUSED_HUFFMAN) return UW_ERR_CORRUPT;
             e.pipeline = (int32_t)pv;
         }
         if (json_field(obj, "variant", &v)) e.variant = atoi(v.c_str());

@@ -114,6 +114,13 @@ cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas
                                  unsigned long long epoch, cudaStream_t s);
 constexpr int kDecodeBesideSmem = (1 << 12) * 4 + 4 * 32 * 32 * 4;   // LUT + 4 warps of staging
 int decode_ctas_per_sm();
+// Fused Huffman-decode GEMV/small-batch product (no decoded plane in HBM):
+// Y[M,N] = X[M,K] . W^T straight from the Huffman form, M <= kFusedMaxM per
+// launch, K a multiple of 256.  Workspace: fused_ws_bytes.
+constexpr int kFusedMaxM = 16;
+size_t fused_ws_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M, void* Y, int out_f32, void* ws,
+                                 size_t ws_bytes, cudaStream_t s, uw_status* st);
 
 // ---- GEMM (uw_gemm.cu)
 enum GemmSource { kSrcDense = 0, kSrcExponent = 1, kSrcPalette = 2 };
@@ -144,6 +151,16 @@ struct GemmArgs {
     int64_t band_tasks = 0, ntasks = 0;
     int static_sm = 0;                // sm plane and verbatim flags read from the committed blob (no kernel writes it)
     int static_s2 = 0;                // second plane too (the stored index plane)
+    // paired call (gate and up, direct palette, SwiGLU epilogue): the up
+    // projection's planes; Y = silu(X.Wg^T) * (X.Wu^T)
+    int pair = 0;
+    const uint8_t* sm2 = nullptr;
+    const uint8_t* idx2 = nullptr;
+    const uint32_t* vbits2 = nullptr;
+    const uint32_t* vpre2 = nullptr;
+    const uint8_t* vexp2 = nullptr;
+    const uint32_t* vcol2 = nullptr;
+    const uint8_t* palette2 = nullptr;
 };
 // Work split of the tensor-core kernel: batch tile MG, stage k KB, tiles,
 // (tile, k step) iterations and CTA count P.  fixup: some tile is cut
@@ -154,8 +171,8 @@ struct GemmSplit {
     int64_t tiles = 0, total = 0;
     bool fixup = false, ok = true;
 };
-GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k);
-size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k);
+GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k, int nh = 1);
+size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k, int nh = 1);
 // Tensor-core GEMM; the calls gemv_serves() accepts (by the variant, or with
 // UW_VARIANT_AUTO batch 1 on a projection with few 128-row tiles and no
 // decoder beside) go to the CUDA-core GEMV instead.

@@ -56,15 +56,26 @@ typedef enum {
     UW_ERR_DEVICE = 8        /* a device-side check failed (bad stream data)  */
 } uw_status;
 
-/* The four pipelines of §四種執行管道, and the autotuned choice of
- * §自動調優機制 (UW_PIPE_AUTO: the plan given in the options picks the
- * pipeline and matmul settings for this projection and batch size). */
+/* The four pipelines of §四種執行管道, a fifth that decodes the Huffman
+ * stream inside the product (the pages could not fit the decode table beside
+ * the Hopper matmul's buffers, §解壓與運算資源共享), and the autotuned
+ * choice of §自動調優機制 (UW_PIPE_AUTO: the plan given in the options picks
+ * the pipeline and matmul settings for this projection and batch size). */
 typedef enum {
     UW_PIPE_AUTO = -1,           /* resolved through uw_gemm_opts.plan (see uw_plan_resolve)  */
     UW_PIPE_FULL = 0,            /* Huffman full decode -> BF16 W in workspace -> dense GEMM  */
     UW_PIPE_EXPONENT = 1,        /* Huffman exponent decode -> E in workspace -> reconstructive GEMM */
     UW_PIPE_TRANSCODE = 2,       /* Huffman -> 4-bit index plane in workspace -> reconstructive GEMM */
-    UW_PIPE_DIRECT_PALETTE = 3   /* reconstructive GEMM straight from the stored index plane */
+    UW_PIPE_DIRECT_PALETTE = 3,  /* reconstructive GEMM straight from the stored index plane */
+    UW_PIPE_FUSED_HUFFMAN = 4    /* an addition to the four: the Huffman stream decoded inside the
+                                    product itself (no decoded plane in HBM); CUDA cores, batches of
+                                    up to 16 rows per pass (larger M: one pass per 16 rows); needs
+                                    the Huffman form and K a multiple of 256 (else
+                                    UW_ERR_UNSUPPORTED); variant, grid, split_k and sm_dec are
+                                    ignored.  Its summation order differs from the other
+                                    pipelines' (k ranges of 256-weight segments per warp, added in
+                                    order), so it agrees with them within the GEMM tolerance, not
+                                    bit for bit; it does not depend on the launch. */
 } uw_pipeline;
 
 /* Matmul variant: which kernel family computes the product. */
@@ -277,6 +288,56 @@ uw_status uw_dense_gemm_workspace(int64_t M, int64_t N, int64_t K, int variant, 
 uw_status uw_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K,
                         void* Y, int out_f32, int variant, int grid, int split_k, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- layer sequences
+ * §跨層管道化: layers whose weights need a runtime Huffman decode ("hard")
+ * alternate with layers kept in the pre-converted palette form ("easy"), so
+ * that decompression never runs twice in a row and the decode of a hard
+ * layer overlaps the matmul of the easy layer before it.  uw_gemm_sequence
+ * runs a list of projections in order on `stream` (item i may read what item
+ * i-1 wrote); every hard item's palette transcode runs on a library side
+ * stream into one of two workspace buffers, as early as its buffer allows
+ * (after the GEMM of the hard item two before it), and its GEMM waits for
+ * it.  dec_ctas > 0: the transcodes run as that many small decoder CTAs that
+ * fit beside the GEMM CTAs (which then leave room for one), so decode and
+ * matmul share the SMs; 0: the standalone decoder.  The result of each item
+ * equals uw_gemm of that item alone (transcode pipeline for hard items,
+ * direct palette for easy ones, tensor cores) bit for bit.  Items on one
+ * device that run beside each other in two calls at once must not overlap
+ * (they share the side stream's events). */
+typedef struct {
+    const uw_blob* blob;
+    const uint16_t* X;       /* device BF16 [M, K]                                       */
+    void* Y;                 /* device [M, N], BF16 or float32 (out_f32)                 */
+    int32_t hard;            /* 1: from the Huffman form (needs it); 0: from the palette form */
+} uw_seq_item;
+
+uw_status uw_sequence_workspace(const uw_seq_item* items, int n, int64_t M, size_t* bytes);
+
+uw_status uw_gemm_sequence(const uw_seq_item* items, int n, int64_t M, int out_f32, int dec_ctas,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- gate + up, SwiGLU
+ * §未來方向 names SwiGLU as the activation of the MLP: the gate and up
+ * projections read the same X, and the down projection reads
+ *   H[M,N] = silu(X . Wg^T) * (X . Wu^T),   silu(z) = z / (1 + e^-z).
+ * uw_gemm_swiglu computes H in one launch from the palette forms of both
+ * matrices: every tile of 128 rows carries the gate and the up rows, each
+ * stage stages both matrices' tiles, TMEM holds two accumulators, and the
+ * epilogue applies the SwiGLU in float32 before rounding H to BF16 (or
+ * writing float32 with out_f32).  X is read once per tile for both products
+ * and neither product goes to HBM.
+ *   gate, up: committed blobs of the same shape [N, K] holding the palette
+ *     form; X: device BF16 [M, K]; H: device [M, N].
+ *   opts: pipeline UW_PIPE_DIRECT_PALETTE (others: UW_ERR_UNSUPPORTED),
+ *     variant UW_VARIANT_AUTO or UW_VARIANT_TENSOR, sm_dec 0; grid, split_k,
+ *     stages, out_f32 and the workspace as in uw_gemm.  Batch tiles are at
+ *     most 128 rows (two accumulators share TMEM with the rebuilt tiles). */
+uw_status uw_gemm_swiglu_workspace(const uw_blob* gate, const uw_blob* up, int64_t M, const uw_gemm_opts* opts,
+                                   size_t* bytes);
+
+uw_status uw_gemm_swiglu(const uint16_t* X, int64_t M, const uw_blob* gate, const uw_blob* up, void* H,
+                         const uw_gemm_opts* opts, void* stream);
 
 /* ---------------------------------------------------------------- allocation-free GEMM
  * An addition of this library; the pages have no counterpart.

@@ -119,7 +119,7 @@ def _sampled(X, W, Y, n_samples, seed, bf16_out):
     ns = rng.integers(0, N, n_samples)
     ref = np.array([O.gemm_one(X, W, int(m), int(n), "f32") for m, n in zip(ms, ns)])
     # floor from the sampled references' scale
-    check_gemm(Y[ms, ns], ref, bf16_out=bf16_out)
+    check_gemm(Y[ms, ns], ref, bf16_out=bf16_out, K=W.shape[1])
 
 
 @pytest.fixture(scope="module")
@@ -139,20 +139,21 @@ def _full_size_all_paths(W, blob, M, seed):
     float32 outputs, against the oracle's fp32-accumulated product."""
     X = S.activations(M, W.shape[1], seed=seed)
     R = oracle_gemm(X, W, "f32")
+    K = W.shape[1]
     Xd = dev16(X)
     ref = None
     for pipe in PIPES:
         Yb = _f32(uw.uw_gemm(Xd, blob, pipe))
-        check_gemm(Yb, R, bf16_out=True)
+        check_gemm(Yb, R, bf16_out=True, K=K)
         if ref is None:
             ref = Yb
         assert np.array_equal(Yb, ref), pipe
-    check_gemm(_f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True)), R, bf16_out=False)
+    check_gemm(_f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True)), R, bf16_out=False, K=K)
     Wd = dev16(W)
     Yd = _f32(uw.uw_dense_gemm(Xd, Wd))
-    check_gemm(Yd, R, bf16_out=True)
+    check_gemm(Yd, R, bf16_out=True, K=K)
     assert np.array_equal(Yd, ref)
-    check_gemm(_f32(uw.uw_dense_gemm(Xd, Wd, out_f32=True)), R, bf16_out=False)
+    check_gemm(_f32(uw.uw_dense_gemm(Xd, Wd, out_f32=True)), R, bf16_out=False, K=K)
     assert uw.uw_last_device_status() == 0
 
 
@@ -386,3 +387,249 @@ def test_bounded_wait_expires_with_timeout_status():
     assert int(lines["status"]) == 7          # UW_ERR_TIMEOUT
     after = lines["after"].split()
     assert int(after[0]) == 0 and float(after[1]) < 1e-2
+
+
+# ---------------------------------------------------------------------------
+# Fused Huffman-decode product (UW_PIPE_FUSED_HUFFMAN): the stream is decoded
+# inside the product, no decoded plane goes to HBM.
+# ---------------------------------------------------------------------------
+FUSED_SHAPES = {
+    "384x512": lambda: S.weight_with_verbatim_rows(384, 512, seed=31, frac_groups=0.01),
+    "200x1024": lambda: S.weight_with_verbatim_rows(200, 1024, seed=34, frac_groups=0.02),
+    "high_entropy_96x4096": lambda: _high_entropy_rows(96, 4096),
+}
+
+
+def _high_entropy_rows(N, K):
+    rng = np.random.default_rng(12)
+    W = S.gaussian_weight(N, K, seed=24)
+    ex = rng.integers(112, 128, 32 * K).astype(np.uint16)
+    W[:32] = ((ex << 7) | rng.integers(0, 0x8080, 32 * K).astype(np.uint16) & 0x807F).reshape(32, K)
+    return W
+
+
+_fcache = {}
+
+
+def _fcase(shape):
+    if shape not in _fcache:
+        W = FUSED_SHAPES[shape]()
+        _fcache[shape] = (W, uw.uw_compress(dev16(W)))
+    return _fcache[shape]
+
+
+@pytest.mark.parametrize("shape", list(FUSED_SHAPES))
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 17, 40])
+def test_fused_huffman_matches_oracle(shape, M):
+    W, blob = _fcase(shape)
+    X = S.activations(M, W.shape[1], seed=2000 + M)
+    R32 = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    Y32 = _f32(uw.uw_gemm(Xd, blob, "fused_huffman", out_f32=True))
+    check_gemm(Y32, R32, bf16_out=False)
+    check_gemm(Y32, O.gemm(X, W, "f64"), bf16_out=False)
+    Yb = _f32(uw.uw_gemm(Xd, blob, "fused_huffman"))
+    check_gemm(Yb, R32, bf16_out=True)
+    # deterministic: the same call gives the same bits
+    assert np.array_equal(_f32(uw.uw_gemm(Xd, blob, "fused_huffman", out_f32=True)), Y32)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_fused_huffman_graph_replays():
+    """Captured once and replayed: the per-call tag is reused, so the last
+    warp of each row group resets its counter; every replay must match."""
+    W, blob = _fcase("200x1024")
+    X = S.activations(4, 1024, seed=2100)
+    R = O.gemm(X, W, "f32")
+    Xd = dev16(X)
+    Y = torch.empty(4, 200, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(uw.uw_gemm_workspace(blob, 4, "fused_huffman"), dtype=torch.uint8, device="cuda")
+    uw.uw_gemm(Xd, blob, "fused_huffman", out=Y, out_f32=True, ws=ws)
+    torch.cuda.synchronize()
+    first = _f32(Y)
+    check_gemm(first, R, bf16_out=False)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        uw.uw_gemm(Xd, blob, "fused_huffman", out=Y, out_f32=True, ws=ws)
+    for _ in range(3):
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(_f32(Y), first)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_fused_huffman_rejects_unsupported():
+    W, blob = _case("200x1408")            # K = 1408 is not a multiple of 256
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm(dev16(S.activations(2, 1408, 1)), blob, "fused_huffman")
+    assert ei.value.status == 4
+    Wp, _ = _fcase("384x512")
+    bp = uw.uw_compress(dev16(Wp), forms=uw.UW_FORM_PALETTE)   # no Huffman form
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm(dev16(S.activations(2, 512, 1)), bp, "fused_huffman")
+    assert ei.value.status == 4
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_fused_huffman_full_size_gate(gate_case, M):
+    W, blob = gate_case
+    X = S.activations(M, 4096, seed=2200 + M)
+    R = oracle_gemm(X, W, "f32")
+    check_gemm(_f32(uw.uw_gemm(dev16(X), blob, "fused_huffman")), R, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_fused_huffman_full_size_down(down_case, M):
+    W, blob = down_case
+    X = S.activations(M, 14336, seed=2300 + M)
+    R = oracle_gemm(X, W, "f32")
+    check_gemm(_f32(uw.uw_gemm(dev16(X), blob, "fused_huffman")), R, bf16_out=True, K=14336)
+    assert uw.uw_last_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# Gate + up in one launch with the SwiGLU epilogue (uw_gemm_swiglu)
+# ---------------------------------------------------------------------------
+SWIGLU_PAIRS = {
+    "384x512": lambda: (S.weight_with_verbatim_rows(384, 512, seed=51, frac_groups=0.01),
+                        S.weight_with_verbatim_rows(384, 512, seed=52, frac_groups=0.01)),
+    "200x1408": lambda: (S.weight_with_verbatim_rows(200, 1408, seed=53, frac_groups=0.01),
+                         S.gaussian_weight(200, 1408, seed=54, std=0.03)),
+}
+_scache = {}
+
+
+def _scase(name):
+    if name not in _scache:
+        Wg, Wu = SWIGLU_PAIRS[name]()
+        _scache[name] = (Wg, Wu, uw.uw_compress(dev16(Wg)), uw.uw_compress(dev16(Wu)))
+    return _scache[name]
+
+
+@pytest.mark.parametrize("name", list(SWIGLU_PAIRS))
+@pytest.mark.parametrize("M", [1, 3, 16, 17, 64, 100, 128, 129, 300])
+def test_swiglu_matches_oracle(name, M):
+    from tests.gpu_util import check_swiglu
+    Wg, Wu, bg, bu = _scase(name)
+    X = S.activations(M, Wg.shape[1], seed=3000 + M)
+    G = O.gemm(X, Wg, "f32")
+    U = O.gemm(X, Wu, "f32")
+    Xd = dev16(X)
+    H32 = _f32(uw.uw_gemm_swiglu(Xd, bg, bu, out_f32=True))
+    check_swiglu(H32, G, U, bf16_out=False)
+    Hb = _f32(uw.uw_gemm_swiglu(Xd, bg, bu))
+    check_swiglu(Hb, G, U, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("opts", [dict(grid=7), dict(grid=1), dict(split_k=1), dict(split_k=3), dict(stages=2),
+                                  dict(variant="tensor")])
+def test_swiglu_splits(opts):
+    """Stream-K and whole-multiple splits cut the paired accumulators; the
+    finisher adds both halves before the SwiGLU.  All splits agree with the
+    oracle."""
+    from tests.gpu_util import check_swiglu
+    Wg, Wu, bg, bu = _scase("384x512")
+    for M in (5, 80, 200):
+        X = S.activations(M, 512, seed=3100 + M)
+        H = _f32(uw.uw_gemm_swiglu(dev16(X), bg, bu, out_f32=True, **opts))
+        check_swiglu(H, O.gemm(X, Wg, "f32"), O.gemm(X, Wu, "f32"), bf16_out=False)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_swiglu_rejects_unsupported():
+    Wg, Wu, bg, bu = _scase("384x512")
+    X = dev16(S.activations(2, 512, seed=1))
+    for kw in (dict(pipeline="exponent"), dict(variant="gemv")):
+        with pytest.raises(uw.UnweightError) as ei:
+            uw.uw_gemm_swiglu(X, bg, bu, **kw)
+        assert ei.value.status == 4
+    _, _, b2, _ = _scase("200x1408")
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm_swiglu(X, bg, b2)
+    assert ei.value.status == 2
+    bh = uw.uw_compress(dev16(Wu), forms=uw.UW_FORM_HUFFMAN)
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm_swiglu(X, bg, bh)
+    assert ei.value.status == 4
+
+
+@pytest.fixture(scope="module")
+def gate_up_case():
+    Wg = S.gate_projection(seed=2)
+    Wu = S.gate_projection(seed=3)
+    return Wg, Wu, uw.uw_compress(dev16(Wg)), uw.uw_compress(dev16(Wu))
+
+
+@pytest.mark.parametrize("M", [1, 64, 256])
+def test_swiglu_full_size_every_output(gate_up_case, M):
+    """The Llama-3.1-8B gate+up pair W[14336,4096] x 2: every element of H
+    against the oracle."""
+    from tests.gpu_util import check_swiglu
+    Wg, Wu, bg, bu = gate_up_case
+    X = S.activations(M, 4096, seed=2 + S.X_SEED_OFFSET + M)
+    G = oracle_gemm(X, Wg, "f32")
+    U = oracle_gemm(X, Wu, "f32")
+    check_swiglu(_f32(uw.uw_gemm_swiglu(dev16(X), bg, bu)), G, U, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+def test_swiglu_full_size_large_batch_sampled(gate_up_case):
+    """M = 1024 (eight 128-row batch tiles): sampled outputs against the
+    oracle, one output element at a time."""
+    Wg, Wu, bg, bu = gate_up_case
+    M = 1024
+    X = S.activations(M, 4096, seed=2 + S.X_SEED_OFFSET + M)
+    H = _f32(uw.uw_gemm_swiglu(dev16(X), bg, bu))
+    rng = np.random.default_rng(9)
+    ms, ns = rng.integers(0, M, 512), rng.integers(0, 14336, 512)
+    G = np.array([O.gemm_one(X, Wg, int(m), int(n), "f32") for m, n in zip(ms, ns)])
+    U = np.array([O.gemm_one(X, Wu, int(m), int(n), "f32") for m, n in zip(ms, ns)])
+    from tests.gpu_util import check_swiglu
+    check_swiglu(H[ms, ns], G, U, bf16_out=True)
+    assert uw.uw_last_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# Layer sequences with hard (Huffman, transcoded ahead) and easy (palette)
+# projections (uw_gemm_sequence)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("pattern", ["hehe", "hhhh", "eeee", "ehhe"])
+@pytest.mark.parametrize("dec_ctas", [0, 37])
+@pytest.mark.parametrize("M", [1, 16, 100])
+def test_sequence_chain_matches_oracle(pattern, dec_ctas, M):
+    """A chain of four 512x512 projections, item i reading item i-1's BF16
+    output.  Each item's output against the oracle on the input the GPU fed
+    it, and bit for bit against the same item run alone."""
+    n = len(pattern)
+    Ws = [S.weight_with_verbatim_rows(512, 512, seed=400 + i, frac_groups=0.01) for i in range(n)]
+    blobs = [uw.uw_compress(dev16(w)) for w in Ws]
+    X0 = dev16(S.activations(M, 512, seed=410 + M))
+    Ys = [torch.empty(M, 512, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    items = [(blobs[i], X0 if i == 0 else Ys[i - 1], Ys[i], pattern[i] == "h") for i in range(n)]
+    for rep in range(2):
+        for y in Ys:
+            y.fill_(float("nan"))
+        uw.uw_gemm_sequence(items, M, dec_ctas=dec_ctas)
+        torch.cuda.synchronize()
+        xin = X0
+        for i in range(n):
+            Xh = host16(xin)
+            check_gemm(_f32(Ys[i]), O.gemm(Xh, Ws[i], "f32"), bf16_out=True)
+            alone = uw.uw_gemm(xin, blobs[i], "transcode" if pattern[i] == "h" else "direct_palette", variant="tensor")
+            assert np.array_equal(host16(alone), host16(Ys[i])), (i, rep)
+            xin = Ys[i]
+    assert uw.uw_last_device_status() == 0
+
+
+def test_sequence_rejects_missing_forms():
+    W = S.gaussian_weight(256, 512, seed=420)
+    bp = uw.uw_compress(dev16(W), forms=uw.UW_FORM_PALETTE)
+    X = dev16(S.activations(4, 512, seed=1))
+    Y = torch.empty(4, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(uw.UnweightError) as ei:
+        uw.uw_gemm_sequence([(bp, X, Y, True)], 4)
+    assert ei.value.status == 4
