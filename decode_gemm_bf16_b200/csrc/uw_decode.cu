@@ -63,13 +63,16 @@ struct DecodeParams {
 // Decodes segment `seg` (nsym symbols, a multiple of 64) into `row`: word k of
 // the segment (8 nibbles) is stored at row[(k + rot) & 31].
 //
-// Bit reservoir in two 32-bit registers: `hi` holds the next 32 stream bits
-// (all valid whenever the table is read), `lo` the following ones, of which
-// the top `nlo` are valid.  One table read decodes up to five symbols from the
-// 12-bit window hi >> 20; consuming them is a funnel shift.  When lo runs dry
-// the prefetched word `nxt` tops the reservoir up.  Word reads are clamped to
-// the stream, so a corrupt stream cannot read outside it; an undecodable
-// window still advances (12 bits) and is reported once per segment.
+// Bit reservoir: a 64-bit `buf` holds the next stream bits, most significant
+// first, `nv` of them valid.  A refill adds 32 bits whenever fewer than 32
+// are left, so every refill check is followed by two table reads of at most
+// 12 bits each with no further check.  One table read decodes up to five
+// symbols from the 12-bit window buf >> 52; consuming them is a 64-bit shift.
+// The prefetched word `nxt` is the next refill.  Word reads are clamped to the
+// stream, so a corrupt stream cannot read outside it; an undecodable window
+// still advances (12 bits) and is reported once per segment.  The second read
+// of a pair may decode past the segment's last symbol (the bits of the next
+// segment or the padding); nothing is stored for it.
 template <bool SMEM>
 __device__ __forceinline__ uint32_t ldw(const uint32_t* sp, int64_t i) {
     if (SMEM) return sp[i];
@@ -90,40 +93,39 @@ __device__ __forceinline__ void decode_bits(const DecodeParams& p, const uint32_
     const int64_t room = last_word - wi;
     const uint32_t last = room > 0x7FFFFFFF ? 0x7FFFFFFFu : (uint32_t)room;   // last readable index
     const uint32_t sh = (uint32_t)(bitpos & 31u);
-    const uint32_t w0 = ldw<SMEM>(sp, 0), w1 = ldw<SMEM>(sp, 1);
-    uint32_t nxt = ldw<SMEM>(sp, 2);                // the bits right after lo's valid ones
-    uint32_t hi = __funnelshift_l(w1, w0, sh);      // stream bits [bitpos, bitpos + 32)
-    uint32_t lo = w1 << sh;                         // rest of w1: 32 - sh valid bits
-    int nlo = 32 - (int)sh;
+    uint64_t buf = ((uint64_t)ldw<SMEM>(sp, 0) << 32 | (uint64_t)ldw<SMEM>(sp, 1)) << sh;
+    int nv = 64 - (int)sh;                          // 33..64 valid bits
+    uint32_t nxt = ldw<SMEM>(sp, 2);
     uint32_t idx = 3;
     uint32_t acc = 0, accn = 0, flags = 0;
     int k = 0, kr = rot;
     const int words = nsym >> 3;
     while (k < words) {
-        const uint32_t ent = lut[hi >> 20];
-        flags |= ent;
-        const uint32_t nb = lut_bits(ent);
-        hi = __funnelshift_l(lo, hi, nb);
-        lo <<= nb;
-        nlo -= (int)nb;
-        const uint32_t sy = ent >> kLutSymShift;
-        const uint32_t accn2 = accn + lut_nibble_bits(ent);
-        acc |= sy << accn;
-        if (nlo < 0) {
-            hi |= nxt >> (32 + nlo);
-            lo = nxt << (-nlo);
-            nlo += 32;
+        if (nv < 32) {
+            buf |= (uint64_t)nxt << (32 - nv);       // shift 1..24
+            nv += 32;
             nxt = ldw<SMEM>(sp, min(idx, last));
             idx++;
         }
-        if (accn2 >= 32u) {
-            row[kr] = acc;
-            kr = (kr + 1) & 31;
-            k++;
-            acc = sy >> (32u - accn);     // accn >= 12 here, so the shift is in [1, 20]
-            accn = accn2 - 32u;
-        } else {
-            accn = accn2;
+#pragma unroll
+        for (int t = 0; t < 2; t++) {
+            const uint32_t ent = lut[(uint32_t)(buf >> 52)];
+            flags |= ent;
+            const uint32_t nb = lut_bits(ent);
+            buf <<= nb;
+            nv -= (int)nb;
+            const uint32_t sy = ent >> kLutSymShift;
+            const uint32_t accn2 = accn + lut_nibble_bits(ent);
+            acc |= sy << accn;
+            if (accn2 >= 32u) {
+                if (k < words) row[kr] = acc;
+                kr = (kr + 1) & 31;
+                k++;
+                acc = sy >> (32u - accn);     // accn >= 12 here, so the shift is in [1, 20]
+                accn = accn2 - 32u;
+            } else {
+                accn = accn2;
+            }
         }
     }
     if (flags & kLutInvalid) raise_status(UW_ERR_DEVICE);
@@ -318,21 +320,22 @@ __global__ void __launch_bounds__(WARPS * 32, kStaged<MODE, WARPS> ? 3 : 4) k_de
 // nibbles and the activations share one CTA's shared memory with the
 // multiply.
 //
-// Work split: a warp owns 32 consecutive rows (lane = row) and a range of
-// kseg consecutive 256-weight segments of each.  Per segment, each lane
-// decodes its row's 256 symbols from the segment's start bit (the decoder
-// core above) into its shared-memory words, then walks them 16 weights at a
-// time: sign+mantissa bytes from the plane (16-byte loads), exponents from the
-// palette (or the verbatim store), BF16 rebuilt in registers and widened,
-// fused multiply-adds in k order into per-batch-row sums (even and odd
-// weights apart).  All lanes read the same activations at the same time
-// (shared-memory broadcast).  With several k ranges per row, each warp
-// publishes its 32 x M partial sums and the last warp of the row group to
-// arrive (a tagged counter) adds them in k-range order: the result does not
-// depend on the launch, only on the shape.
+// Work split, the decoders' own: a warp task is 32 consecutive 256-weight
+// segments (8192 weights; whole segments of consecutive rows, since
+// K % 256 == 0).  Phase 1: lane l decodes segment l of the task from its own
+// start bit into its shared-memory words (the decoder core above), while the
+// task's sign+mantissa bytes are requested into L2.  Phase 2: the warp walks
+// the task in order, two segments per step (a half warp each, 16 weights a
+// lane): sign+mantissa bytes in coalesced 256-byte reads, exponents from the
+// palette or the verbatim store, BF16 rebuilt in registers, fused
+// multiply-adds with the activations (consecutive 64-byte blocks per lane,
+// conflict-free), then a fixed xor tree over the 16 lanes gives each
+// segment's sum and the segment sums of a row are added in order.  A row
+// whose segments span several tasks is stored in pieces, and the last task of
+// the row to arrive (a tagged counter per row) adds the pieces in order: the
+// result depends on the shape only, never on the launch.
 // ---------------------------------------------------------------------------
 constexpr int kFusedWarps = 8;
-constexpr size_t kFusedXsMax = 64 * 1024;   // fp32 activations in shared memory up to this size
 
 struct FusedParams {
     DecodeParams d;
@@ -340,12 +343,10 @@ struct FusedParams {
     int M;
     int64_t N, K, KG;
     int S;                     // 256-weight segments per row
-    int kseg;                  // segments per k range
-    int nkr;                   // k ranges per row
-    int64_t ngroups;           // groups of 32 rows
-    int64_t items;             // ngroups * nkr warp tasks
-    float* part;               // [nkr][N][M] partial sums
-    unsigned long long* cnt;   // [ngroups] tagged arrival counters
+    int64_t ntasks;            // tasks of 32 segments
+    int pmax;                  // pieces per row at most
+    float* part;               // [N][pmax][M] pieces of rows that span tasks
+    unsigned long long* cnt;   // [N] tagged arrival counters
     unsigned long long epoch;
     void* Y;
     int out_f32;
@@ -356,198 +357,217 @@ __device__ __forceinline__ void fma_bf16x2(float2& acc, uint32_t w, float x0, fl
     acc.y = fmaf(__uint_as_float(w & 0xFFFF0000u), x1, acc.y);
 }
 
-template <int MB, bool XS>
-__global__ void __launch_bounds__(kFusedWarps * 32, 2) k_fused_huffman(const FusedParams p) {
+__device__ __forceinline__ void fused_store(const FusedParams& p, int64_t row, int m, float v) {
+    if (p.out_f32) reinterpret_cast<float*>(p.Y)[(int64_t)m * p.N + row] = v;
+    else {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        reinterpret_cast<uint16_t*>(p.Y)[(int64_t)m * p.N + row] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+}
+
+// Row `row`'s sums (racc[m], identical in every lane) for the segments of
+// task `task`: the output itself when the row lies inside the task, else a
+// piece, and the row's last arriving task adds the pieces.  Warp-uniform.
+template <int MB>
+__device__ __forceinline__ void fused_flush(const FusedParams& p, int64_t task, int64_t row, const float (&racc)[MB],
+                                            int lane) {
+    const int64_t s0 = row * p.S, s1 = s0 + p.S;             // the row's segments
+    const int64_t t_first = s0 / 32, t_last = (s1 - 1) / 32;
+    float v = 0.f;
+#pragma unroll
+    for (int m = 0; m < MB; m++)
+        if (m == lane) v = racc[m];
+    if (t_first == t_last) {
+        if (lane < p.M) fused_store(p, row, lane, v);
+        return;
+    }
+    const int pieces = (int)(t_last - t_first + 1);
+    if (lane < p.M) p.part[(row * p.pmax + (task - t_first)) * p.M + lane] = v;
+    __threadfence();
+    __syncwarp();
+    unsigned c = 0;
+    if (lane == 0) c = arrive_counter(p.cnt + row, p.epoch);
+    c = __shfl_sync(0xFFFFFFFFu, c, 0);
+    if (c == (unsigned)pieces) {
+        __threadfence();
+        if (lane < p.M) {
+            float sum = 0.f;
+            for (int q = 0; q < pieces; q++) sum += __ldcg(p.part + (row * p.pmax + q) * p.M + lane);
+            fused_store(p, row, lane, sum);
+        }
+        // a replay of the same captured call reuses its tag: start again from zero
+        if (lane == 0) p.cnt[row] = 0ull;
+    }
+}
+
+// Four CTAs of 8 warps per SM (64 registers a thread at batch 1-2): the
+// decode chains are latency-bound and want every warp the SM can hold; the
+// activations are read through L1 (all lanes of a half warp read one
+// contiguous KB), so shared memory holds only the table and the nibbles.
+template <int MB>
+__global__ void __launch_bounds__(kFusedWarps * 32, MB <= 2 ? 4 : 2) k_fused_huffman(const FusedParams p) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     uint32_t* stage = smem + kLutSize;
-    float* xs = reinterpret_cast<float*>(stage + kFusedWarps * 32 * 32);
     {
         const uint4* src = reinterpret_cast<const uint4*>(p.d.lut);
         uint4* dst = reinterpret_cast<uint4*>(lut);
         for (int i = threadIdx.x; i < kLutSize / 4; i += kFusedWarps * 32) dst[i] = __ldg(&src[i]);
     }
     // programmatic stream serialization: the table comes from the committed
-    // blob; activations, partial sums and outputs after the previous kernel
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (XS) {
-        const int64_t n4 = (int64_t)p.M * p.K / 4;
-        for (int64_t c = threadIdx.x; c < n4; c += kFusedWarps * 32) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.X) + c);
-            reinterpret_cast<float4*>(xs)[c] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
-                                                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
-        }
-    }
+    // blob; activations, pieces and outputs after the previous kernel
     __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* st = stage + warp * (32 * 32) + lane * 32;
+    uint32_t* st = stage + warp * (32 * 32);
     const uint32_t P0 = p.d.pal[0], P1 = p.d.pal[1], P2 = p.d.pal[2], P3 = p.d.pal[3];
     const int M = p.M;
-    for (int64_t item = (int64_t)blockIdx.x * kFusedWarps + warp; item < p.items;
-         item += (int64_t)gridDim.x * kFusedWarps) {
-        const int64_t rg = item / p.nkr;
-        const int kr = (int)(item - rg * p.nkr);
-        const int64_t r = rg * 32 + lane;
-        const bool valid = r < p.N;
-        const int j0 = kr * p.kseg, j1 = min(p.S, j0 + p.kseg);
-        float2 acc[MB];
-#pragma unroll
-        for (int m = 0; m < MB; m++) acc[m] = make_float2(0.f, 0.f);
-        if (valid) {
-            for (int j = j0; j < j1; j++) {
-                const int64_t seg = r * p.S + j;
-                const uint64_t bitpos = __ldg(&p.d.chunk_off[seg >> 4]) + __ldg(&p.d.seg_rel[seg]);
-                decode_bits<false>(p.d, lut, p.d.stream, p.d.nwords - 1, bitpos, kSeg, st, lane);
-                const int64_t kbase = (int64_t)j * kSeg;
-                const uint8_t* smr = p.d.sm + r * p.K + kbase;
-#pragma unroll 1
-                for (int q = 0; q < kSeg / kGroup; q++) {
-                    const int64_t g = r * p.KG + (kbase >> 6) + q;
-                    const uint32_t vw = __ldg(&p.d.vbits[g >> 5]);
-                    const bool verb = (vw >> (g & 31)) & 1u;
-                    const uint8_t* vsrc = nullptr;
-                    if (verb) {
-                        const int64_t rank = __ldg(&p.d.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
-                        vsrc = p.d.vexp + rank * kGroup;
-                    }
-#pragma unroll 2
-                    for (int i = 0; i < kGroup / 16; i++) {
-                        const int c = q * 4 + i;   // 16-weight chunk of the segment
-                        const uint4 sv = __ldcs(reinterpret_cast<const uint4*>(smr + c * 16));
-                        uint32_t E[4];
-                        if (verb) {
-                            const uint4 e = __ldg(reinterpret_cast<const uint4*>(vsrc + i * 16));
-                            E[0] = e.x; E[1] = e.y; E[2] = e.z; E[3] = e.w;
-                        } else {
-                            const uint32_t w0 = st[(2 * c + lane) & 31], w1 = st[(2 * c + 1 + lane) & 31];
-                            if (p.d.pal_small) {
-                                const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
-                                E[0] = palette4_small(w0, x0, P0, P1, P2, P3);
-                                E[1] = palette4_small(w0 >> 16, x0 >> 16, P0, P1, P2, P3);
-                                E[2] = palette4_small(w1, x1, P0, P1, P2, P3);
-                                E[3] = palette4_small(w1 >> 16, x1 >> 16, P0, P1, P2, P3);
-                            } else {
-                                E[0] = palette4(w0, P0, P1, P2, P3);
-                                E[1] = palette4(w0 >> 16, P0, P1, P2, P3);
-                                E[2] = palette4(w1, P0, P1, P2, P3);
-                                E[3] = palette4(w1 >> 16, P0, P1, P2, P3);
-                            }
-                        }
-                        const uint32_t S4[4] = {sv.x, sv.y, sv.z, sv.w};
-                        uint32_t wv[8];
-#pragma unroll
-                        for (int t = 0; t < 4; t++) {
-                            const uint2 mm = merge4(E[t], S4[t]);
-                            wv[2 * t] = mm.x;
-                            wv[2 * t + 1] = mm.y;
-                        }
-                        const int64_t k = kbase + c * 16;
-#pragma unroll
-                        for (int m = 0; m < MB; m++) {
-                            if (m < M) {
-                                if (XS) {
-                                    const float4* x4 = reinterpret_cast<const float4*>(xs + (int64_t)m * p.K + k);
-#pragma unroll
-                                    for (int t = 0; t < 4; t++) {
-                                        const float4 xv = x4[t];
-                                        fma_bf16x2(acc[m], wv[2 * t], xv.x, xv.y);
-                                        fma_bf16x2(acc[m], wv[2 * t + 1], xv.z, xv.w);
-                                    }
-                                } else {
-                                    const uint4* xp = reinterpret_cast<const uint4*>(p.X + (int64_t)m * p.K + k);
-#pragma unroll
-                                    for (int t = 0; t < 2; t++) {
-                                        const uint4 xv = __ldg(xp + t);
-                                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                                        for (int u = 0; u < 4; u++)
-                                            fma_bf16x2(acc[m], wv[4 * t + u], __uint_as_float(xw[u] << 16),
-                                                       __uint_as_float(xw[u] & 0xFFFF0000u));
-                                    }
-                                }
-                            }
-                        }
-                    }
-                }
+    const int half = lane >> 4, hl = lane & 15;
+    for (int64_t task = (int64_t)blockIdx.x * kFusedWarps + warp; task < p.ntasks;
+         task += (int64_t)gridDim.x * kFusedWarps) {
+        const int64_t base = task * kTaskElems, seg0 = task * 32;
+        {
+            // the task's sign+mantissa bytes, read in phase 2, into L2 now
+            const int64_t off = base + (int64_t)lane * kSeg;
+            if (off < p.d.n) {
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.d.sm + off));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.d.sm + off + 128));
             }
         }
-        if (p.nkr == 1) {
-            if (valid) {
+        // ---- phase 1: one segment per lane
+        {
+            const int64_t seg = seg0 + lane;
+            if (seg < p.d.nseg) {
+                const uint64_t bitpos = __ldg(&p.d.chunk_off[seg >> 4]) + __ldg(&p.d.seg_rel[seg]);
+                decode_bits<false>(p.d, lut, p.d.stream, p.d.nwords - 1, bitpos, kSeg, st + lane * 32, lane);
+            }
+        }
+        __syncwarp();
+        // ---- phase 2: two segments per step, 16 weights a lane
+        float racc[MB];
+#pragma unroll
+        for (int m = 0; m < MB; m++) racc[m] = 0.f;
+        int64_t rcur = -1;
+        // row and segment-within-row of the two segments of the step (segments
+        // 2 it and 2 it + 1 of the task), advanced by two segments per step
+        const int64_t row0 = seg0 / p.S;
+        const int jr0 = (int)(seg0 - row0 * p.S);
+        int64_t rw[2] = {row0, row0};
+        int jw[2] = {jr0, jr0 + 1};
+        if (jw[1] >= p.S) { jw[1] -= p.S; rw[1]++; }
+#pragma unroll 1
+        for (int it = 0; it < 16; it++) {
+            const int j = 2 * it + half;               // segment of the task
+            const int k0 = 2 * hl;                     // first nibble word of this lane
+            const int64_t gs = seg0 + j;
+            float2 pacc[MB];
+#pragma unroll
+            for (int m = 0; m < MB; m++) pacc[m] = make_float2(0.f, 0.f);
+            if (gs < p.d.nseg) {
+                const int64_t e = base + (int64_t)j * kSeg + k0 * 8;   // element index
+                const int64_t kk = (int64_t)(half ? jw[1] : jw[0]) * kSeg + k0 * 8;   // k within the row
+                const uint4 sv = __ldg(reinterpret_cast<const uint4*>(p.d.sm + e));
+                uint32_t E[4];
+                const int64_t g = e >> 6;
+                const uint32_t vw = __ldg(&p.d.vbits[g >> 5]);
+                if ((vw >> (g & 31)) & 1u) {
+                    const int64_t rank = __ldg(&p.d.vpre[g >> 5]) + __popc(vw & ((1u << (g & 31)) - 1u));
+                    const uint4 ev = __ldg(reinterpret_cast<const uint4*>(p.d.vexp + rank * kGroup + (e & 63)));
+                    E[0] = ev.x; E[1] = ev.y; E[2] = ev.z; E[3] = ev.w;
+                } else {
+                    const uint32_t* r = st + j * 32;
+                    const uint32_t w0 = r[(k0 + j) & 31], w1 = r[(k0 + 1 + j) & 31];
+                    if (p.d.pal_small) {
+                        const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
+                        E[0] = palette4_small(w0, x0, P0, P1, P2, P3);
+                        E[1] = palette4_small(w0 >> 16, x0 >> 16, P0, P1, P2, P3);
+                        E[2] = palette4_small(w1, x1, P0, P1, P2, P3);
+                        E[3] = palette4_small(w1 >> 16, x1 >> 16, P0, P1, P2, P3);
+                    } else {
+                        E[0] = palette4(w0, P0, P1, P2, P3);
+                        E[1] = palette4(w0 >> 16, P0, P1, P2, P3);
+                        E[2] = palette4(w1, P0, P1, P2, P3);
+                        E[3] = palette4(w1 >> 16, P0, P1, P2, P3);
+                    }
+                }
+                const uint32_t S4[4] = {sv.x, sv.y, sv.z, sv.w};
+                uint32_t wv[8];
+#pragma unroll
+                for (int t = 0; t < 4; t++) {
+                    const uint2 mm = merge4(E[t], S4[t]);
+                    wv[2 * t] = mm.x;
+                    wv[2 * t + 1] = mm.y;
+                }
 #pragma unroll
                 for (int m = 0; m < MB; m++) {
-                    if (m >= M) break;
-                    const float v = acc[m].x + acc[m].y;
-                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[(int64_t)m * p.N + r] = v;
-                    else {
-                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                        reinterpret_cast<uint16_t*>(p.Y)[(int64_t)m * p.N + r] = *reinterpret_cast<const uint16_t*>(&h);
-                    }
-                }
-            }
-            continue;
-        }
-        // several k ranges: publish, and the last warp of the row group sums
-        if (valid) {
+                    if (m < M) {
+                        const uint4* xp = reinterpret_cast<const uint4*>(p.X + (int64_t)m * p.K + kk);
 #pragma unroll
-            for (int m = 0; m < MB; m++)
-                if (m < M) p.part[((int64_t)kr * p.N + r) * M + m] = acc[m].x + acc[m].y;
-        }
-        __threadfence();
-        __syncwarp();
-        unsigned c = 0;
-        if (lane == 0) c = arrive_counter(p.cnt + rg, p.epoch);
-        c = __shfl_sync(0xFFFFFFFFu, c, 0);
-        if (c == (unsigned)p.nkr) {
-            __threadfence();
-            if (valid) {
-                for (int m = 0; m < M; m++) {
-                    float v = 0.f;
-                    for (int kk = 0; kk < p.nkr; kk++) v += __ldcg(p.part + ((int64_t)kk * p.N + r) * M + m);
-                    if (p.out_f32) reinterpret_cast<float*>(p.Y)[(int64_t)m * p.N + r] = v;
-                    else {
-                        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                        reinterpret_cast<uint16_t*>(p.Y)[(int64_t)m * p.N + r] = *reinterpret_cast<const uint16_t*>(&h);
+                        for (int t = 0; t < 2; t++) {
+                            const uint4 xv = __ldg(xp + t);
+                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                            for (int u = 0; u < 4; u++)
+                                fma_bf16x2(pacc[m], wv[4 * t + u], __uint_as_float(xw[u] << 16),
+                                           __uint_as_float(xw[u] & 0xFFFF0000u));
+                        }
                     }
                 }
             }
-            // a replay of the same captured call reuses its tag: start again from zero
-            if (lane == 0) p.cnt[rg] = 0ull;
+            // segment sums: a fixed xor tree over each half warp, then both
+            // halves' sums to every lane
+            float s_lo[MB], s_hi[MB];
+#pragma unroll
+            for (int m = 0; m < MB; m++) {
+                float v = pacc[m].x + pacc[m].y;
+                v += __shfl_xor_sync(0xFFFFFFFFu, v, 8);
+                v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+                v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+                v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+                s_lo[m] = __shfl_sync(0xFFFFFFFFu, v, 0);
+                s_hi[m] = __shfl_sync(0xFFFFFFFFu, v, 16);
+            }
+            // rows in order (warp-uniform)
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int64_t gsh = seg0 + 2 * it + h;
+                if (gsh >= p.d.nseg) break;
+                const int64_t row = rw[h];
+                if (row != rcur) {
+                    if (rcur >= 0) fused_flush<MB>(p, task, rcur, racc, lane);
+                    rcur = row;
+#pragma unroll
+                    for (int m = 0; m < MB; m++) racc[m] = 0.f;
+                }
+#pragma unroll
+                for (int m = 0; m < MB; m++) racc[m] += h ? s_hi[m] : s_lo[m];
+            }
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                jw[h] += 2;
+                while (jw[h] >= p.S) {
+                    jw[h] -= p.S;
+                    rw[h]++;
+                }
+            }
         }
+        if (rcur >= 0) fused_flush<MB>(p, task, rcur, racc, lane);
+        __syncwarp();   // phase 1 of the next task overwrites the nibbles
     }
-}
-
-// Split of one fused call: k ranges per row and segments per range, so that
-// about 24 warp tasks per SM exist.
-struct FusedSplit {
-    int S, kseg, nkr;
-    int64_t ngroups, items;
-};
-
-FusedSplit fused_split(int64_t N, int64_t K) {
-    FusedSplit f;
-    f.S = (int)(K / kSeg);
-    f.ngroups = (N + 31) / 32;
-    const int64_t target = (int64_t)num_sms() * 24;
-    int64_t kseg = (f.S * f.ngroups + target / 2) / target;
-    if (kseg < 1) kseg = 1;
-    if (kseg > f.S) kseg = f.S;
-    f.kseg = (int)kseg;
-    f.nkr = (f.S + f.kseg - 1) / f.kseg;
-    f.items = f.ngroups * f.nkr;
-    return f;
 }
 
 }  // namespace
 
 static DecodeParams decode_params(const uw_blob* b, void* out);
 
+static int fused_pmax(int64_t K) { return (int)((K / kSeg + 31) / 32) + 1; }
+
 size_t fused_ws_bytes(int64_t M, int64_t N, int64_t K) {
     if (K % kSeg) return 0;
-    const FusedSplit f = fused_split(N, K);
     const int64_t mc = M < kFusedMaxM ? M : kFusedMaxM;
-    const size_t part = (size_t)f.nkr * N * mc * 4;
-    return ((part + 255) & ~size_t(255)) + (((size_t)f.ngroups * 8 + 255) & ~size_t(255));
+    const size_t part = (size_t)N * fused_pmax(K) * mc * 4;
+    return ((part + 255) & ~size_t(255)) + (((size_t)N * 8 + 255) & ~size_t(255));
 }
 
 cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M, void* Y, int out_f32, void* ws,
@@ -564,44 +584,34 @@ cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M,
     p.N = b->geo.N;
     p.K = b->geo.K;
     p.KG = b->geo.KG;
-    const FusedSplit f = fused_split(p.N, p.K);
-    p.S = f.S;
-    p.kseg = f.kseg;
-    p.nkr = f.nkr;
-    p.ngroups = f.ngroups;
-    p.items = f.items;
-    const size_t part = (size_t)f.nkr * p.N * M * 4;
+    p.S = (int)(p.K / kSeg);
+    p.ntasks = (b->geo.nseg + 31) / 32;
+    p.pmax = fused_pmax(p.K);
+    const size_t part = (size_t)p.N * p.pmax * M * 4;
     p.part = (float*)ws;
     p.cnt = (unsigned long long*)((uint8_t*)ws + ((part + 255) & ~size_t(255)));
     p.epoch = gemm_next_epoch();
     p.Y = Y;
     p.out_f32 = out_f32;
-    const size_t xbytes = (size_t)M * p.K * 4;
-    const bool xs = xbytes <= kFusedXsMax;
-    const size_t smem = (size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4 + (xs ? xbytes : 0);
+    const size_t smem = (size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4;
     const int mb = M == 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
     typedef void (*Kern)(const FusedParams);
-    Kern kern = nullptr;
-#define UW_FUSED_CASE(B)                                                  \
-    if (mb == B) kern = xs ? k_fused_huffman<B, true> : k_fused_huffman<B, false>;
-    UW_FUSED_CASE(1)
-    UW_FUSED_CASE(2)
-    UW_FUSED_CASE(4)
-    UW_FUSED_CASE(8)
-    UW_FUSED_CASE(16)
-#undef UW_FUSED_CASE
-    static bool attr_set[5][2][64] = {};
+    Kern kern = mb == 1 ? k_fused_huffman<1> : mb == 2 ? k_fused_huffman<2> : mb == 4 ? k_fused_huffman<4>
+              : mb == 8 ? k_fused_huffman<8> : k_fused_huffman<16>;
+    static bool carve_set[5][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     const int mi = mb == 1 ? 0 : mb == 2 ? 1 : mb == 4 ? 2 : mb == 8 ? 3 : 4;
-    bool& done = attr_set[mi][xs ? 1 : 0][dev & 63];
-    if (!done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)((size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4 + kFusedXsMax));
+    if (!carve_set[mi][dev & 63]) {
+        // four CTAs of 48 KB per SM need the largest shared-memory carveout
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
-        done = true;
+        carve_set[mi][dev & 63] = true;
     }
-    const int64_t grid = (p.items + kFusedWarps - 1) / kFusedWarps;
+    // every task is resident at once when possible; otherwise CTAs loop
+    const int per_sm = mb <= 2 ? 4 : 2;
+    int64_t grid = (p.ntasks + kFusedWarps - 1) / kFusedWarps;
+    if (grid > (int64_t)num_sms() * per_sm) grid = (int64_t)num_sms() * per_sm;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kFusedWarps * 32);

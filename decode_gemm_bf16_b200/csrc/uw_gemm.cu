@@ -107,6 +107,7 @@ struct GemmParams {
     uint64_t timeout_ns;
     int static_sm;                 // sign+mantissa plane and verbatim flags come from the committed blob
     int static_s2;                 // so does the second plane (the stored index plane)
+    int pf_ahead;                  // weight tiles requested into L2 this many iterations ahead of their load (0: none)
 };
 
 // Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
@@ -163,6 +164,31 @@ struct SegWalker {
     }
 };
 
+// L2 prefetch of the weight tiles (planes no kernel writes) of this CTA's
+// iteration `it` (absolute index in the (tile, k step) sequence).
+template <int SRC, int KB, int NH>
+__device__ __forceinline__ void prefetch_weights(const GemmParams& p, uint32_t it, const CUtensorMap* const (&maps_a)[2],
+                                                 const CUtensorMap* const (&maps_s2)[2],
+                                                 const CUtensorMap* const (&maps_v)[2]) {
+    const uint32_t tile = it / (uint32_t)p.kt_count;
+    const int kt = (int)(it - tile * (uint32_t)p.kt_count);
+    const int n_tile = (int)(tile / (uint32_t)p.m_tiles);
+    constexpr int kHalves = KB / 64;
+    if (SRC == kSrcDense) {
+#pragma unroll
+        for (int hb = 0; hb < kHalves; hb++) tma_prefetch_2d(maps_a[0], kt * KB + hb * 64, n_tile * 128);
+        return;
+    }
+#pragma unroll
+    for (int h = 0; h < NH; h++) {
+        tma_prefetch_2d(maps_a[h], kt * KB, n_tile * 128);
+        if (SRC == kSrcPalette) {
+            tma_prefetch_2d(maps_v[h], n_tile * 4, kt * kHalves);
+            if (p.static_s2) tma_prefetch_2d(maps_s2[h], kt * (KB / 2), n_tile * 128);
+        }
+    }
+}
+
 __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
@@ -179,23 +205,23 @@ __device__ __forceinline__ uint32_t sw32_off(int r, int c) { return r * 32 + ((c
 // taddr .. +15 (one BF16 pair per column).  Sign+mantissa and exponent
 // tiles have rows of KB bytes (swizzle KB), index tiles rows of KB/2 bytes.
 template <int SRC, int KB>
-__device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet& ps, const uint8_t* stage, int64_t n0,
+__device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet& ps, uint32_t stage, int64_t n0,
                                             int kt, int q, int j, int lane, uint32_t taddr) {
     const int r = 32 * q + lane;
     auto row_off = [&](int c) { return KB == 128 ? sw128_off(r, c) : sw64_off(r, c); };
-    const uint8_t* SM = stage + ps.off_sm;
-    const uint4 s0 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j));
-    const uint4 s1 = *reinterpret_cast<const uint4*>(SM + row_off(2 * j + 1));
+    const uint32_t SM = stage + ps.off_sm;
+    const uint4 s0 = lds128(SM + row_off(2 * j));
+    const uint4 s1 = lds128(SM + row_off(2 * j + 1));
     uint32_t E[8];
     if (SRC == kSrcExponent) {
-        const uint8_t* EX = stage + ps.off_s2;
-        const uint4 e0 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j));
-        const uint4 e1 = *reinterpret_cast<const uint4*>(EX + row_off(2 * j + 1));
+        const uint32_t EX = stage + ps.off_s2;
+        const uint4 e0 = lds128(EX + row_off(2 * j));
+        const uint4 e1 = lds128(EX + row_off(2 * j + 1));
         E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
         E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
     } else {
         const int grp = j >> 1;   // 64-weight group within the stage
-        const uint32_t vw = *reinterpret_cast<const uint32_t*>(stage + ps.off_v + 16 * grp + 4 * q);
+        const uint32_t vw = lds32(stage + ps.off_v + 16 * grp + 4 * q);
         if ((vw >> lane) & 1u) {
             // verbatim group: raw exponents from the verbatim store
             const int64_t g = (n0 + r) * p.KG + (int64_t)kt * (KB / kGroup) + grp;
@@ -206,8 +232,7 @@ __device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet&
             E[0] = e0.x; E[1] = e0.y; E[2] = e0.z; E[3] = e0.w;
             E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
         } else {
-            const uint4 ix = *reinterpret_cast<const uint4*>(
-                stage + ps.off_s2 + (KB == 128 ? sw64_off(r, j) : sw32_off(r, j)));
+            const uint4 ix = lds128(stage + ps.off_s2 + (KB == 128 ? sw64_off(r, j) : sw32_off(r, j)));
             const uint32_t w[4] = {ix.x, ix.y, ix.z, ix.w};
             const uint32_t P0 = ps.pal[0], P1 = ps.pal[1], P2 = ps.pal[2], P3 = ps.pal[3];
             if (ps.pal_small) {
@@ -485,7 +510,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     }
                 }
             }
+            // weight tiles further ahead than the ring holds go to L2 now, so
+            // that their loads, when the ring frees up, are L2 hits
+            const uint32_t it_begin = iter_begin(blockIdx.x, p.total_iters, p.P);
+            const uint32_t it_end = iter_begin(blockIdx.x + 1, p.total_iters, p.P);
+            const bool pf = p.pf_ahead > 0 && (SRC == kSrcDense || p.static_sm) && !p.band_ready;
+            // a dense W may be the output of the previous kernel (the full
+            // pipeline's decode): its prefetch waits for that kernel
+            if (pf && leader && SRC != kSrcDense)
+                for (uint32_t i = it_begin + (uint32_t)npre; i < it_begin + (uint32_t)(npre + p.pf_ahead) && i < it_end; i++)
+                    prefetch_weights<SRC, KB, NH>(p, i, maps_a, maps_s2, maps_v);
             asm volatile("griddepcontrol.wait;" ::: "memory");
+            if (pf && leader && SRC == kSrcDense)
+                for (uint32_t i = it_begin; i < it_begin + (uint32_t)p.pf_ahead && i < it_end; i++)
+                    prefetch_weights<SRC, KB, NH>(p, i, maps_a, maps_s2, maps_v);
             SegWalker wk(blockIdx.x, p);
             Segment sg;
             int64_t q = 0;
@@ -525,6 +563,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     if (!leader) continue;
+                    if (pf) {
+                        // keeps pf_ahead iterations requested beyond the one loaded now
+                        const uint32_t ahead = it_begin + (uint32_t)q + (uint32_t)p.pf_ahead;
+                        if (ahead < it_end) prefetch_weights<SRC, KB, NH>(p, ahead, maps_a, maps_s2, maps_v);
+                    }
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
 #pragma unroll
                     for (int hb = 0; hb < kHalves; hb++)
@@ -637,7 +680,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 #pragma unroll
                     for (int pc = 0; pc < kPieces; pc++) {
                         const int j = hh * kPieces + pc;
-                        rebuild_row<SRC, KB>(p, p.ps[h], smem + (size_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
+                        rebuild_row<SRC, KB>(p, p.ps[h], smem_base + (uint32_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
                                              tlane + (uint32_t)(KB / 2) * (uint32_t)(NH * s + h) + 16u * (uint32_t)j);
                     }
                 }
@@ -735,10 +778,12 @@ __global__ void __launch_bounds__(kThreadsDense, 1)
     gemm_body<kSrcDense, KB, 1>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
 }
 
-// Rebuilding sources: 22 warps held to 72 registers, which leaves one warp's
-// worth of registers per SM sub-partition for a decoder CTA running beside.
+// Rebuilding sources: 22 warps, six of them on two of the four SM
+// sub-partitions, whose 16 K registers each allow 80 registers a thread; 72
+// when a decoder CTA runs beside the GEMM (that leaves one warp's worth of
+// registers per sub-partition for it).
 template <int SRC, int KB>
-__global__ void __maxnreg__(72)
+__global__ void __maxnreg__(80)
     k_gemm_recon(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
@@ -746,11 +791,20 @@ __global__ void __maxnreg__(72)
     gemm_body<SRC, KB, 1>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
 }
 
+template <int SRC, int KB>
+__global__ void __maxnreg__(72)
+    k_gemm_recon_beside(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
+                        const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
+    gemm_body<SRC, KB, 1>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
+}
+
 // Gate and up projections in one launch (direct palette, SwiGLU epilogue):
 // each stage carries both matrices' tiles for the same rows and k, each
 // tile accumulates into two halves of TMEM.
 template <int KB>
-__global__ void __maxnreg__(72)
+__global__ void __maxnreg__(80)
     k_gemm_swiglu(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
                   const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
@@ -862,7 +916,9 @@ GemmSplit gemm_split(int64_t M, int64_t N, int64_t K, int grid, int split_k, int
     // stage k: 128 for small batch tiles (halves the per-stage TMA, barrier
     // and MMA-issue overhead per weight byte), 64 where a stage is already
     // large (batch tiles above 64 rows)
-    g.KB = (g.MG <= 64 && K % 128 == 0) ? 128 : 64;
+    // (paired tiles keep 64-k stages: two A slots per stage would leave too
+    // few 128-k stages in TMEM)
+    g.KB = (g.MG <= 64 && K % 128 == 0 && nh == 1) ? 128 : 64;
     g.m_tiles = (int)((M + g.MG - 1) / g.MG);
     g.n_tiles = (int)((N + kBlockN - 1) / kBlockN);
     g.kt = (int)(K / g.KB);
@@ -960,6 +1016,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.timeout_ns = timeout_ns();
     p.static_sm = a.static_sm;
     p.static_s2 = a.static_s2;
+    // L2 prefetch distance for the weight tiles: larger batch tiles consume
+    // a stage faster relative to the memory latency
+    p.pf_ahead = p.MG >= 128 ? 6 : 4;
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
     const int halves = KB / kBoxK;
@@ -1004,6 +1063,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (a.src != kSrcDense) {
         const int s_tmem = (int)((512u - acc_cols) / (uint32_t)(NH * KB / 2));
         if (S > s_tmem) S = s_tmem;
+        // The two rebuild groups take alternate iterations, so with an odd
+        // ring a group comes back to a slot two phases later, and a parity
+        // wait cannot tell that phase from the one before it (a group that is
+        // ahead would rebuild a slot whose new tiles have not landed).  An
+        // even ring gives every slot to one group, one phase after another.
+        S &= ~1;
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.stages = S;
@@ -1064,6 +1129,11 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     GemmKernel kern;
     if (a.pair)
         kern = KB == 128 ? k_gemm_swiglu<128> : k_gemm_swiglu<64>;
+    else if (a.smem_cap > 0 && a.src != kSrcDense)   // room left for decoder CTAs beside
+        kern = KB == 128 ? (a.src == kSrcExponent ? k_gemm_recon_beside<kSrcExponent, 128>
+                                                  : k_gemm_recon_beside<kSrcPalette, 128>)
+                         : (a.src == kSrcExponent ? k_gemm_recon_beside<kSrcExponent, 64>
+                                                  : k_gemm_recon_beside<kSrcPalette, 64>);
     else if (KB == 128)
         kern = a.src == kSrcDense      ? k_gemm_dense<128>
                : a.src == kSrcExponent ? k_gemm_recon<kSrcExponent, 128>

@@ -633,3 +633,21 @@ def test_sequence_rejects_missing_forms():
     with pytest.raises(uw.UnweightError) as ei:
         uw.uw_gemm_sequence([(bp, X, Y, True)], 4)
     assert ei.value.status == 4
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_repeated_calls_bit_identical_full_size(gate_up_case, M):
+    """The same call thirty times in a row gives the same bits (the split and
+    the summation order depend on the shape only).  Out-of-order completions
+    of the stage ring's loads once let a rebuild group run ahead into a slot
+    whose tiles had not landed (an odd ring); repeats catch that kind of race."""
+    Wg, Wu, bg, bu = gate_up_case
+    X = dev16(S.activations(M, 4096, seed=4000 + M))
+    calls = {"swiglu": lambda: uw.uw_gemm_swiglu(X, bg, bu, out_f32=True),
+             "direct_palette": lambda: uw.uw_gemm(X, bg, "direct_palette", out_f32=True),
+             "exponent": lambda: uw.uw_gemm(X, bu, "exponent", out_f32=True)}
+    for name, fn in calls.items():
+        ref = fn().clone()
+        for _ in range(30):
+            assert torch.equal(fn(), ref), name
+    assert uw.uw_last_device_status() == 0
