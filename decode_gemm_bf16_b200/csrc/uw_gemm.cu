@@ -107,7 +107,6 @@ struct GemmParams {
     uint64_t timeout_ns;
     int static_sm;                 // sign+mantissa plane and verbatim flags come from the committed blob
     int static_s2;                 // so does the second plane (the stored index plane)
-    int pf_ahead;                  // weight tiles requested into L2 this many iterations ahead of their load (0: none)
 };
 
 // Stream-K split: CTA b owns iterations [iter_begin(b), iter_begin(b+1)) of
@@ -163,31 +162,6 @@ struct SegWalker {
         return true;
     }
 };
-
-// L2 prefetch of the weight tiles (planes no kernel writes) of this CTA's
-// iteration `it` (absolute index in the (tile, k step) sequence).
-template <int SRC, int KB, int NH>
-__device__ __forceinline__ void prefetch_weights(const GemmParams& p, uint32_t it, const CUtensorMap* const (&maps_a)[2],
-                                                 const CUtensorMap* const (&maps_s2)[2],
-                                                 const CUtensorMap* const (&maps_v)[2]) {
-    const uint32_t tile = it / (uint32_t)p.kt_count;
-    const int kt = (int)(it - tile * (uint32_t)p.kt_count);
-    const int n_tile = (int)(tile / (uint32_t)p.m_tiles);
-    constexpr int kHalves = KB / 64;
-    if (SRC == kSrcDense) {
-#pragma unroll
-        for (int hb = 0; hb < kHalves; hb++) tma_prefetch_2d(maps_a[0], kt * KB + hb * 64, n_tile * 128);
-        return;
-    }
-#pragma unroll
-    for (int h = 0; h < NH; h++) {
-        tma_prefetch_2d(maps_a[h], kt * KB, n_tile * 128);
-        if (SRC == kSrcPalette) {
-            tma_prefetch_2d(maps_v[h], n_tile * 4, kt * kHalves);
-            if (p.static_s2) tma_prefetch_2d(maps_s2[h], kt * (KB / 2), n_tile * 128);
-        }
-    }
-}
 
 __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -510,20 +484,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     }
                 }
             }
-            // weight tiles further ahead than the ring holds go to L2 now, so
-            // that their loads, when the ring frees up, are L2 hits
-            const uint32_t it_begin = iter_begin(blockIdx.x, p.total_iters, p.P);
-            const uint32_t it_end = iter_begin(blockIdx.x + 1, p.total_iters, p.P);
-            const bool pf = p.pf_ahead > 0 && (SRC == kSrcDense || p.static_sm) && !p.band_ready;
-            // a dense W may be the output of the previous kernel (the full
-            // pipeline's decode): its prefetch waits for that kernel
-            if (pf && leader && SRC != kSrcDense)
-                for (uint32_t i = it_begin + (uint32_t)npre; i < it_begin + (uint32_t)(npre + p.pf_ahead) && i < it_end; i++)
-                    prefetch_weights<SRC, KB, NH>(p, i, maps_a, maps_s2, maps_v);
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            if (pf && leader && SRC == kSrcDense)
-                for (uint32_t i = it_begin; i < it_begin + (uint32_t)p.pf_ahead && i < it_end; i++)
-                    prefetch_weights<SRC, KB, NH>(p, i, maps_a, maps_s2, maps_v);
             SegWalker wk(blockIdx.x, p);
             Segment sg;
             int64_t q = 0;
@@ -563,11 +524,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     if (!leader) continue;
-                    if (pf) {
-                        // keeps pf_ahead iterations requested beyond the one loaded now
-                        const uint32_t ahead = it_begin + (uint32_t)q + (uint32_t)p.pf_ahead;
-                        if (ahead < it_end) prefetch_weights<SRC, KB, NH>(p, ahead, maps_a, maps_s2, maps_v);
-                    }
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
 #pragma unroll
                     for (int hb = 0; hb < kHalves; hb++)
@@ -656,7 +612,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     } else if (kRecon && warp >= kReconWarp0) {
         // ------------------------------------------------------------ reconstruct
         // warp w may only touch TMEM lanes 32(w%4)..+31.  Two groups of 8
-        // warps take alternate stages (two stages rebuilt at once); inside a
+        // warps take the even and the odd ring slots (two stages rebuilt at
+        // once; with an odd ring the even group has one slot more); inside a
         // group, two warps per lane quarter, one per half of the stage's k
         // (one or two 32-k pieces each), for each weight matrix of the tile.
         constexpr int kPieces = KB / 64;   // 32-k pieces per warp and stage
@@ -672,7 +629,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         while (ok && wk.next(sg)) {
             const int64_t n0 = (sg.tile / p.m_tiles) * kBlockN;
             for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
-                if ((int)(q & 1) != group) continue;
+                // A ring slot always belongs to the same group (slot parity),
+                // so a group's waits on a slot see consecutive mbarrier
+                // phases.  Taking alternate iterations instead would, with an
+                // odd ring, bring a group back to a slot two phases later,
+                // which a parity wait cannot tell from the phase before: a
+                // group ahead of the loads would rebuild a slot whose tiles
+                // had not landed.
+                if ((rp.s & 1) != group) continue;
                 const int s = rp.s;
                 if (!mbar_wait(smem_u32(&full_bar[s]), rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
 #pragma unroll
@@ -1016,9 +980,6 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     p.timeout_ns = timeout_ns();
     p.static_sm = a.static_sm;
     p.static_s2 = a.static_s2;
-    // L2 prefetch distance for the weight tiles: larger batch tiles consume
-    // a stage faster relative to the memory latency
-    p.pf_ahead = p.MG >= 128 ? 6 : 4;
 
     // stage layout (all tiles 1024-byte aligned; swizzled TMA destinations)
     const int halves = KB / kBoxK;
@@ -1063,12 +1024,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (a.src != kSrcDense) {
         const int s_tmem = (int)((512u - acc_cols) / (uint32_t)(NH * KB / 2));
         if (S > s_tmem) S = s_tmem;
-        // The two rebuild groups take alternate iterations, so with an odd
-        // ring a group comes back to a slot two phases later, and a parity
-        // wait cannot tell that phase from the one before it (a group that is
-        // ahead would rebuild a slot whose new tiles have not landed).  An
-        // even ring gives every slot to one group, one phase after another.
-        S &= ~1;
+
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.stages = S;

@@ -156,8 +156,7 @@ typedef struct {
                                 k ranges (at most its k steps), one CTA each, grid ignored.
                                 split_k >= 2 needs tiles * split_k <= SMs (else
                                 UW_ERR_INVALID_ARG)                                        */
-    int32_t stages;          /* 0: the deepest stage ring that fits; >= 2: at most this many
-                                (rebuilding pipelines round the ring down to an even depth) */
+    int32_t stages;          /* 0: the deepest stage ring that fits; >= 2: at most this many */
     int32_t projection;      /* UW_PIPE_AUTO: the projection index looked up in `plan`     */
     const uw_plan_entry* plan;   /* UW_PIPE_AUTO: the autotuner's entries (host memory)    */
     int32_t plan_entries;
