@@ -658,6 +658,57 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def run_profile(args):
+    """One call shape, alone, for a profiler's launch list or capture:
+    `--profile gate/M=1024` runs that projection's call over the layers of a
+    small stack, `--profile step` every projection at every batch of the
+    step (the library's own plan choice, no autotuning); `--warmup` passes,
+    then `--steps` passes, and it prints the time per pass.  Not a bench
+    line."""
+    import torch
+    import decode_gemm_bf16_b200 as uw
+    import synthetic as S
+
+    if args.profile == "step":
+        calls = [(p, M) for M in MS for p in PROJ]
+    else:
+        proj, mpart = args.profile.split("/")
+        calls = [(proj, int(mpart.split("=")[1]))]
+    used = sorted({PROJ.index(p) for p, _ in calls})
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    blobs = []
+    for layer in range(args.layers):
+        mats = S.stack_layer_device(layer, dev)
+        blobs.append({j: uw.uw_compress(mats[j]) for j in used})
+        del mats
+    X = {(p, M): S.activations_device(M, SHAPES[p][1], seed=17 + M, device=dev) for p, M in calls}
+    Y = {(p, M): torch.empty(M, SHAPES[p][0], dtype=torch.bfloat16, device=dev) for p, M in calls}
+    ws = torch.zeros(max(uw.uw_gemm_workspace(blobs[0][PROJ.index(p)], M, args.pipeline) for p, M in calls),
+                     dtype=torch.uint8, device=dev)
+
+    def one_pass():
+        for p, M in calls:
+            j = PROJ.index(p)
+            for lb in blobs:
+                uw.uw_gemm(X[(p, M)], lb[j], args.pipeline, out=Y[(p, M)], ws=ws, projection=j)
+
+    for _ in range(max(1, args.warmup)):
+        one_pass()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        one_pass()
+    b.record()
+    torch.cuda.synchronize()
+    if uw.uw_last_device_status() != 0:
+        raise RuntimeError("device status set")
+    us = 1e3 * a.elapsed_time(b) / args.steps
+    print(json.dumps({"profile": args.profile, "pipeline": args.pipeline, "layers": len(blobs),
+                      "calls_per_pass": len(calls) * len(blobs), "us_per_pass": us}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -667,8 +718,13 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--layers", type=int, default=32, help="layers of the stack (32 = Llama-3.1-8B)")
     ap.add_argument("--stack", action="store_true", help="same as the default run (kept for old command lines)")
+    ap.add_argument("--profile", default=None, metavar="PROJ/M=B",
+                    help="time one call shape alone (e.g. gate/M=1024) for a profiler; prints no bench line")
+    ap.add_argument("--pipeline", default="direct_palette", help="pipeline of the --profile call")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -32,7 +32,10 @@
 //     then carries 3 bytes per weight (TMA write + one read) instead of 7,
 //     and holds no A tiles;
 //   * stream-K: the (tile, stage) iterations are split evenly over one CTA
-//     per SM (or one CTA per tile when that is cheaper, see launch_gemm); a
+//     per SM (or one CTA per tile when that is cheaper, see launch_gemm);
+//     tiles are numbered batch-tile-major, so the CTAs working on the batch
+//     tiles of one weight tile do so at about the same time and its planes
+//     come from HBM about once (L2 serves the other reads); a
 //     tile cut between CTAs is finished by the CTA holding its first k steps,
 //     which reaches it last and adds the others' fp32 partial rows in k order
 //     (deterministic).  This covers batch 1-1024 and the long-K down
@@ -465,7 +468,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 SegWalker wk0(blockIdx.x, p);
                 Segment sg0;
                 while (npre < S && wk0.next(sg0)) {
-                    const int n_tile = (int)(sg0.tile / p.m_tiles);
+                    const int n_tile = (int)(sg0.tile % p.n_tiles);
                     for (int kt = sg0.kt0; kt < sg0.kt1 && npre < S; kt++, npre++) {
                         if (!leader) continue;
                         const uint32_t st = smem_base + npre * p.stage_bytes;
@@ -492,7 +495,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             bool ok = true;
             int ready_band = -1;
             while (ok && wk.next(sg)) {
-                const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
+                const int n_tile = (int)(sg.tile % p.n_tiles), m_tile = (int)(sg.tile / p.n_tiles);
                 if (p.band_ready && n_tile != ready_band) {
                     // the rows of this tile come from the decoder running beside us
                     const int64_t t0 = (int64_t)n_tile * p.band_tasks;
@@ -627,7 +630,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         RingPos rp;
         bool ok = true;
         while (ok && wk.next(sg)) {
-            const int64_t n0 = (sg.tile / p.m_tiles) * kBlockN;
+            const int64_t n0 = (int64_t)(sg.tile % p.n_tiles) * kBlockN;
             for (int kt = sg.kt0; kt < sg.kt1; kt++, q++, rp.advance(S)) {
                 // A ring slot always belongs to the same group (slot parity),
                 // so a group's waits on a slot see consecutive mbarrier
@@ -676,7 +679,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         const int AW4 = p.acc_w / 4;
         bool ok = true;
         while (ok && wk.next(sg)) {
-            const int n_tile = (int)(sg.tile / p.m_tiles), m_tile = (int)(sg.tile % p.m_tiles);
+            const int n_tile = (int)(sg.tile % p.n_tiles), m_tile = (int)(sg.tile / p.n_tiles);
             const int64_t n = (int64_t)n_tile * kBlockN + r;
             const int64_t m0 = (int64_t)m_tile * p.MG;
             const bool whole = sg.kt0 == 0 && sg.kt1 == p.kt_count;
