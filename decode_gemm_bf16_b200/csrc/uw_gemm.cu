@@ -73,13 +73,15 @@ constexpr int kThreadsRecon = (kReconWarp0 + kReconWarps) * 32;
 // source), sign+mantissa 128 x KB bytes, exponents 128 x KB bytes or palette
 // indices 128 x KB/2 bytes, and KB/64 words of 128 verbatim flags.
 constexpr uint32_t kTileA64 = kBlockN * kBoxK * 2;       // 16 KB: one 64-k box of BF16 weights
-constexpr int kFinBufs = 4;                              // finisher staging rows in flight per warp
+constexpr uint32_t kVSlot = 128;     // shared bytes per verbatim-flag slot (stage, matrix) of the flag ring
+constexpr uint32_t kStgBytes = 4096; // output transpose buffers: 1 KB per epilogue warp
+constexpr int kEpiBar = 1;           // named barrier of the four epilogue warps
 
 // One weight matrix's planes as a stage sees them: where its TMA tiles sit
 // in the stage, its verbatim store and its palette.  A paired call (gate and
 // up projections, SwiGLU epilogue) carries two.
 struct PlaneSet {
-    uint32_t off_sm, off_s2, off_v;   // stage offsets: sign+mantissa, exponent/index, verbatim flags
+    uint32_t off_sm, off_s2;          // stage offsets: sign+mantissa, exponent/index
     int pal_small;                    // all palette exponents < 128: cheaper lookup
     const uint32_t* vbits;
     const uint32_t* vpre;
@@ -100,7 +102,9 @@ struct GemmParams {
     void* Y;
     int out_f32;
     float* partial;                // [2P][MG/4][128][4]: float4 j of row r at (slot*MG/4 + j)*128 + r
-    int fin_cb;                    // finisher column block (16, 32 or 64)
+    uint32_t vring_off;            // shared offset of the verbatim-flag ring (kVSlot per stage and matrix)
+    uint32_t stg_off;              // shared offset of the epilogue warps' transpose buffers (1 KB each)
+    int y_vec;                     // outputs leave in 16-byte runs (else element stores)
     unsigned long long* flags;     // [2P][128]: call tag once a slot's row is published
     unsigned long long epoch;      // 48-bit tag of this call
     // decoder running beside the GEMM: band b of 128 rows is ready when
@@ -180,10 +184,11 @@ __device__ __forceinline__ uint32_t sw32_off(int r, int c) { return r * 32 + ((c
 // Rebuilds weight row r = 32q + lane, k = 32j .. 32j+31 of the stage's tile
 // (stage of KB k at stage index kt) and writes it to TMEM lane r, columns
 // taddr .. +15 (one BF16 pair per column).  Sign+mantissa and exponent
-// tiles have rows of KB bytes (swizzle KB), index tiles rows of KB/2 bytes.
+// tiles have rows of KB bytes (swizzle KB), index tiles rows of KB/2 bytes;
+// the stage's verbatim flags (KB/64 words of 128 rows) sit at `vflags`.
 template <int SRC, int KB>
-__device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet& ps, uint32_t stage, int64_t n0,
-                                            int kt, int q, int j, int lane, uint32_t taddr) {
+__device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet& ps, uint32_t stage, uint32_t vflags,
+                                            int64_t n0, int kt, int q, int j, int lane, uint32_t taddr) {
     const int r = 32 * q + lane;
     auto row_off = [&](int c) { return KB == 128 ? sw128_off(r, c) : sw64_off(r, c); };
     const uint32_t SM = stage + ps.off_sm;
@@ -198,7 +203,7 @@ __device__ __forceinline__ void rebuild_row(const GemmParams& p, const PlaneSet&
         E[4] = e1.x; E[5] = e1.y; E[6] = e1.z; E[7] = e1.w;
     } else {
         const int grp = j >> 1;   // 64-weight group within the stage
-        const uint32_t vw = lds32(stage + ps.off_v + 16 * grp + 4 * q);
+        const uint32_t vw = lds32(vflags + 16 * grp + 4 * q);
         if ((vw >> lane) & 1u) {
             // verbatim group: raw exponents from the verbatim store
             const int64_t g = (n0 + r) * p.KG + (int64_t)kt * (KB / kGroup) + grp;
@@ -272,11 +277,84 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&g)[16], const uint32_t
     }
 }
 
+// True on all four epilogue warps when `pred` holds on any of their threads
+// (a barrier with an OR reduction).
+__device__ __forceinline__ bool epi_any(bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)pred), "n"(kEpiBar), "n"(4 * 32)
+        : "memory");
+    return res != 0;
+}
+
+// Where finished outputs go.  Thread r of the four epilogue warps holds
+// output row n0 + r for 16 consecutive batch rows, so a direct store writes
+// 2 bytes per lane at 16 addresses N apart.  Instead each warp transposes
+// its 32 rows x 16 batch rows through its own 1 KB of shared memory
+// (BF16; fp32 goes 8 batch rows at a time) and writes them back with
+// 16-byte stores, four lanes per 64-byte run of a batch row: 2 vector
+// stores a lane instead of 16 scalar ones.  Without 16-byte rows (Y
+// misaligned, N not a multiple of 8 BF16 / 4 fp32) every thread stores its
+// own elements.
+struct EpiCtx {
+    void* Y;
+    int64_t M, N;
+    int out_f32, vec;
+    uint32_t stg;   // shared address of this warp's 1 KB transpose buffer
+};
+
+// Outputs Y[m .. m+15, n0 + r] = v[0..15] (fp32 bit patterns); called by
+// whole warps (the same m).
+__device__ __forceinline__ void emit16(const EpiCtx& e, const uint32_t (&v)[16], int64_t n0, int r, int64_t m) {
+    if (!e.vec) {
+        store_y(e.Y, e.M, e.N, e.out_f32, v, n0 + r, m);
+        return;
+    }
+    const int lane = r & 31;
+    const int64_t nw = n0 + (r & ~31);   // this warp's first output row
+    if (e.out_f32) {
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            if (m + 8 * h >= e.M) break;
+#pragma unroll
+            for (int i = 0; i < 8; i++) sts32(e.stg + (uint32_t)(i * 128 + lane * 4), v[8 * h + i]);
+            __syncwarp();
+#pragma unroll
+            for (int s = 0; s < 2; s++) {
+                const int idx = s * 32 + lane, t = idx >> 3, seg = idx & 7;
+                const uint4 x = lds128(e.stg + (uint32_t)(t * 128 + seg * 16));
+                const int64_t mt = m + 8 * h + t, nn = nw + seg * 4;
+                if (mt < e.M && nn < e.N) *reinterpret_cast<uint4*>(reinterpret_cast<float*>(e.Y) + mt * e.N + nn) = x;
+            }
+            __syncwarp();
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) sts16(e.stg + (uint32_t)(i * 64 + lane * 2), f2bf(__uint_as_float(v[i])));
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < 2; s++) {
+            const int idx = s * 32 + lane, t = idx >> 2, seg = idx & 3;
+            const uint4 x = lds128(e.stg + (uint32_t)(t * 64 + seg * 16));
+            const int64_t mt = m + t, nn = nw + seg * 8;
+            if (mt < e.M && nn < e.N) *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(e.Y) + mt * e.N + nn) = x;
+        }
+        __syncwarp();
+    }
+}
+
 // Output of a finished accumulator in TMEM: Y directly, or (paired gate and
-// up accumulators) SwiGLU of the two halves.
-__device__ __forceinline__ void write_out(void* Y, int64_t M, int64_t N, int out_f32, int MG, int nh, uint32_t trow,
-                                          int64_t n, int64_t m0) {
+// up accumulators) SwiGLU of the two halves.  Accumulator columns of batch
+// rows past M are skipped.
+__device__ __forceinline__ void write_out(const EpiCtx& e, int MG, int nh, uint32_t trow, int64_t n0, int r,
+                                          int64_t m0) {
     for (int c0 = 0; c0 < MG; c0 += 16) {
+        if (m0 + c0 >= e.M) break;
         uint32_t v[16];
         tmem_ld16(trow + (uint32_t)c0, v);
         if (nh == 2) {
@@ -284,106 +362,114 @@ __device__ __forceinline__ void write_out(void* Y, int64_t M, int64_t N, int out
             tmem_ld16(trow + (uint32_t)(MG + c0), u);
             tmem_wait_ld();
             swiglu16(v, u, h);
-            store_y(Y, M, N, out_f32, h, n, m0 + c0);
+            emit16(e, h, n0, r, m0 + c0);
         } else {
             tmem_wait_ld();
-            store_y(Y, M, N, out_f32, v, n, m0 + c0);
+            emit16(e, v, n0, r, m0 + c0);
         }
     }
 }
 
 // Finisher of a split tile: own accumulator (TMEM) + the partial rows of
-// CTAs blockIdx.x + 1 .. b_last in that order, then Y.  Columns go in blocks
-// of CB; this warp's accumulator rows (32 x CB) and kFinBufs staging rows
-// live in `fin` (rows of CB + 4 floats: a 16-byte bank shift per lane), and
-// the (block, contributor) items stream in with asynchronous copies,
-// kFinBufs - 1 ahead.  A paired accumulator (gate and up halves) is summed
-// back into TMEM and written through the SwiGLU afterwards.  Kept out of
-// line: it runs once per CTA and would otherwise set the register budget of
-// the whole kernel.
+// CTAs blockIdx.x + 1 .. b_last, added in that (k) order, then Y.  The
+// finisher's segment is its CTA's last, so the stage ring is idle: the
+// contributors' partials come into it with bulk copies.  A contributor's
+// partial is stored as float4 columns of 128 rows, so any block of columns
+// of it is one contiguous piece; the columns go in blocks as wide as the
+// ring holds for every contributor (and both halves of a paired tile), one
+// round of copies per block.  Kept out of line: it runs once per CTA and
+// would otherwise set the register budget of the whole kernel.
 struct FinArgs {
     const float* partial;
-    void* Y;
-    int64_t M, N;
-    int AW, MG, nh, CB, out_f32;   // accumulator columns (nh * MG), output columns, halves
+    uint32_t ring, ring_bytes, bar;   // idle stage ring and its mbarrier (shared addresses)
+    int AW, MG, nh;                   // accumulator columns (nh * MG), output columns, halves
     uint32_t total, P, kt;
+    uint64_t timeout_ns;
 };
 
-__device__ __noinline__ void finish_tile(const FinArgs f, uint32_t tile, uint32_t b_last, int64_t n, int64_t m0,
-                                         uint32_t trow, float* fin, int lane) {
-    const int CB = f.CB, RS = CB + 4;
-    const int AW4 = f.AW / 4;
-    const int r = (int)(threadIdx.x & 127);
+// Returns the updated finisher barrier phase.
+__device__ __noinline__ uint32_t finish_tile(const FinArgs f, const EpiCtx e, uint32_t fin_phase,
+                                          uint32_t tile, uint32_t b_last, int64_t n0, int r, int64_t m0, uint32_t trow,
+                                          volatile int* abort_flag) {
     const uint32_t nb = b_last - blockIdx.x;   // contributors, in k order after this CTA
-    const uint32_t nblk = (uint32_t)((f.AW + CB - 1) / CB);
-    const uint32_t items = nb * nblk;
-    float* facc = fin + lane * RS;
-    const uint32_t fbuf = smem_u32(fin + 32 * RS + lane * RS);   // staging rows, 32*RS floats apart
-    const float4* part4 = reinterpret_cast<const float4*>(f.partial);
-    // item t = (block t / nb, contributor t % nb) -> staging row t % kFinBufs;
-    // every call commits one group (possibly empty) so that groups count items
-    auto issue = [&](uint32_t t) {
-        if (t < items) {
-            const uint32_t blk = t / nb, i = t - blk * nb;
-            const int cb0 = (int)blk * CB;
-            const int cw = f.AW - cb0 < CB ? f.AW - cb0 : CB;
-            const uint32_t sl = slot_of(blockIdx.x + 1 + i, tile, f.total, f.P, f.kt);
-            const float4* src = part4 + ((size_t)sl * AW4 + cb0 / 4) * kBlockN + r;
-            const uint32_t dst = fbuf + (t % kFinBufs) * (uint32_t)(32 * RS * 4);
-            for (int q = 0; q < cw / 4; q++) cp_async16(dst + 16u * q, src + (size_t)q * kBlockN);
+    const uint32_t col_bytes = kBlockN * 4u;   // one column of one partial
+    const size_t slot_floats = (size_t)f.AW * kBlockN;
+    // Block width: the widest multiple of 16 columns that the ring holds for
+    // every contributor; when not even 16 do, blocks of 16 columns take the
+    // contributors in rounds, and the running sum goes back into TMEM
+    // between rounds.
+    const uint32_t unit = (uint32_t)f.nh * col_bytes * 16u;
+    uint32_t CB = 16, R = f.ring_bytes / unit;
+    if (nb * unit <= f.ring_bytes) {
+        R = nb;
+        CB = (f.ring_bytes / (nb * (uint32_t)f.nh * col_bytes)) & ~15u;
+        if (CB > (uint32_t)f.MG) CB = (uint32_t)f.MG;
+    }
+    for (int cb0 = 0; cb0 < f.MG; cb0 += (int)CB) {
+        if (m0 + cb0 >= e.M) break;   // batch rows past M: never output
+        const uint32_t cw = (uint32_t)f.MG - (uint32_t)cb0 < CB ? (uint32_t)f.MG - (uint32_t)cb0 : CB;
+        const uint32_t piece = cw * col_bytes;
+        for (uint32_t i0 = 0; i0 < nb; i0 += R) {
+        const uint32_t cnt = nb - i0 < R ? nb - i0 : R;
+        const bool last = i0 + cnt == nb;
+        named_bar_sync(kEpiBar, 4 * 32);   // the ring is no longer read (previous round, or the MMA)
+        if (r == 0) {
+            // the tags acquired before (one per row, ordered before this
+            // thread by the barrier) cover the partials; the copies read
+            // them through the async proxy
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(f.bar, cnt * (uint32_t)f.nh * piece);
+            for (uint32_t i = 0; i < cnt; i++) {
+                const uint32_t sl = slot_of(blockIdx.x + 1 + i0 + i, tile, f.total, f.P, f.kt);
+                for (int h = 0; h < f.nh; h++)
+                    bulk_load(f.ring + (i * (uint32_t)f.nh + (uint32_t)h) * piece,
+                              f.partial + (size_t)sl * slot_floats + (size_t)(h * f.MG + cb0) * kBlockN, piece, f.bar);
+            }
         }
-        cp_async_commit();
-    };
-    for (uint32_t t = 0; t + 1 < (uint32_t)kFinBufs; t++) issue(t);
-    uint32_t t = 0;
-    for (uint32_t blk = 0; blk < nblk; blk++) {
-        const int cb0 = (int)blk * CB;
-        const int cw = f.AW - cb0 < CB ? f.AW - cb0 : CB;
-        for (int c = 0; c < cw; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(trow + (uint32_t)(cb0 + c), v);
+        mbar_wait(f.bar, fin_phase, f.timeout_ns, abort_flag);
+        fin_phase ^= 1u;
+        for (int c0 = cb0; c0 < cb0 + (int)cw; c0 += 16) {
+            if (m0 + c0 >= e.M) break;
+            uint32_t v[16], u[16];
+            tmem_ld16(trow + (uint32_t)c0, v);
+            if (f.nh == 2) tmem_ld16(trow + (uint32_t)(f.MG + c0), u);
             tmem_wait_ld();
-            float4* a4 = reinterpret_cast<float4*>(facc + c);
+            for (uint32_t i = 0; i < cnt; i++) {
+                const uint32_t base = f.ring + i * (uint32_t)f.nh * piece + (uint32_t)(c0 - cb0) * col_bytes + (uint32_t)r * 16u;
 #pragma unroll
-            for (int i = 0; i < 4; i++)
-                a4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-        }
-        for (uint32_t i = 0; i < nb; i++, t++) {
-            issue(t + kFinBufs - 1);
-            cp_async_wait<kFinBufs - 1>();   // item t has landed
-            const float4* b4 = reinterpret_cast<const float4*>(fin + (1 + t % kFinBufs) * 32 * RS + lane * RS);
-            float4* a4 = reinterpret_cast<float4*>(facc);
-            for (int q = 0; q < cw / 4; q++) {
-                float4 x = a4[q];
-                const float4 y = b4[q];
-                x.x += y.x;
-                x.y += y.y;
-                x.z += y.z;
-                x.w += y.w;
-                a4[q] = x;
+                for (int q = 0; q < 4; q++) {
+                    const uint4 x = lds128(base + (uint32_t)q * (4u * col_bytes));
+                    v[4 * q] = __float_as_uint(__uint_as_float(v[4 * q]) + __uint_as_float(x.x));
+                    v[4 * q + 1] = __float_as_uint(__uint_as_float(v[4 * q + 1]) + __uint_as_float(x.y));
+                    v[4 * q + 2] = __float_as_uint(__uint_as_float(v[4 * q + 2]) + __uint_as_float(x.z));
+                    v[4 * q + 3] = __float_as_uint(__uint_as_float(v[4 * q + 3]) + __uint_as_float(x.w));
+                }
+                if (f.nh == 2) {
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        const uint4 x = lds128(base + piece + (uint32_t)q * (4u * col_bytes));
+                        u[4 * q] = __float_as_uint(__uint_as_float(u[4 * q]) + __uint_as_float(x.x));
+                        u[4 * q + 1] = __float_as_uint(__uint_as_float(u[4 * q + 1]) + __uint_as_float(x.y));
+                        u[4 * q + 2] = __float_as_uint(__uint_as_float(u[4 * q + 2]) + __uint_as_float(x.z));
+                        u[4 * q + 3] = __float_as_uint(__uint_as_float(u[4 * q + 3]) + __uint_as_float(x.w));
+                    }
+                }
+            }
+            if (!last) {
+                tmem_st16(trow + (uint32_t)c0, v);   // running sum, back into the accumulator
+                if (f.nh == 2) tmem_st16(trow + (uint32_t)(f.MG + c0), u);
+            } else if (f.nh == 2) {
+                uint32_t h[16];
+                swiglu16(v, u, h);
+                emit16(e, h, n0, r, m0 + c0);
+            } else {
+                emit16(e, v, n0, r, m0 + c0);
             }
         }
-        for (int c = 0; c < cw; c += 16) {
-            uint32_t v[16];
-            const uint4* a4 = reinterpret_cast<const uint4*>(facc + c);
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const uint4 x = a4[i];
-                v[4 * i] = x.x;
-                v[4 * i + 1] = x.y;
-                v[4 * i + 2] = x.z;
-                v[4 * i + 3] = x.w;
-            }
-            if (f.nh == 2) tmem_st16(trow + (uint32_t)(cb0 + c), v);   // the sum, back into the accumulator
-            else store_y(f.Y, f.M, f.N, f.out_f32, v, n, m0 + cb0 + c);
+        if (!last) tmem_wait_st();
         }
     }
-    cp_async_wait<0>();
-    if (f.nh == 2) {
-        tmem_wait_st();
-        write_out(f.Y, f.M, f.N, f.out_f32, f.MG, 2, trow, n, m0);
-    }
+    return fin_phase;
 }
 
 template <int SRC, int KB, int NH>
@@ -404,7 +490,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     uint64_t* accf_bar = empty_bar + kMaxStages;
     uint64_t* acce_bar = accf_bar + 1;
     uint64_t* final_bar = acce_bar + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    uint64_t* fin_bar = final_bar + 1;   // finisher: contributors' partials landed in the ring
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -422,6 +509,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         mbar_init(smem_u32(accf_bar), 1);
         mbar_init(smem_u32(acce_bar), kEpiWarps);
         mbar_init(smem_u32(final_bar), 1);
+        mbar_init(smem_u32(fin_bar), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -450,6 +538,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     if (warp != kProdWarp) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t smem_base = smem_u32(smem);
+    const uint32_t vring = smem_base + p.vring_off;
 
     if (warp == kProdWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -479,7 +568,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                             const PlaneSet& ps = p.ps[h];
                             tma_load_2d(st + ps.off_sm, maps_a[h], kt * KB, n_tile * kBlockN, fb);
                             if (SRC == kSrcPalette) {
-                                tma_load_2d(st + ps.off_v, maps_v[h], n_tile * (kBlockN / 32), kt * kHalves, fb);
+                                tma_load_2d(vring + (uint32_t)(npre * NH + h) * kVSlot, maps_v[h],
+                                            n_tile * (kBlockN / 32), kt * kHalves, fb);
                                 if (p.static_s2)
                                     tma_load_2d(st + ps.off_s2, maps_s2[h], kt * (KB / 2), n_tile * kBlockN, fb);
                             }
@@ -544,7 +634,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                                 tma_load_2d(st + ps.off_s2, maps_s2[h], kt * KB, n_tile * kBlockN, fb);
                             else {
                                 tma_load_2d(st + ps.off_s2, maps_s2[h], kt * (KB / 2), n_tile * kBlockN, fb);
-                                tma_load_2d(st + ps.off_v, maps_v[h], n_tile * (kBlockN / 32), kt * kHalves, fb);
+                                tma_load_2d(vring + (uint32_t)(s * NH + h) * kVSlot, maps_v[h],
+                                            n_tile * (kBlockN / 32), kt * kHalves, fb);
                             }
                         }
                     }
@@ -647,7 +738,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 #pragma unroll
                     for (int pc = 0; pc < kPieces; pc++) {
                         const int j = hh * kPieces + pc;
-                        rebuild_row<SRC, KB>(p, p.ps[h], smem_base + (uint32_t)s * p.stage_bytes, n0, kt, quarter, j, lane,
+                        rebuild_row<SRC, KB>(p, p.ps[h], smem_base + (uint32_t)s * p.stage_bytes,
+                                             vring + (uint32_t)(s * NH + h) * kVSlot, n0, kt, quarter, j, lane,
                                              tlane + (uint32_t)(KB / 2) * (uint32_t)(NH * s + h) + 16u * (uint32_t)j);
                     }
                 }
@@ -665,39 +757,37 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         // waits for the tags, adds the partials to its own accumulator in k
         // order and writes Y, then clears the tags for a replay of this call.
         // Partials are stored float4-interleaved across rows, so every warp
-        // access covers 512 contiguous bytes.  The finisher's segment is its
-        // CTA's last, so the stage ring is idle by then: it stages partial
-        // rows there with asynchronous copies (one round trip per block of
-        // columns and contributor instead of one per 16 columns).
+        // access covers 512 contiguous bytes and one contributor's partial is
+        // one contiguous block.  The four warps decide together to stop on a
+        // failed wait: the finisher synchronises them.
         SegWalker wk(blockIdx.x, p);
         Segment sg;
         int j = 0;
         const int r = warp * 32 + lane;
         const uint32_t trow = tacc + ((uint32_t)(warp * 32) << 16);
-        // finisher staging: this warp's 1 + kFinBufs rows-of-32 of fin_cb + 4 floats
-        float* fin = reinterpret_cast<float*>(smem) + (size_t)warp * (1 + kFinBufs) * 32 * (p.fin_cb + 4);
         const int AW4 = p.acc_w / 4;
-        bool ok = true;
-        while (ok && wk.next(sg)) {
+        const EpiCtx ec = {p.Y, p.M, p.N, p.out_f32, p.y_vec, smem_base + p.stg_off + (uint32_t)warp * 1024u};
+        uint32_t fin_phase = 0;
+        while (wk.next(sg)) {
             const int n_tile = (int)(sg.tile % p.n_tiles), m_tile = (int)(sg.tile / p.n_tiles);
-            const int64_t n = (int64_t)n_tile * kBlockN + r;
+            const int64_t n0 = (int64_t)n_tile * kBlockN;
             const int64_t m0 = (int64_t)m_tile * p.MG;
             const bool whole = sg.kt0 == 0 && sg.kt1 == p.kt_count;
             const bool finisher = !whole && sg.kt0 == 0;
             const uint32_t kt = (uint32_t)p.kt_count;
             const uint32_t b_last = finisher ? iter_owner(sg.tile * kt + kt - 1, p.total_iters, p.P) : 0u;
-            if (finisher) {
-                for (uint32_t b = blockIdx.x + 1; ok && b <= b_last; b++) {
+            bool good = true;
+            if (finisher)
+                for (uint32_t b = blockIdx.x + 1; good && b <= b_last; b++) {
                     const uint32_t sl = slot_of(b, sg.tile, p.total_iters, p.P, kt);
-                    ok = wait_tag(p.flags + (size_t)sl * kBlockN + r, p.epoch, p.timeout_ns, abort_flag);
+                    good = wait_tag(p.flags + (size_t)sl * kBlockN + r, p.epoch, p.timeout_ns, abort_flag);
                 }
-                if (!ok) break;
-            }
-            if (!mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000)) break;
+            if (good) good = mbar_wait(smem_u32(accf_bar), (uint32_t)(j & 1), p.timeout_ns, abort_flag, 20000);
+            if (epi_any(!good)) break;
             tc_fence_after();
             const uint32_t slot = 2u * blockIdx.x + (sg.first ? 0u : 1u);
             if (whole) {
-                write_out(p.Y, p.M, p.N, p.out_f32, p.MG, NH, trow, n, m0);
+                write_out(ec, p.MG, NH, trow, n0, r, m0);
             } else if (!finisher) {
                 // publish the partial rows (every accumulator column)
                 float4* dst = reinterpret_cast<float4*>(p.partial) + (size_t)slot * AW4 * kBlockN + r;
@@ -711,9 +801,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                                                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
                 }
             } else {
-                const FinArgs fa = {p.partial, p.Y, p.M, p.N, p.acc_w, p.MG, NH, p.fin_cb, p.out_f32,
-                                    p.total_iters, (uint32_t)p.P, kt};
-                finish_tile(fa, sg.tile, b_last, n, m0, trow, fin, lane);
+                const FinArgs fa = {p.partial, smem_base, (uint32_t)p.stages * p.stage_bytes, smem_u32(fin_bar),
+                                    p.acc_w, p.MG, NH, p.total_iters, (uint32_t)p.P, kt, p.timeout_ns};
+                fin_phase = finish_tile(fa, ec, fin_phase, sg.tile, b_last, n0, r, m0, trow, abort_flag);
             }
             tc_fence_before();
             __syncwarp();
@@ -1007,16 +1097,21 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
                 off = al1k(ps.off_s2 + sm_bytes);
                 p.tx_bytes += 2 * sm_bytes;
             } else {
-                ps.off_v = al1k(ps.off_s2 + idx_bytes);
-                off = al1k(ps.off_v + v_bytes);
+                // (the stage's verbatim flags go to the flag ring)
+                off = al1k(ps.off_s2 + idx_bytes);
                 p.tx_bytes += sm_bytes + idx_bytes + v_bytes;
             }
         }
     }
     p.stage_bytes = al1k(off);
+    // after the ring: barriers (1 KB), the verbatim-flag ring (palette
+    // source: kVSlot per stage and matrix), the output transpose buffers;
+    // plus 1 KB to align the dynamic shared memory base
     const size_t ctrl = 1024;
-    size_t budget = 227 * 1024 - 1024 - ctrl;
-    if (a.smem_cap > 0 && (size_t)a.smem_cap < budget + 2048) budget = (size_t)a.smem_cap - 2048;
+    const size_t vring = a.src == kSrcPalette ? al1k((uint32_t)(kMaxStages * NH) * kVSlot) : 0;
+    const size_t reserved = 1024 + ctrl + vring + kStgBytes;
+    size_t budget = 227 * 1024 - reserved;
+    if (a.smem_cap > 0 && (size_t)a.smem_cap < budget + reserved) budget = (size_t)a.smem_cap - reserved;
     int S = (int)(budget / p.stage_bytes);
     if (S > kMaxStages) S = kMaxStages;
     if (a.stages >= 2 && S > a.stages) S = a.stages;
@@ -1031,20 +1126,20 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     }
     if (S < 2) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
     p.stages = S;
-    // finisher staging in the idle ring: 4 warps x (1 + kFinBufs) rows-of-32 x (CB + 4) floats
-    p.fin_cb = 0;
-    for (int cb = 64; cb >= 16; cb >>= 1)
-        if (cb <= p.acc_w && (size_t)4 * (1 + kFinBufs) * 32 * (cb + 4) * 4 <= (size_t)S * p.stage_bytes) {
-            p.fin_cb = cb;
-            break;
-        }
-    if (p.fin_cb == 0) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
+    // the finisher brings at least 16 columns of one contributor's partial
+    // into the idle ring at once
+    if (sp.fixup && (size_t)NH * 16 * kBlockN * 4 > (size_t)S * p.stage_bytes) {
+        *st = UW_ERR_UNSUPPORTED;
+        return cudaSuccess;
+    }
+    p.vring_off = (uint32_t)((size_t)S * p.stage_bytes + ctrl);
+    p.stg_off = (uint32_t)(p.vring_off + vring);
     p.a_col0 = acc_cols;
     uint32_t need_cols = a.src == kSrcDense ? acc_cols : acc_cols + (uint32_t)(NH * KB / 2) * (uint32_t)S;
     p.tmem_cols = 32;
     while (p.tmem_cols < need_cols) p.tmem_cols <<= 1;
     if (p.tmem_cols > 512) { *st = UW_ERR_UNSUPPORTED; return cudaSuccess; }
-    size_t smem = (size_t)S * p.stage_bytes + ctrl + 1024;
+    size_t smem = (size_t)S * p.stage_bytes + reserved;
 
     CUtensorMap tx{}, ta{}, ts2{}, tv{}, ta2{}, ts22{}, tv2{};
     bool ok = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, a.K, a.M, a.K * 2, kBoxK, p.MG,
@@ -1082,6 +1177,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
         tv2 = tv;
     }
     if (!ok) { *st = UW_ERR_CUDA; return cudaSuccess; }
+    // Y in 16-byte runs of a batch row where its rows allow (see emit16)
+    const size_t ye = a.out_f32 ? 4 : 2;
+    p.y_vec = ((uintptr_t)a.Y % 16 == 0) && (a.N * ye) % 16 == 0;
 
     typedef void (*GemmKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                                const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams);
