@@ -31,6 +31,10 @@ MS = [1, 3, 16, 17, 64, 100, 256, 300]
 _cache = {}
 
 
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
 def _case(shape):
     if shape not in _cache:
         W = SHAPES[shape]()
@@ -209,12 +213,13 @@ def test_workspace_contents_do_not_matter(fill):
 @pytest.mark.parametrize("sm_dec", [1, 37, 148, 300])
 def test_decoder_beside_gemm(pipe, sm_dec):
     """Decoder CTAs running beside the GEMM (SM split): the GEMM waits for
-    each 128-row band; the result is the same as decode-then-GEMM."""
+    each 128-row band; the result is the same as decode-then-GEMM with one
+    k range per CTA (the split the GEMM beside a decoder uses)."""
     W, blob = _case("200x1408")
     X = S.activations(24, 1408, seed=11)
     R = O.gemm(X, W, "f32")
     Xd = dev16(X)
-    ref = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True))
+    ref = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True, grid=_sms()))
     for _ in range(2):
         Y = _f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True, sm_dec=sm_dec))
         check_gemm(Y, R, bf16_out=False)
@@ -227,7 +232,7 @@ def test_decoder_beside_gemm_full_size(gate_case):
     X = S.activations(16, 4096, seed=12)
     Xd = dev16(X)
     for pipe in ["exponent", "transcode"]:
-        ref = _f32(uw.uw_gemm(Xd, blob, pipe))
+        ref = _f32(uw.uw_gemm(Xd, blob, pipe, grid=_sms()))   # one k range per CTA, as beside a decoder
         Y = _f32(uw.uw_gemm(Xd, blob, pipe, sm_dec=74))
         assert np.array_equal(Y, ref)
         _sampled(X, W, Y, 64, seed=5, bf16_out=True)
@@ -650,4 +655,57 @@ def test_repeated_calls_bit_identical_full_size(gate_up_case, M):
         ref = fn().clone()
         for _ in range(30):
             assert torch.equal(fn(), ref), name
+    assert uw.uw_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_small_batch_full_size_gate_repeats(gate_case, M):
+    """Batch tiles of 16 rows on the default grid (stream-K over one CTA per
+    SM, cut tiles finished from the partials of the others): every output
+    against the oracle; repeated calls, and a CUDA graph replaying four of
+    them on one workspace (the per-row tags of one call must not be taken
+    for the next call's), give the same bits."""
+    W, blob = gate_case
+    X = S.activations(M, 4096, seed=120 + M)
+    Xd = dev16(X)
+    R = oracle_gemm(X, W, "f32")
+    Y = _f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True))
+    check_gemm(Y, R, bf16_out=False)
+    for _ in range(3):
+        assert np.array_equal(_f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True)), Y)
+    assert np.array_equal(_f32(uw.uw_gemm(Xd, blob, "direct_palette", out_f32=True, grid=_sms())), Y)
+    outs = [torch.empty(M, W.shape[0], dtype=torch.float32, device="cuda") for _ in range(4)]
+    ws = torch.zeros(uw.uw_gemm_workspace(blob, M, "direct_palette"), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for o in outs:
+            uw.uw_gemm(Xd, blob, "direct_palette", out=o, out_f32=True, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for o in outs:
+            uw.uw_gemm(Xd, blob, "direct_palette", out=o, out_f32=True, ws=ws)
+    for _ in range(3):
+        for o in outs:
+            o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for o in outs:
+            assert np.array_equal(o.cpu().numpy(), Y)
+    del g
+    assert uw.uw_last_device_status() == 0
+
+
+def test_dense_agrees_with_palette_batch8():
+    """The dense baseline and the rebuilding pipelines share the tile and
+    k-range split: equal bits at batch 8 on 40 row tiles cut by stream-K."""
+    W = S.weight_with_verbatim_rows(5120, 2048, seed=130, frac_groups=0.01)
+    blob = uw.uw_compress(dev16(W))
+    X = S.activations(8, 2048, seed=131)
+    Xd = dev16(X)
+    R = O.gemm(X, W, "f32")
+    Yd = _f32(uw.uw_dense_gemm(Xd, dev16(W), out_f32=True))
+    check_gemm(Yd, R, bf16_out=False)
+    for pipe in ["exponent", "transcode", "direct_palette"]:
+        assert np.array_equal(_f32(uw.uw_gemm(Xd, blob, pipe, out_f32=True)), Yd), pipe
     assert uw.uw_last_device_status() == 0
