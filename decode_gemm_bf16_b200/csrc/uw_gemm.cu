@@ -105,6 +105,10 @@ struct GemmParams {
     uint32_t vring_off;            // shared offset of the verbatim-flag ring (kVSlot per stage and matrix)
     uint32_t stg_off;              // shared offset of the epilogue warps' transpose buffers (1 KB each)
     int y_vec;                     // outputs leave in 16-byte runs (else element stores)
+    // SwiGLU in three launches: the finished accumulators go here instead
+    // of Y, per tile as float4 columns of 128 rows (block t at t * MG * 128
+    // floats; the stream-K partial layout)
+    float* gate_out;
     unsigned long long* flags;     // [2P][128]: call tag once a slot's row is published
     unsigned long long epoch;      // 48-bit tag of this call
     // decoder running beside the GEMM: band b of 128 rows is ready when
@@ -348,11 +352,31 @@ __device__ __forceinline__ void emit16(const EpiCtx& e, const uint32_t (&v)[16],
     }
 }
 
+// SwiGLU in three launches (batch tiles above 128 rows): the gate and the up
+// launch each store their finished accumulator columns c0 .. c0+15 of tile
+// `tile` (this thread's row r) as four float4 in the tile's block --
+// coalesced 512-byte warp stores, no conversion -- and k_swiglu_blocks
+// combines the two block arrays into H.
+struct GinCtx {
+    float* out;
+    int MG;
+};
+__device__ __forceinline__ void gin_emit(const GinCtx& gc, const uint32_t (&v)[16], uint32_t tile, int r, int c0) {
+    float4* dst = reinterpret_cast<float4*>(gc.out) + ((size_t)tile * (size_t)(gc.MG / 4) + (size_t)(c0 / 4)) * kBlockN +
+                  (size_t)r;
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+        dst[(size_t)q * kBlockN] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                               __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+}
+
 // Output of a finished accumulator in TMEM: Y directly, or (paired gate and
-// up accumulators) SwiGLU of the two halves.  Accumulator columns of batch
-// rows past M are skipped.
-__device__ __forceinline__ void write_out(const EpiCtx& e, int MG, int nh, uint32_t trow, int64_t n0, int r,
-                                          int64_t m0) {
+// up accumulators) SwiGLU of the two halves, or (GIN) SwiGLU with the gate
+// projection read from `gin`.  Accumulator columns of batch rows past M are
+// skipped.
+template <bool GIN>
+__device__ __forceinline__ void write_out(const EpiCtx& e, const GinCtx& gc, uint32_t tile, int MG, int nh, uint32_t trow,
+                                          int64_t n0, int r, int64_t m0) {
     for (int c0 = 0; c0 < MG; c0 += 16) {
         if (m0 + c0 >= e.M) break;
         uint32_t v[16];
@@ -365,7 +389,10 @@ __device__ __forceinline__ void write_out(const EpiCtx& e, int MG, int nh, uint3
             emit16(e, h, n0, r, m0 + c0);
         } else {
             tmem_wait_ld();
-            emit16(e, v, n0, r, m0 + c0);
+            if (GIN)
+                gin_emit(gc, v, tile, r, c0);
+            else
+                emit16(e, v, n0, r, m0 + c0);
         }
     }
 }
@@ -388,7 +415,8 @@ struct FinArgs {
 };
 
 // Returns the updated finisher barrier phase.
-__device__ __noinline__ uint32_t finish_tile(const FinArgs f, const EpiCtx e, uint32_t fin_phase,
+template <bool GIN>
+__device__ __noinline__ uint32_t finish_tile(const FinArgs f, const EpiCtx e, const GinCtx gc, uint32_t fin_phase,
                                           uint32_t tile, uint32_t b_last, int64_t n0, int r, int64_t m0, uint32_t trow,
                                           volatile int* abort_flag) {
     const uint32_t nb = b_last - blockIdx.x;   // contributors, in k order after this CTA
@@ -463,7 +491,10 @@ __device__ __noinline__ uint32_t finish_tile(const FinArgs f, const EpiCtx e, ui
                 swiglu16(v, u, h);
                 emit16(e, h, n0, r, m0 + c0);
             } else {
-                emit16(e, v, n0, r, m0 + c0);
+                if (GIN)
+                    gin_emit(gc, v, tile, r, c0);
+                else
+                    emit16(e, v, n0, r, m0 + c0);
             }
         }
         if (!last) tmem_wait_st();
@@ -472,7 +503,7 @@ __device__ __noinline__ uint32_t finish_tile(const FinArgs f, const EpiCtx e, ui
     return fin_phase;
 }
 
-template <int SRC, int KB, int NH>
+template <int SRC, int KB, int NH, bool GIN = false>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_a, const CUtensorMap& tm_s2,
                                           const CUtensorMap& tm_v, const CUtensorMap& tm_a2, const CUtensorMap& tm_s22,
                                           const CUtensorMap& tm_v2, const GemmParams& p) {
@@ -767,6 +798,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         const uint32_t trow = tacc + ((uint32_t)(warp * 32) << 16);
         const int AW4 = p.acc_w / 4;
         const EpiCtx ec = {p.Y, p.M, p.N, p.out_f32, p.y_vec, smem_base + p.stg_off + (uint32_t)warp * 1024u};
+        const GinCtx gc = {p.gate_out, p.MG};
         uint32_t fin_phase = 0;
         while (wk.next(sg)) {
             const int n_tile = (int)(sg.tile % p.n_tiles), m_tile = (int)(sg.tile / p.n_tiles);
@@ -787,7 +819,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             tc_fence_after();
             const uint32_t slot = 2u * blockIdx.x + (sg.first ? 0u : 1u);
             if (whole) {
-                write_out(ec, p.MG, NH, trow, n0, r, m0);
+                write_out<GIN>(ec, gc, sg.tile, p.MG, NH, trow, n0, r, m0);
             } else if (!finisher) {
                 // publish the partial rows (every accumulator column)
                 float4* dst = reinterpret_cast<float4*>(p.partial) + (size_t)slot * AW4 * kBlockN + r;
@@ -803,7 +835,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             } else {
                 const FinArgs fa = {p.partial, smem_base, (uint32_t)p.stages * p.stage_bytes, smem_u32(fin_bar),
                                     p.acc_w, p.MG, NH, p.total_iters, (uint32_t)p.P, kt, p.timeout_ns};
-                fin_phase = finish_tile(fa, ec, fin_phase, sg.tile, b_last, n0, r, m0, trow, abort_flag);
+                fin_phase = finish_tile<GIN>(fa, ec, gc, fin_phase, sg.tile, b_last, n0, r, m0, trow, abort_flag);
             }
             tc_fence_before();
             __syncwarp();
@@ -867,6 +899,18 @@ __global__ void __maxnreg__(80)
                   const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
                   const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
     gemm_body<kSrcPalette, KB, 2>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
+}
+
+// SwiGLU in three launches (batch tiles above 128 rows, where a paired tile
+// would be capped at 128), direct palette: the gate and the up launch keep
+// their accumulators per tile in the workspace.
+template <int KB>
+__global__ void __maxnreg__(80)
+    k_gemm_recon_gin(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_s2, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_s22,
+                     const __grid_constant__ CUtensorMap tm_v2, const GemmParams p) {
+    gemm_body<kSrcPalette, KB, 1, true>(tm_x, tm_a, tm_s2, tm_v, tm_a2, tm_s22, tm_v2, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1035,11 +1079,11 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (a.M == 0) return cudaSuccess;
     if (a.variant < UW_VARIANT_AUTO || a.variant > UW_VARIANT_GEMV) { *st = UW_ERR_INVALID_ARG; return cudaSuccess; }
     const int NH = a.pair ? 2 : 1;
-    if (a.pair && (a.src != kSrcPalette || a.variant == UW_VARIANT_GEMV || a.band_ready)) {
+    if ((a.pair || a.gate_out) && (a.src != kSrcPalette || a.variant == UW_VARIANT_GEMV || a.band_ready || a.smem_cap > 0)) {
         *st = UW_ERR_UNSUPPORTED;
         return cudaSuccess;
     }
-    if (!a.pair && gemv_serves(a)) return launch_gemv(a, s, st);
+    if (!a.pair && !a.gate_out && gemv_serves(a)) return launch_gemv(a, s, st);
     const GemmSplit sp = gemm_split(a.M, a.N, a.K, a.grid, a.split_k, NH);
     if (!sp.ok) { *st = a.split_k > 0 ? UW_ERR_INVALID_ARG : UW_ERR_SHAPE; return cudaSuccess; }
     GemmParams p{};
@@ -1061,6 +1105,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     if (a.pair) set_planes(p.ps[1], a.palette2, a.vbits2, a.vpre2, a.vexp2);
     p.Y = a.Y;
     p.out_f32 = a.out_f32;
+    p.gate_out = a.gate_out;
     size_t need = gemm_ws_bytes(a.M, a.N, a.K, a.grid, a.split_k, NH);
     if (!a.ws || a.ws_bytes < need) { *st = UW_ERR_WORKSPACE; return cudaSuccess; }
     size_t part = sp.fixup ? (size_t)2 * P * p.acc_w * kBlockN * 4 : 0;
@@ -1184,7 +1229,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     typedef void (*GemmKernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                                const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmParams);
     GemmKernel kern;
-    if (a.pair)
+    if (a.gate_out)
+        kern = KB == 128 ? k_gemm_recon_gin<128> : k_gemm_recon_gin<64>;
+    else if (a.pair)
         kern = KB == 128 ? k_gemm_swiglu<128> : k_gemm_swiglu<64>;
     else if (a.smem_cap > 0 && a.src != kSrcDense)   // room left for decoder CTAs beside
         kern = KB == 128 ? (a.src == kSrcExponent ? k_gemm_recon_beside<kSrcExponent, 128>
@@ -1212,6 +1259,55 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, tx, ta, ts2, tv, ta2, ts22, tv2, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// H[m, n] = silu(G) * U from the two launches' tile blocks: thread = one
+// float4 column group (4 batch rows) of one output row; a warp covers 32
+// consecutive output rows, so its loads are 512 contiguous bytes and its
+// stores 32 consecutive outputs of a batch row.
+__global__ void __launch_bounds__(256) k_swiglu_blocks(const float4* __restrict__ G, const float4* __restrict__ U, void* H,
+                                                       int64_t M, int64_t N, int MG, int n_tiles, int64_t groups,
+                                                       int out_f32) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= groups) return;
+    const int r = (int)(i % kBlockN);
+    const int64_t jt = i / kBlockN;               // (tile, column group)
+    const int64_t tile = jt / (MG / 4);
+    const int j = (int)(jt % (MG / 4));
+    const int64_t n = (tile % n_tiles) * kBlockN + r;
+    const int64_t m = (tile / n_tiles) * MG + 4 * j;
+    if (n >= N || m >= M) return;
+    const float4 g = __ldcs(G + i), u = __ldcs(U + i);
+    const float gg[4] = {g.x, g.y, g.z, g.w}, uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        if (m + k >= M) break;
+        const float h = gg[k] / (1.0f + __expf(-gg[k])) * uu[k];
+        if (out_f32)
+            reinterpret_cast<float*>(H)[(m + k) * N + n] = h;
+        else
+            reinterpret_cast<uint16_t*>(H)[(m + k) * N + n] = f2bf(h);
+    }
+}
+
+cudaError_t launch_swiglu_blocks(const float* G, const float* U, void* H, int64_t M, int64_t N, int64_t K, int grid,
+                                 int split_k, int out_f32, cudaStream_t s) {
+    const GemmSplit sp = gemm_split(M, N, K, grid, split_k, 1);
+    const int64_t groups = sp.tiles * (sp.MG / 4) * kBlockN;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((groups + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_swiglu_blocks, reinterpret_cast<const float4*>(G),
+                                       reinterpret_cast<const float4*>(U), H, M, N, sp.MG, sp.n_tiles, groups, out_f32);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

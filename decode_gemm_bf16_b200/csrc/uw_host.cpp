@@ -989,12 +989,40 @@ static uw_status swiglu_check(const uw_blob* g, const uw_blob* u, int64_t M, con
     return UW_OK;
 }
 
+// Batches above 128 rows run the SwiGLU in three launches: a paired tile
+// (gate and up accumulators side by side in TMEM) is capped at 128 batch
+// rows, which doubles the rebuild work per product against the
+// single-matrix kernel's 256-row tiles.  The gate and the up launch write
+// their fp32 products into the workspace per tile; a third, elementwise
+// kernel writes H = silu(G) * U.  (Reading G in the up launch's epilogue was
+// slower: one epilogue warp per sub-partition waits on the loads chunk by
+// chunk.)
+static bool swiglu_split(int64_t M) { return M > 128; }
+static size_t swiglu_gate_bytes(const uw_blob* g, int64_t M, const uw_gemm_opts* o) {
+    const GemmSplit sp = gemm_split(M, g->geo.N, g->geo.K, o->grid, o->split_k, 1);
+    return al256((size_t)sp.tiles * (size_t)sp.MG * 128 * 4);
+}
+static size_t swiglu_ws_bytes(const uw_blob* g, int64_t M, const uw_gemm_opts* o) {
+    if (!swiglu_split(M)) return al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 2));
+    return 2 * swiglu_gate_bytes(g, M, o) + al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 1));
+}
+
+static void set_palette_planes(GemmArgs& a, const uw_blob* b) {
+    a.sm = b->sec(UW_SEC_SM);
+    a.idx = b->sec(UW_SEC_IDX);
+    a.vbits = (const uint32_t*)b->sec(UW_SEC_VBITS);
+    a.vpre = (const uint32_t*)b->sec(UW_SEC_VPRE);
+    a.vexp = b->sec(UW_SEC_VEXP);
+    a.vcol = (const uint32_t*)b->sec(UW_SEC_VCOL);
+    a.palette = b->palette;
+}
+
 extern "C" uw_status uw_gemm_swiglu_workspace(const uw_blob* g, const uw_blob* u, int64_t M, const uw_gemm_opts* o,
                                               size_t* bytes) {
     if (!bytes) return UW_ERR_INVALID_ARG;
     uw_status st = swiglu_check(g, u, M, o);
     if (st) return st;
-    *bytes = M ? al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 2)) : 0;
+    *bytes = M ? swiglu_ws_bytes(g, M, o) : 0;
     return UW_OK;
 }
 
@@ -1004,8 +1032,41 @@ extern "C" uw_status uw_gemm_swiglu(const uint16_t* X, int64_t M, const uw_blob*
     if (st) return st;
     if (M == 0) return UW_OK;
     if (!X || !H || !aligned(X, 16) || !aligned(H, 16)) return UW_ERR_INVALID_ARG;
-    const size_t need = al256(gemm_ws_bytes(M, g->geo.N, g->geo.K, o->grid, o->split_k, 2));
+    const size_t need = swiglu_ws_bytes(g, M, o);
     if (!o->workspace || o->workspace_bytes < need || !aligned(o->workspace, 256)) return UW_ERR_WORKSPACE;
+    if (swiglu_split(M)) {
+        const size_t gbytes = swiglu_gate_bytes(g, M, o);
+        float* G = (float*)o->workspace;
+        float* U = (float*)((uint8_t*)o->workspace + gbytes);
+        GemmArgs a;
+        a.src = kSrcPalette;
+        a.X = X;
+        a.M = M;
+        a.N = g->geo.N;
+        a.K = g->geo.K;
+        a.variant = o->variant;
+        a.grid = o->grid;
+        a.split_k = o->split_k;
+        a.stages = o->stages;
+        a.ws = (uint8_t*)o->workspace + 2 * gbytes;
+        a.ws_bytes = o->workspace_bytes - 2 * gbytes;
+        a.static_sm = 1;
+        a.static_s2 = 1;
+        set_palette_planes(a, g);
+        a.Y = H;                // not written: the accumulators go to G, then U
+        a.out_f32 = o->out_f32 ? 1 : 0;
+        a.gate_out = G;
+        cudaError_t e = launch_gemm(a, (cudaStream_t)stream, &st);
+        if (st) return st;
+        if (cuda_ok(e)) return UW_ERR_CUDA;
+        set_palette_planes(a, u);
+        a.gate_out = U;
+        e = launch_gemm(a, (cudaStream_t)stream, &st);
+        if (st) return st;
+        if (cuda_ok(e)) return UW_ERR_CUDA;
+        return cuda_ok(launch_swiglu_blocks(G, U, H, M, g->geo.N, g->geo.K, o->grid, o->split_k, o->out_f32 ? 1 : 0,
+                                            (cudaStream_t)stream));
+    }
     GemmArgs a;
     a.src = kSrcPalette;
     a.pair = 1;

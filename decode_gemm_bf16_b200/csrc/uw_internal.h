@@ -154,6 +154,10 @@ struct GemmArgs {
     // paired call (gate and up, direct palette, SwiGLU epilogue): the up
     // projection's planes; Y = silu(X.Wg^T) * (X.Wu^T)
     int pair = 0;
+    // SwiGLU in three launches: the launch writes its accumulators per tile
+    // (float4 columns of 128 rows, m_tiles * n_tiles * MG * 128 floats) to
+    // gate_out instead of Y; launch_swiglu_blocks then combines two of them
+    float* gate_out = nullptr;
     const uint8_t* sm2 = nullptr;
     const uint8_t* idx2 = nullptr;
     const uint32_t* vbits2 = nullptr;
@@ -177,6 +181,10 @@ size_t gemm_ws_bytes(int64_t M, int64_t N, int64_t K, int grid, int split_k, int
 // UW_VARIANT_AUTO batch 1 on a projection with few 128-row tiles and no
 // decoder beside) go to the CUDA-core GEMV instead.
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st);
+// H = silu(G) * U from two tile-block arrays written with gate_out (same
+// M, N, K, grid and split_k as the launches that wrote them)
+cudaError_t launch_swiglu_blocks(const float* G, const float* U, void* H, int64_t M, int64_t N, int64_t K, int grid,
+                                 int split_k, int out_f32, cudaStream_t s);
 bool gemv_serves(const GemmArgs& a);
 constexpr int kGemvMaxM = 1;   // batches the GEMV kernel supports
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, uw_status* st);

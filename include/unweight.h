@@ -332,7 +332,13 @@ uw_status uw_gemm_sequence(const uw_seq_item* items, int n, int64_t M, int out_f
  *   opts: pipeline UW_PIPE_DIRECT_PALETTE (others: UW_ERR_UNSUPPORTED),
  *     variant UW_VARIANT_AUTO or UW_VARIANT_TENSOR, sm_dec 0; grid, split_k,
  *     stages, out_f32 and the workspace as in uw_gemm.  Batch tiles are at
- *     most 128 rows (two accumulators share TMEM with the rebuilt tiles). */
+ *     most 128 rows (two accumulators share TMEM with the rebuilt tiles).
+ * Above 128 batch rows the paired tile would need twice the rebuild work of
+ * a 256-row single-matrix tile, so H is computed in three launches on the
+ * same stream instead: the gate and the up projection, each with 256-row
+ * tiles, into float32 blocks in the workspace, then an elementwise kernel
+ * writing silu(G) * U.  The workspace size (uw_gemm_swiglu_workspace) covers
+ * either form. */
 uw_status uw_gemm_swiglu_workspace(const uw_blob* gate, const uw_blob* up, int64_t M, const uw_gemm_opts* opts,
                                    size_t* bytes);
 
