@@ -23,22 +23,20 @@
 namespace uw {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kMaxWarps = 28;                  // warps of a standalone decoder CTA (one CTA per SM)
 constexpr int kBesideWarps = 4;                // decoder CTAs that share SMs with the GEMM
 constexpr int kTaskElems = 32 * kSeg;          // 8192 weights per warp task
 constexpr int kStreamCapW = 768;               // per-warp stream staging, words (3 KB)
 constexpr int kStageSmem = 32 * 32 * 4;        // per-warp decoded nibbles
-// Every decoder stages each task's stream bits in shared memory (3 CTAs per
-// SM): its table walk then refills from shared memory instead of L1 (gate
-// shape: exponent 47.6 -> 42.7 us, full 73.8 -> 66.6 us).  The 4-warp CTAs
-// that run beside a GEMM keep the stream in L1 (their shared memory is
-// fixed).
-template <int MODE, int WARPS>
-constexpr bool kStaged = WARPS == kWarps;
-template <int MODE, int WARPS>
-constexpr size_t kWarpSmem = kStageSmem + (kStaged<MODE, WARPS> ? kStreamCapW * 4 : 0);
-template <int MODE, int WARPS>
-constexpr size_t kDecSmem = kLutSize * 4 + WARPS * kWarpSmem<MODE, WARPS>;
+// The standalone decoders (WARPS == 0: the warp count is the launch's) stage
+// each task's stream bits in shared memory: the table walk then refills from
+// shared memory instead of L1 (gate shape: exponent 47.6 -> 42.7 us, full
+// 73.8 -> 66.6 us).  The 4-warp CTAs that run beside a GEMM keep the stream
+// in L1 (their shared memory is fixed).
+template <int WARPS>
+constexpr bool kStaged = WARPS == 0;
+constexpr size_t kWarpSmemStaged = kStageSmem + kStreamCapW * 4;
+static_assert(kLutSize * 4 + kMaxWarps * kWarpSmemStaged <= 227 * 1024, "decoder smem");
 static_assert(kDecodeBesideSmem == kLutSize * 4 + kBesideWarps * kStageSmem, "beside decoder smem");
 
 struct DecodeParams {
@@ -72,9 +70,9 @@ struct DecodeParams {
 // symbols from the 12-bit window buf >> 52; consuming them is a 64-bit shift.
 // The prefetched word `nxt` is the next refill.  Word reads are clamped to the
 // stream, so a corrupt stream cannot read outside it; an undecodable window
-// still advances (12 bits) and is reported once per segment.  The second read
-// of a pair may decode past the segment's last symbol (the bits of the next
-// segment or the padding); nothing is stored for it.
+// still advances (12 bits) and is reported once per segment.  The last read
+// may decode past the segment's last symbol (the bits of the next segment or
+// the padding); those symbols are never stored.
 template <bool SMEM>
 __device__ __forceinline__ uint32_t ldw(const uint32_t* sp, int64_t i) {
     if (SMEM) return sp[i];
@@ -102,33 +100,45 @@ __device__ __forceinline__ void decode_bits(const DecodeParams& p, const uint32_
     uint32_t acc = 0, accn = 0, flags = 0;
     int k = 0, kr = rot;
     const int words = nsym >> 3;
-    while (k < words) {
+    auto refill = [&]() {
         if (nv < 32) {
             buf |= (uint64_t)nxt << (32 - nv);       // shift 1..24
             nv += 32;
             nxt = ldw<SMEM>(sp, min(idx, last));
             idx++;
         }
-#pragma unroll
-        for (int t = 0; t < 2; t++) {
-            const uint32_t ent = lut[(uint32_t)(buf >> 52)];
-            flags |= ent;
-            const uint32_t nb = lut_bits(ent);
-            buf <<= nb;
-            nv -= (int)nb;
-            const uint32_t sy = ent >> kLutSymShift;
-            const uint32_t accn2 = accn + lut_nibble_bits(ent);
-            acc |= sy << accn;
-            if (accn2 >= 32u) {
-                if (k < words) row[kr] = acc;
-                kr = (kr + 1) & 31;
-                k++;
-                acc = sy >> (32u - accn);     // accn >= 12 here, so the shift is in [1, 20]
-                accn = accn2 - 32u;
-            } else {
-                accn = accn2;
-            }
-        }
+    };
+    // One table read.  A completed word is stored without a branch (lanes
+    // complete words at different reads; selects keep the warp converged).
+    // A read adds at most 20 bits to fewer than 32, so it completes at most
+    // one word.
+    auto step = [&]() {
+        const uint32_t ent = lut[(uint32_t)(buf >> 52)];
+        flags |= ent;
+        const uint32_t nb = lut_bits(ent);
+        buf <<= nb;
+        nv -= (int)nb;
+        const uint32_t sy = ent >> kLutSymShift;
+        const uint32_t accn2 = accn + lut_nibble_bits(ent);
+        acc |= sy << accn;
+        const uint32_t fl = accn2 >> 5;                        // a word is complete
+        if (fl) row[kr] = acc;
+        const uint32_t carry = sy >> ((32u - accn) & 31u);   // used when fl: accn >= 12, shift in [1, 20]
+        acc = fl ? carry : acc;
+        accn = accn2 & 31u;
+        kr = (kr + (int)fl) & 31;
+        k += (int)fl;
+    };
+    // Pairs of reads while at least two words are missing (both stores stay
+    // inside the segment), then single reads up to the last word.
+    while (k < words - 1) {
+        refill();
+        step();
+        step();
+    }
+    while (k < words) {
+        refill();
+        step();
     }
     if (flags & kLutInvalid) raise_status(UW_ERR_DEVICE);
 }
@@ -166,15 +176,16 @@ __device__ __forceinline__ Staging stage_stream(const DecodeParams& p, uint64_t 
 }
 
 template <int MODE, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, kStaged<MODE, WARPS> ? 3 : 4) k_decode(const DecodeParams p) {
-    constexpr bool STAGED = kStaged<MODE, WARPS>;
+__global__ void __launch_bounds__(WARPS ? WARPS * 32 : kMaxWarps * 32, WARPS ? 4 : 1) k_decode(const DecodeParams p) {
+    constexpr bool STAGED = kStaged<WARPS>;
+    const int nwarps = WARPS ? WARPS : (int)(blockDim.x >> 5);
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     uint32_t* stage = smem + kLutSize;
     {
         const uint4* src = reinterpret_cast<const uint4*>(p.lut);
         uint4* dst = reinterpret_cast<uint4*>(lut);
-        for (int i = threadIdx.x; i < kLutSize / 4; i += WARPS * 32) dst[i] = __ldg(&src[i]);
+        for (int i = threadIdx.x; i < kLutSize / 4; i += nwarps * 32) dst[i] = __ldg(&src[i]);
     }
     __syncthreads();
     // programmatic stream serialization: the table load above reads only the
@@ -182,17 +193,17 @@ __global__ void __launch_bounds__(WARPS * 32, kStaged<MODE, WARPS> ? 3 : 4) k_de
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* st = stage + warp * (kWarpSmem<MODE, WARPS> / 4);
+    uint32_t* st = stage + warp * ((STAGED ? kWarpSmemStaged : kStageSmem) / 4);
     uint32_t* sbuf = st + 32 * 32;
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
     const uint32_t P0 = p.pal[0], P1 = p.pal[1], P2 = p.pal[2], P3 = p.pal[3];
-    const int64_t stride = (int64_t)gridDim.x * WARPS;
+    const int64_t stride = (int64_t)gridDim.x * nwarps;
 
     // Staged software pipeline per warp: the stream bits of the
     // next task are copied into shared memory (asynchronously) while this
     // task's outputs are written; the next task's segment offsets load during
     // this task's decode.
-    int64_t task = (int64_t)blockIdx.x * WARPS + warp;
+    int64_t task = (int64_t)blockIdx.x * nwarps + warp;
     uint64_t bitpos = 0;
     Staging g = {0, 0, false};
     if (STAGED && task < ntasks) {
@@ -629,8 +640,6 @@ cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M,
     return cudaGetLastError();
 }
 
-int decode_ctas_per_sm() { return 4; }
-
 static DecodeParams decode_params(const uw_blob* b, void* out) {
     DecodeParams p;
     p.stream = (const uint32_t*)b->sec(UW_SEC_STREAM);
@@ -658,19 +667,20 @@ static DecodeParams decode_params(const uw_blob* b, void* out) {
     return p;
 }
 
+// WARPS == 0: `warps` warps a CTA (staged stream); otherwise WARPS.
 template <int WARPS>
-static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid, cudaStream_t s) {
+static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid, int warps, cudaStream_t s) {
     void (*kern)(const DecodeParams) = mode == kDecodeFull       ? k_decode<kDecodeFull, WARPS>
                                        : mode == kDecodeExponent ? k_decode<kDecodeExponent, WARPS>
                                                                  : k_decode<kDecodeTranscode, WARPS>;
-    const size_t smem = mode == kDecodeFull       ? kDecSmem<kDecodeFull, WARPS>
-                        : mode == kDecodeExponent ? kDecSmem<kDecodeExponent, WARPS>
-                                                  : kDecSmem<kDecodeTranscode, WARPS>;
+    const size_t per_warp = kStaged<WARPS> ? kWarpSmemStaged : kStageSmem;
+    const size_t smem = (size_t)kLutSize * 4 + (size_t)warps * per_warp;
+    const size_t smem_max = (size_t)kLutSize * 4 + (size_t)(WARPS ? WARPS : kMaxWarps) * per_warp;
     static bool attr_set[3][64] = {{false}};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[mode][dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
         // SMs running decoder CTAs keep the largest shared-memory carveout, so
         // a GEMM CTA can still be placed beside them
         if (e == cudaSuccess)
@@ -680,7 +690,7 @@ static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid,
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(WARPS * 32);
+    cfg.blockDim = dim3(warps * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -693,14 +703,32 @@ static cudaError_t launch_decode_impl(const DecodeParams& p, int mode, int grid,
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s) {
+// One CTA per SM.  A warp's tasks take about the same time, so the launch
+// lasts as many task times as the busiest warp has tasks: the fewest rounds
+// R that kMaxWarps warps per SM allow, then the fewest warps that still
+// finish in R rounds (gate shape: 7168 tasks = 2 rounds of 25 warps on 148
+// SMs; CTAs of 8 warps, three per SM, left 64 tasks for a third round on 8
+// SMs).  `sms` > 0 overrides the SM count.
+void decode_grid(int64_t ntasks, int sms, int* grid, int* warps) {
+    if (sms <= 0) sms = num_sms();
+    if (ntasks < 1) ntasks = 1;
+    const int64_t per_round = (int64_t)sms * kMaxWarps;
+    const int64_t rounds = (ntasks + per_round - 1) / per_round;
+    int64_t w = (ntasks + (int64_t)sms * rounds - 1) / ((int64_t)sms * rounds);
+    if (w > kMaxWarps) w = kMaxWarps;
+    if (w < 1) w = 1;
+    int64_t g = (ntasks + w * rounds - 1) / (w * rounds);
+    if (g > sms) g = sms;
+    *grid = (int)g;
+    *warps = (int)w;
+}
+
+cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int sms, cudaStream_t s) {
     DecodeParams p = decode_params(b, out);
     const int64_t ntasks = (p.n + kTaskElems - 1) / kTaskElems;
-    const int64_t need = (ntasks + kWarps - 1) / kWarps;
-    int grid = grid_ctas > 0 ? grid_ctas : num_sms() * (mode == kDecodeTranscode ? 3 : decode_ctas_per_sm());
-    if (grid > need) grid = (int)need;
-    if (grid < 1) grid = 1;
-    return launch_decode_impl<kWarps>(p, mode, grid, s);
+    int grid = 0, warps = 0;
+    decode_grid(ntasks, sms, &grid, &warps);
+    return launch_decode_impl<0>(p, mode, grid, warps, s);
 }
 
 cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas, unsigned long long* band_ready,
@@ -712,7 +740,7 @@ cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas
     const int64_t need = (ntasks + kBesideWarps - 1) / kBesideWarps;
     int grid = ctas > need ? (int)need : ctas;
     if (grid < 1) grid = 1;
-    return launch_decode_impl<kBesideWarps>(p, mode, grid, s);
+    return launch_decode_impl<kBesideWarps>(p, mode, grid, kBesideWarps, s);
 }
 
 int decode_status_take() { return unit_status_take(); }

@@ -107,13 +107,16 @@ cudaError_t launch_encode(const uint16_t* W, const Geometry& g, const uint8_t in
 
 // ---- decoders (uw_decode.cu)
 enum DecodeMode { kDecodeFull = 0, kDecodeExponent = 1, kDecodeTranscode = 2 };
-cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int grid_ctas, cudaStream_t s);
+// Standalone decoder; `sms` > 0 stands in for the device's SM count.
+cudaError_t launch_decode(const uw_blob* b, int mode, void* out, int sms, cudaStream_t s);
 // Decoder that runs beside the GEMM: `ctas` CTAs of 4 warps, each finished
 // 8192-weight task counted in band_ready[task / (K/64)] under call tag `epoch`.
 cudaError_t launch_decode_beside(const uw_blob* b, int mode, void* out, int ctas, unsigned long long* band_ready,
                                  unsigned long long epoch, cudaStream_t s);
 constexpr int kDecodeBesideSmem = (1 << 12) * 4 + 4 * 32 * 32 * 4;   // LUT + 4 warps of staging
-int decode_ctas_per_sm();
+// Standalone decoder launch shape for `ntasks` warp tasks: CTAs and warps a
+// CTA (one CTA per SM, every warp the same number of tasks at most).
+void decode_grid(int64_t ntasks, int sms, int* grid, int* warps);
 // Fused Huffman-decode GEMV/small-batch product (no decoded plane in HBM):
 // Y[M,N] = X[M,K] . W^T straight from the Huffman form, M <= kFusedMaxM per
 // launch, K a multiple of 256.  Workspace: fused_ws_bytes.
