@@ -96,6 +96,7 @@ struct GemmParams {
     int acc_w;            // accumulator columns per tile: nh * MG (gate in [0, MG), up in [MG, 2 MG))
     uint32_t total_iters;
     uint32_t stage_bytes, off_a, off_b, tx_bytes;
+    uint32_t tx_x;        // rebuilding sources: the stage's X bytes (on their own barrier; tx_bytes = the planes)
     uint32_t tmem_cols;   // TMEM columns allocated (power of two)
     uint32_t a_col0;      // first TMEM column of the rebuilt-A stages (nh * KB/2 columns each)
     PlaneSet ps[2];
@@ -518,7 +519,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
     uint64_t* recon_bar = full_bar + kMaxStages;
     uint64_t* empty_bar = recon_bar + kMaxStages;
-    uint64_t* accf_bar = empty_bar + kMaxStages;
+    // rebuilding sources: a stage's X tile lands on its own barrier (the MMA
+    // waits for it), so the rebuild waits only for the weight planes
+    uint64_t* xfull_bar = empty_bar + kMaxStages;
+    uint64_t* accf_bar = xfull_bar + kMaxStages;
     uint64_t* acce_bar = accf_bar + 1;
     uint64_t* final_bar = acce_bar + 1;
     uint64_t* fin_bar = final_bar + 1;   // finisher: contributors' partials landed in the ring
@@ -536,6 +540,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&recon_bar[s]), kReconGroupWarps);
             mbar_init(smem_u32(&empty_bar[s]), 1);
+            mbar_init(smem_u32(&xfull_bar[s]), 1);
         }
         mbar_init(smem_u32(accf_bar), 1);
         mbar_init(smem_u32(acce_bar), kEpiWarps);
@@ -634,9 +639,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                         if (leader) {
                             const uint32_t st = smem_base + s * p.stage_bytes;
                             const uint32_t fb = smem_u32(&full_bar[s]);
+                            const uint32_t xb = smem_u32(&xfull_bar[s]);
+                            mbar_arrive_expect_tx(xb, p.tx_x);
 #pragma unroll
                             for (int hb = 0; hb < kHalves; hb++)
-                                tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, fb);
+                                tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, xb);
                             if (SRC == kSrcExponent)
                                 tma_load_2d(st + p.ps[0].off_s2, &tm_s2, kt * KB, n_tile * kBlockN, fb);
                             else if (!p.static_s2)
@@ -649,9 +656,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     if (!leader) continue;
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
+                    const uint32_t xb = kRecon ? smem_u32(&xfull_bar[s]) : fb;
+                    if (kRecon) mbar_arrive_expect_tx(xb, p.tx_x);
 #pragma unroll
                     for (int hb = 0; hb < kHalves; hb++)
-                        tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, fb);
+                        tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, xb);
                     if (SRC == kSrcDense) {
 #pragma unroll
                         for (int hb = 0; hb < kHalves; hb++)
@@ -674,8 +683,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             }
             if (!ok) {
                 // drain: every load already issued must land before the CTA exits
-                for (int64_t qq = q - S < 0 ? 0 : q - S; qq < q; qq++)
+                for (int64_t qq = q - S < 0 ? 0 : q - S; qq < q; qq++) {
                     mbar_wait(smem_u32(&full_bar[qq % S]), (uint32_t)((qq / S) & 1), p.timeout_ns, nullptr);
+                    if (kRecon) mbar_wait(smem_u32(&xfull_bar[qq % S]), (uint32_t)((qq / S) & 1), p.timeout_ns, nullptr);
+                }
             }
         }
     } else if (warp == kMmaWarp) {
@@ -698,6 +709,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     const int s = rp.s;
                     const uint32_t wb = kRecon ? smem_u32(&recon_bar[s]) : smem_u32(&full_bar[s]);
                     if (!mbar_wait(wb, rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
+                    if (kRecon && !mbar_wait(smem_u32(&xfull_bar[s]), rp.ph, p.timeout_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t st = smem_base + s * p.stage_bytes;
                     if (!leader) continue;
@@ -1124,7 +1136,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, uw_status* st) {
     const uint32_t b_bytes = (uint32_t)p.MG * 128 * halves;
     auto al1k = [](uint32_t x) { return (x + 1023u) & ~1023u; };
     uint32_t off = 0;
-    p.tx_bytes = b_bytes;
+    p.tx_bytes = a.src == kSrcDense ? b_bytes : 0;
+    p.tx_x = b_bytes;
     if (a.src == kSrcDense) {
         p.off_a = 0;
         p.off_b = kTileA64 * halves;
