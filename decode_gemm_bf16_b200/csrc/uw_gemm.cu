@@ -658,14 +658,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                     mbar_arrive_expect_tx(fb, p.tx_bytes);
                     const uint32_t xb = kRecon ? smem_u32(&xfull_bar[s]) : fb;
                     if (kRecon) mbar_arrive_expect_tx(xb, p.tx_x);
-#pragma unroll
-                    for (int hb = 0; hb < kHalves; hb++)
-                        tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, xb);
                     if (SRC == kSrcDense) {
 #pragma unroll
                         for (int hb = 0; hb < kHalves; hb++)
                             tma_load_2d(st + p.off_a + hb * kTileA64, &tm_a, kt * KB + hb * kBoxK, n_tile * kBlockN, fb);
                     } else {
+                        // the weight planes first: the rebuild waits for them
 #pragma unroll
                         for (int h = 0; h < NH; h++) {
                             const PlaneSet& ps = p.ps[h];
@@ -679,6 +677,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                             }
                         }
                     }
+#pragma unroll
+                    for (int hb = 0; hb < kHalves; hb++)
+                        tma_load_2d(st + p.off_b + hb * p.MG * 128, &tm_x, kt * KB + hb * kBoxK, m_tile * p.MG, xb);
                 }
             }
             if (!ok) {
