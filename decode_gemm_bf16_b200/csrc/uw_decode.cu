@@ -413,19 +413,24 @@ __device__ __forceinline__ void fused_flush(const FusedParams& p, int64_t task, 
     }
 }
 
-// Four CTAs of 8 warps per SM (64 registers a thread at batch 1-2): the
-// decode chains are latency-bound and want every warp the SM can hold; the
+// Batch 1-2 (STAGED): the decoders' launch shape -- one CTA per SM with
+// as many warps as make every warp's task count equal, each warp's stream
+// words staged in shared memory one task ahead.  Batch 4-16: two CTAs of 8
+// warps per SM (more registers a thread), the stream read through L1.  The
 // activations are read through L1 (all lanes of a half warp read one
-// contiguous KB), so shared memory holds only the table and the nibbles.
-template <int MB>
-__global__ void __launch_bounds__(kFusedWarps * 32, MB <= 2 ? 4 : 2) k_fused_huffman(const FusedParams p) {
+// contiguous KB), so shared memory holds only the table, the nibbles and the
+// staged stream.
+template <int MB, bool STAGED>
+__global__ void __launch_bounds__(STAGED ? kMaxWarps * 32 : kFusedWarps * 32, STAGED ? 1 : 2)
+    k_fused_huffman(const FusedParams p) {
+    const int nwarps = STAGED ? (int)(blockDim.x >> 5) : kFusedWarps;
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     uint32_t* stage = smem + kLutSize;
     {
         const uint4* src = reinterpret_cast<const uint4*>(p.d.lut);
         uint4* dst = reinterpret_cast<uint4*>(lut);
-        for (int i = threadIdx.x; i < kLutSize / 4; i += kFusedWarps * 32) dst[i] = __ldg(&src[i]);
+        for (int i = threadIdx.x; i < kLutSize / 4; i += nwarps * 32) dst[i] = __ldg(&src[i]);
     }
     // programmatic stream serialization: the table comes from the committed
     // blob; activations, pieces and outputs after the previous kernel
@@ -433,12 +438,21 @@ __global__ void __launch_bounds__(kFusedWarps * 32, MB <= 2 ? 4 : 2) k_fused_huf
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* st = stage + warp * (32 * 32);
+    uint32_t* st = stage + warp * ((STAGED ? kWarpSmemStaged : kStageSmem) / 4);
+    uint32_t* sbuf = st + 32 * 32;
     const uint32_t P0 = p.d.pal[0], P1 = p.d.pal[1], P2 = p.d.pal[2], P3 = p.d.pal[3];
     const int M = p.M;
     const int half = lane >> 4, hl = lane & 15;
-    for (int64_t task = (int64_t)blockIdx.x * kFusedWarps + warp; task < p.ntasks;
-         task += (int64_t)gridDim.x * kFusedWarps) {
+    const int64_t stride = (int64_t)gridDim.x * nwarps;
+    int64_t task = (int64_t)blockIdx.x * nwarps + warp;
+    uint64_t bitpos = 0;
+    Staging g = {0, 0, false};
+    if (STAGED && task < p.ntasks) {
+        bitpos = segment_bitpos(p.d, task * 32 + lane);
+        const uint64_t endb = lane == 31 ? segment_bitpos(p.d, task * 32 + 32) : 0;
+        g = stage_stream(p.d, __shfl_sync(0xFFFFFFFFu, bitpos, 0), __shfl_sync(0xFFFFFFFFu, endb, 31), sbuf, lane);
+    }
+    for (; task < p.ntasks; task += stride) {
         const int64_t base = task * kTaskElems, seg0 = task * 32;
         {
             // the task's sign+mantissa bytes, read in phase 2, into L2 now
@@ -448,15 +462,32 @@ __global__ void __launch_bounds__(kFusedWarps * 32, MB <= 2 ? 4 : 2) k_fused_huf
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(p.d.sm + off + 128));
             }
         }
+        const int64_t next = task + stride;
+        uint64_t nbit = 0, nend = 0;
+        if (STAGED && next < p.ntasks) {
+            nbit = segment_bitpos(p.d, next * 32 + lane);
+            if (lane == 31) nend = segment_bitpos(p.d, next * 32 + 32);
+        }
+        if (STAGED) {
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            __syncwarp();
+        }
         // ---- phase 1: one segment per lane
         {
             const int64_t seg = seg0 + lane;
             if (seg < p.d.nseg) {
-                const uint64_t bitpos = __ldg(&p.d.chunk_off[seg >> 4]) + __ldg(&p.d.seg_rel[seg]);
-                decode_bits<false>(p.d, lut, p.d.stream, p.d.nwords - 1, bitpos, kSeg, st + lane * 32, lane);
+                if (STAGED && g.staged)
+                    decode_bits<true>(p.d, lut, sbuf, g.nw - 1, bitpos - (uint64_t)g.w0a * 32u, kSeg, st + lane * 32, lane);
+                else {
+                    const uint64_t bp = STAGED ? bitpos : __ldg(&p.d.chunk_off[seg >> 4]) + __ldg(&p.d.seg_rel[seg]);
+                    decode_bits<false>(p.d, lut, p.d.stream, p.d.nwords - 1, bp, kSeg, st + lane * 32, lane);
+                }
             }
         }
         __syncwarp();
+        if (STAGED && next < p.ntasks)
+            g = stage_stream(p.d, __shfl_sync(0xFFFFFFFFu, nbit, 0), __shfl_sync(0xFFFFFFFFu, nend, 31), sbuf, lane);
+        if (STAGED) bitpos = nbit;
         // ---- phase 2: two segments per step, 16 weights a lane
         float racc[MB];
 #pragma unroll
@@ -606,28 +637,38 @@ cudaError_t launch_fused_huffman(const uw_blob* b, const uint16_t* X, int64_t M,
     p.epoch = gemm_next_epoch();
     p.Y = Y;
     p.out_f32 = out_f32;
-    const size_t smem = (size_t)kLutSize * 4 + kFusedWarps * 32 * 32 * 4;
     const int mb = M == 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+    const bool staged = mb <= 2;
     typedef void (*Kern)(const FusedParams);
-    Kern kern = mb == 1 ? k_fused_huffman<1> : mb == 2 ? k_fused_huffman<2> : mb == 4 ? k_fused_huffman<4>
-              : mb == 8 ? k_fused_huffman<8> : k_fused_huffman<16>;
-    static bool carve_set[5][64] = {};
+    Kern kern = mb == 1 ? k_fused_huffman<1, true> : mb == 2 ? k_fused_huffman<2, true> : mb == 4 ? k_fused_huffman<4, false>
+              : mb == 8 ? k_fused_huffman<8, false> : k_fused_huffman<16, false>;
+    // batch 1-2: one CTA per SM, warps as for the decoders; else two CTAs of
+    // 8 warps per SM (every task resident at once when possible, otherwise
+    // CTAs loop)
+    int grid = 0, warps = kFusedWarps;
+    if (staged) {
+        decode_grid(p.ntasks, 0, &grid, &warps);
+    } else {
+        int64_t g = (p.ntasks + kFusedWarps - 1) / kFusedWarps;
+        if (g > (int64_t)num_sms() * 2) g = (int64_t)num_sms() * 2;
+        grid = (int)g;
+    }
+    const size_t smem = (size_t)kLutSize * 4 + (size_t)warps * (staged ? kWarpSmemStaged : kStageSmem);
+    const size_t smem_max = staged ? (size_t)kLutSize * 4 + (size_t)kMaxWarps * kWarpSmemStaged : smem;
+    static bool attr_set[5][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     const int mi = mb == 1 ? 0 : mb == 2 ? 1 : mb == 4 ? 2 : mb == 8 ? 3 : 4;
-    if (!carve_set[mi][dev & 63]) {
-        // four CTAs of 48 KB per SM need the largest shared-memory carveout
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (!attr_set[mi][dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+        // the largest shared-memory carveout: the CTAs above fill it
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
-        carve_set[mi][dev & 63] = true;
+        attr_set[mi][dev & 63] = true;
     }
-    // every task is resident at once when possible; otherwise CTAs loop
-    const int per_sm = mb <= 2 ? 4 : 2;
-    int64_t grid = (p.ntasks + kFusedWarps - 1) / kFusedWarps;
-    if (grid > (int64_t)num_sms() * per_sm) grid = (int64_t)num_sms() * per_sm;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kFusedWarps * 32);
+    cfg.blockDim = dim3((unsigned)warps * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
