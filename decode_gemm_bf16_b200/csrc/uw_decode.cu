@@ -342,8 +342,9 @@ __global__ void __launch_bounds__(WARPS ? WARPS * 32 : kMaxWarps * 32, WARPS ? 4
 // lane): sign+mantissa bytes in coalesced 256-byte reads, exponents from the
 // palette or the verbatim store, BF16 rebuilt in registers, fused
 // multiply-adds with the activations (consecutive 64-byte blocks per lane,
-// conflict-free), then a fixed xor tree over the 16 lanes gives each
-// segment's sum and the segment sums of a row are added in order.  A row
+// conflict-free); each lane sums its products over the steps that stay on
+// the same rows, then a fixed xor tree over the 16 lanes gives the sums and
+// they are added to their rows in order.  A row
 // whose segments span several tasks is stored in pieces, and the last task of
 // the row to arrive (a tagged counter per row) adds the pieces in order: the
 // result depends on the shape only, never on the launch.
@@ -500,6 +501,11 @@ __global__ void __launch_bounds__(STAGED ? kMaxWarps * 32 : kFusedWarps * 32, ST
         int64_t rw[2] = {row0, row0};
         int jw[2] = {jr0, jr0 + 1};
         if (jw[1] >= p.S) { jw[1] -= p.S; rw[1]++; }
+        // lane partial sums of the steps since the halves' rows last changed
+        float lacc[MB];
+#pragma unroll
+        for (int m = 0; m < MB; m++) lacc[m] = 0.f;
+        int it0 = 0;   // first step of the current group
 #pragma unroll 1
         for (int it = 0; it < 16; it++) {
             const int j = 2 * it + half;               // segment of the task
@@ -559,34 +565,9 @@ __global__ void __launch_bounds__(STAGED ? kMaxWarps * 32 : kFusedWarps * 32, ST
                     }
                 }
             }
-            // segment sums: a fixed xor tree over each half warp, then both
-            // halves' sums to every lane
-            float s_lo[MB], s_hi[MB];
 #pragma unroll
-            for (int m = 0; m < MB; m++) {
-                float v = pacc[m].x + pacc[m].y;
-                v += __shfl_xor_sync(0xFFFFFFFFu, v, 8);
-                v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-                v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-                v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-                s_lo[m] = __shfl_sync(0xFFFFFFFFu, v, 0);
-                s_hi[m] = __shfl_sync(0xFFFFFFFFu, v, 16);
-            }
-            // rows in order (warp-uniform)
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const int64_t gsh = seg0 + 2 * it + h;
-                if (gsh >= p.d.nseg) break;
-                const int64_t row = rw[h];
-                if (row != rcur) {
-                    if (rcur >= 0) fused_flush<MB>(p, task, rcur, racc, lane);
-                    rcur = row;
-#pragma unroll
-                    for (int m = 0; m < MB; m++) racc[m] = 0.f;
-                }
-#pragma unroll
-                for (int m = 0; m < MB; m++) racc[m] += h ? s_hi[m] : s_lo[m];
-            }
+            for (int m = 0; m < MB; m++) lacc[m] += pacc[m].x + pacc[m].y;
+            const int64_t r0 = rw[0], r1 = rw[1];
 #pragma unroll
             for (int h = 0; h < 2; h++) {
                 jw[h] += 2;
@@ -594,6 +575,38 @@ __global__ void __launch_bounds__(STAGED ? kMaxWarps * 32 : kFusedWarps * 32, ST
                     jw[h] -= p.S;
                     rw[h]++;
                 }
+            }
+            // at the end of the task or where a half's row changes: the
+            // group's sums (a fixed xor tree over each half warp, then both
+            // halves' sums to every lane), added to the rows in order
+            // (warp-uniform)
+            if (it == 15 || seg0 + 2 * (it + 1) >= p.d.nseg || rw[0] != r0 || rw[1] != r1) {
+                float s_lo[MB], s_hi[MB];
+#pragma unroll
+                for (int m = 0; m < MB; m++) {
+                    float v = lacc[m];
+                    v += __shfl_xor_sync(0xFFFFFFFFu, v, 8);
+                    v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+                    v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+                    v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+                    s_lo[m] = __shfl_sync(0xFFFFFFFFu, v, 0);
+                    s_hi[m] = __shfl_sync(0xFFFFFFFFu, v, 16);
+                    lacc[m] = 0.f;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    if (seg0 + 2 * it0 + h >= p.d.nseg) break;   // no segment of this half in the group
+                    const int64_t row = h ? r1 : r0;
+                    if (row != rcur) {
+                        if (rcur >= 0) fused_flush<MB>(p, task, rcur, racc, lane);
+                        rcur = row;
+#pragma unroll
+                        for (int m = 0; m < MB; m++) racc[m] = 0.f;
+                    }
+#pragma unroll
+                    for (int m = 0; m < MB; m++) racc[m] += h ? s_hi[m] : s_lo[m];
+                }
+                it0 = it + 1;
             }
         }
         if (rcur >= 0) fused_flush<MB>(p, task, rcur, racc, lane);
