@@ -440,15 +440,17 @@ def test_fused_huffman_matches_oracle(shape, M):
     assert uw.uw_last_device_status() == 0
 
 
-def test_fused_huffman_graph_replays():
+@pytest.mark.parametrize("M", [1, 4])
+def test_fused_huffman_graph_replays(M):
     """Captured once and replayed: the per-call tag is reused, so the last
-    warp of each row group resets its counter; every replay must match."""
+    warp of each row group resets its counter; every replay must match
+    (batch 1: one CTA per SM with staged stream words; batch 4: 8-warp CTAs)."""
     W, blob = _fcase("200x1024")
-    X = S.activations(4, 1024, seed=2100)
+    X = S.activations(M, 1024, seed=2100)
     R = O.gemm(X, W, "f32")
     Xd = dev16(X)
-    Y = torch.empty(4, 200, dtype=torch.float32, device="cuda")
-    ws = torch.zeros(uw.uw_gemm_workspace(blob, 4, "fused_huffman"), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(M, 200, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(uw.uw_gemm_workspace(blob, M, "fused_huffman"), dtype=torch.uint8, device="cuda")
     uw.uw_gemm(Xd, blob, "fused_huffman", out=Y, out_f32=True, ws=ws)
     torch.cuda.synchronize()
     first = _f32(Y)
@@ -477,7 +479,7 @@ def test_fused_huffman_rejects_unsupported():
     assert ei.value.status == 4
 
 
-@pytest.mark.parametrize("M", [1, 16, 64])
+@pytest.mark.parametrize("M", [1, 2, 16, 64])
 def test_fused_huffman_full_size_gate(gate_case, M):
     W, blob = gate_case
     X = S.activations(M, 4096, seed=2200 + M)
