@@ -585,16 +585,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             // Weight planes read from the committed blob (the sign+mantissa
             // plane and verbatim flags of every rebuilding pipeline, the index
             // plane of the direct-palette one) are not written by any kernel:
-            // the first ring's worth of those tiles is requested before the
-            // wait on the previous kernel, so it streams in during that
-            // kernel's tail; activations and decoded planes follow the wait.
+            // up to four stages of those tiles are requested before the wait
+            // on the previous kernel, so they stream in during that kernel's
+            // tail; activations and decoded planes follow the wait.  (More
+            // stages compete with the previous kernel's last CTAs for HBM:
+            // the down projection at batch 1-8 takes 26.8 us with a whole
+            // ring requested early, 26.4 us with four stages; two stages are
+            // 1-4 % slower.)
             int npre = 0;
+            const int npre_max = S < 4 ? S : 4;
             if (kRecon && p.static_sm && !p.band_ready) {
                 SegWalker wk0(blockIdx.x, p);
                 Segment sg0;
-                while (npre < S && wk0.next(sg0)) {
+                while (npre < npre_max && wk0.next(sg0)) {
                     const int n_tile = (int)(sg0.tile % p.n_tiles);
-                    for (int kt = sg0.kt0; kt < sg0.kt1 && npre < S; kt++, npre++) {
+                    for (int kt = sg0.kt0; kt < sg0.kt1 && npre < npre_max; kt++, npre++) {
                         if (!leader) continue;
                         const uint32_t st = smem_base + npre * p.stage_bytes;
                         const uint32_t fb = smem_u32(&full_bar[npre]);
